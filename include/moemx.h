@@ -1,0 +1,208 @@
+/*
+ * moemx.h - C ABI of libmoemx: the expert MLP of one mixture-of-experts layer on one
+ * NVIDIA B200 (sm_100a), forward and backward, with MXFP8 or BF16 GEMM operands.
+ *
+ * What the library computes is the chain the pages describe as
+ *   GroupedLinear(gate_up) -> ScaledSwiGLU -> GroupedLinear(down)
+ * (ai4snews, paragraph 3; sitech.ge, "Memory and quantization overhead"), with the tokens
+ * of every expert gathered by the per-expert counts ``split_sizes`` into one grouped call
+ * (sitech.ge, "Grouped experts instead of a Python loop"; andresseo.expert, "Fragmented
+ * Expert Kernels"), and operands in MXFP8: 8-bit E4M3 elements with one power-of-two
+ * E8M0 scale per block of 32 consecutive values along the GEMM's K (sitech.ge, "Memory and
+ * quantization overhead"; ai4snews, paragraph 2), quantised every step from 16-bit masters.
+ *
+ * Conventions for every entry point
+ *  - Pointers are DEVICE pointers unless the comment says host.  The caller allocates and
+ *    owns every buffer; the library never allocates device memory inside a call (the only
+ *    allocation is the small status block made by moe_ctx_create).
+ *  - Tensors are row-major and contiguous.  bf16 = IEEE bfloat16 (2 bytes).  E4M3 codes and
+ *    E8M0 scale bytes are uint8.  Device buffers must be 16-byte aligned.
+ *  - ``stream`` is a cudaStream_t (NULL = legacy default stream).  Every call only enqueues
+ *    work and returns; nothing synchronises except moe_get_status.
+ *  - Host-side checks return an error code and enqueue nothing.  Errors found on the device
+ *    (an expert index out of range, a split_sizes that disagrees with topk_idx, a bounded
+ *    wait that expired) are recorded in the context's device status word; the kernels that
+ *    find them stop early without trapping.  moe_get_status reads and clears that word.
+ *  - Calls that share a context may run on different streams; they share only the status word.
+ */
+#ifndef MOEMX_H
+#define MOEMX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Rows of the permuted (expert-sorted) token space are grouped into per-expert segments
+ * padded to a multiple of this many rows.  128 is one tensor-core tile and a multiple of the
+ * 32-row MXFP8 block, so token-axis scale blocks never straddle two experts. */
+#define MOE_ROW_ALIGN 128
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, negative or zero size, bad flag              */
+  MOE_ERR_SHAPE = 2,        /* a size breaks an alignment rule stated below               */
+  MOE_ERR_UNSUPPORTED = 3,  /* device is not sm_100, or E/k beyond the stated maxima      */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (launch, tensor map)    */
+  MOE_ERR_DEVICE = 5,       /* device-detected: expert index out of range or a caller
+                               split_sizes that does not match topk_idx                   */
+  MOE_ERR_TIMEOUT = 6,      /* a bounded in-kernel wait expired; the kernel gave up       */
+  MOE_ERR_WORKSPACE = 7     /* a workspace / saved buffer is smaller than required        */
+} moe_status_t;
+
+typedef enum { MOE_PREC_BF16 = 0, MOE_PREC_MXFP8 = 1 } moe_precision_t;
+
+/* flags of mxfp8_quantize */
+#define MXFP8_ROWWISE 1        /* blocks of 32 along each row                              */
+#define MXFP8_COLWISE_T 2      /* blocks of 32 down each column, written transposed        */
+#define MXFP8_SF_MMA_LAYOUT 4  /* scales in the tensor-core tile layout instead of row-major */
+
+#define MOE_MAX_EXPERTS 256
+#define MOE_MAX_TOPK 8
+
+typedef struct moe_ctx_s* moe_ctx_t;
+
+/* Create a context bound to CUDA device ``device`` (allocates a 256-byte device status block).
+ * Returns MOE_ERR_UNSUPPORTED unless the device is compute capability 10.0. */
+moe_status_t moe_ctx_create(moe_ctx_t* ctx, int device);
+moe_status_t moe_ctx_destroy(moe_ctx_t ctx);
+
+/* Synchronise ``stream``, then read and clear the device status word.  Returns MOE_OK,
+ * MOE_ERR_DEVICE or MOE_ERR_TIMEOUT (device errors), or MOE_ERR_CUDA if the stream itself
+ * reported an error. */
+moe_status_t moe_get_status(moe_ctx_t ctx, void* stream);
+
+/* Debug hooks (tests only).  When set, the gate_up GEMM epilogue writes the fp32 value of
+ * a = silu(g)*u*p it quantises into ``a_f32`` [capacity, f], and the down-projection dgrad
+ * epilogue writes the fp32 dh = [dg, du] it quantises into ``dh_f32`` [capacity, 2f]; pass
+ * NULL to switch off.  The buffers must outlive every call that runs while set. */
+moe_status_t moe_ctx_set_debug_dump(moe_ctx_t ctx, float* a_f32, float* dh_f32);
+
+const char* moe_status_string(moe_status_t s);
+
+/* ---------------------------------------------------------------------------------------
+ * mxfp8_quantize: bf16 -> MXFP8 (sitech.ge "Memory and quantization overhead": one scale per
+ * block of 32 consecutive values; ai4snews paragraph 2).
+ *
+ * x        bf16 [batch, rows, cols]
+ * flags    MXFP8_ROWWISE and/or MXFP8_COLWISE_T, optionally | MXFP8_SF_MMA_LAYOUT
+ * q_row    uint8 [batch, rows, cols] E4M3 codes, blocks of 32 along each row   (ROWWISE)
+ * s_row    uint8 E8M0 bytes, [batch, rows, cols/32] row-major, or the MMA layout (ROWWISE)
+ * q_colT   uint8 [batch, cols, rows] codes of blocks of 32 down each column, transposed
+ * s_colT   uint8 E8M0 bytes, [batch, cols, rows/32] row-major, or the MMA layout
+ *
+ * Scale rule: e = the smallest integer with amax <= 448 * 2^e over the block (clamped to
+ * [-127, 127]), byte = e + 127; element code = E4M3(v * 2^-e) rounded to nearest-even,
+ * saturating (no element can exceed 448 under this rule); all-zero blocks get byte 0.
+ *
+ * MMA layout (MXFP8_SF_MMA_LAYOUT): a scale matrix S[R][KB] (R rows, KB = K/32 blocks) is
+ * stored as 512-byte tiles, tile (R/128 index rb, KB/4 index kb4) at byte (rb*KB/4 + kb4)*512,
+ * and inside a tile S[r][kb] sits at 16*(r%32) + 4*((r/32)%4) + kb%4.  It needs R and K to be
+ * multiples of 128 for each batch; a batch's tiles follow the previous batch's.
+ *
+ * Shapes: cols % 32 == 0; rows % 32 == 0 when COLWISE_T is set; with the MMA layout rows and
+ * cols must be multiples of 128.  Returns MOE_ERR_SHAPE otherwise.
+ */
+moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t rows, int64_t cols,
+                            int flags, uint8_t* q_row, uint8_t* s_row, uint8_t* q_colT, uint8_t* s_colT,
+                            void* stream);
+
+/* Inverse of mxfp8_quantize for row-wise data (tests): out[r][c] = decode(q[r][c]) * 2^(s-127),
+ * fp32 [rows, cols]; ``sf_mma_layout`` says how ``s`` is laid out.  cols % 32 == 0. */
+moe_status_t mxfp8_dequantize(moe_ctx_t ctx, const uint8_t* q, const uint8_t* s, int64_t rows, int64_t cols,
+                              int sf_mma_layout, float* out, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Routing bookkeeping and token permutation (sitech.ge "Grouped experts instead of a Python
+ * loop": GroupedLinear gathers each expert's tokens and takes per-expert counts).
+ *
+ * capacity = moe_capacity_rows(T, k, E): the padded row count for the worst-case routing.
+ * Slot s = t*k + j (token t, choice j) goes to expert topk_idx[t][j]; experts keep their slots
+ * in increasing s (a stable counting sort); expert e owns rows [poffsets[e], poffsets[e+1])
+ * of the permuted space, its split_sizes[e] slots first, then zero padding up to a multiple
+ * of MOE_ROW_ALIGN.  Rows past poffsets[E] up to capacity are padding as well.
+ */
+int64_t moe_capacity_rows(int64_t T, int k, int E);
+
+/* x            bf16 [T, d] or NULL (routing only)
+ * topk_idx     int32 [T, k], values in [0, E)
+ * topk_prob    fp32 [T, k] or NULL
+ * split_sizes_in int32 [E] or NULL: if given it must equal the histogram of topk_idx
+ *              (MOE_ERR_DEVICE otherwise, reported by moe_get_status)
+ * outputs      split_sizes int32 [E]; poffsets int32 [E+1]; sorted_to_src int32 [capacity]
+ *              (slot of each row, -1 for padding); src_to_sorted int32 [T*k] (row of each slot);
+ *              prob_perm fp32 [capacity] or NULL (topk_prob of each row, 0 for padding);
+ *              x_perm bf16 [capacity, d] or NULL (x[slot/k] per row, zeros for padding)
+ * Limits: 1 <= k <= MOE_MAX_TOPK, 1 <= E <= MOE_MAX_EXPERTS, d % 32 == 0. */
+moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, const float* topk_prob,
+                         int64_t T, int k, int E, int64_t d, const int32_t* split_sizes_in,
+                         int32_t* split_sizes, int32_t* poffsets, int32_t* sorted_to_src,
+                         int32_t* src_to_sorted, float* prob_perm, void* x_perm, void* stream);
+
+/* Combine rows back to tokens: y[t] = bf16( sum_{j<k} w_j * fp32(y_perm[src_to_sorted[t*k+j]]) )
+ * summed in fp32 in order j = 0..k-1, with w_j = probs[t][j] (fp32 products) or 1 if probs is
+ * NULL (the fused layer applies the probability inside ScaledSwiGLU, so it combines with NULL).
+ * y_perm bf16 [capacity, d]; y bf16 [T, d]; d % 8 == 0. */
+moe_status_t moe_unpermute(moe_ctx_t ctx, const void* y_perm, const int32_t* src_to_sorted, const float* probs,
+                           int64_t T, int k, int64_t d, void* y, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * The fused layer (ai4snews paragraph 3: Sequential(GroupedLinear(gate_up), ScaledSwiGLU(),
+ * GroupedLinear(down)) with a matching fused backward; sitech.ge "Memory and quantization
+ * overhead").  For slot (t, j), e = topk_idx[t][j], p = topk_prob[t][j]:
+ *   h = x_t W1_e^T,  g = h[0:f], u = h[f:2f],  a = silu(g) * u * p,  y_t += a W2_e^T
+ * W1_e = w_gate_up[e] bf16 [2f, d] (gate rows first), W2_e = w_down[e] bf16 [d, f].
+ * MXFP8: every GEMM operand is quantised along that GEMM's K with blocks of 32; the weights
+ * are quantised from the bf16 masters inside each call.  a is requantised straight from the
+ * gate_up GEMM's epilogue into the down GEMM's operand; h never goes to memory except the bf16
+ * copy saved for the backward when ``training`` is set.  Products accumulate in fp32.
+ *
+ * w_gate_up, w_down, dw_gate_up, dw_down are HOST arrays of E device pointers (each expert
+ * keeps its own weight tensor, ai4snews paragraph 1).
+ * Shapes: d % 256 == 0, f % 256 == 0, 1 <= k <= MOE_MAX_TOPK, 1 <= E <= MOE_MAX_EXPERTS.
+ *
+ * saved: written by a training forward, read by the backward; moe_saved_size bytes.
+ * workspace: scratch for one call; moe_fwd_workspace_size / moe_bwd_workspace_size bytes.
+ * Neither may be shared by two calls in flight at once.
+ */
+size_t moe_saved_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec);
+size_t moe_fwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training);
+size_t moe_bwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec);
+
+/* x bf16 [T, d]; topk_idx int32 [T, k]; topk_prob fp32 [T, k]; split_sizes int32 [E] or NULL
+ * (checked against topk_idx on the device when given); y bf16 [T, d]. */
+moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, const float* topk_prob,
+                                 const int32_t* split_sizes, const void* const* w_gate_up,
+                                 const void* const* w_down, int64_t T, int64_t d, int64_t f, int E, int k,
+                                 moe_precision_t prec, int training, void* y, void* saved, size_t saved_bytes,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* dy bf16 [T, d]; saved from a training forward with the same arguments; outputs dx bf16 [T, d],
+ * dw_gate_up[e] bf16 [2f, d], dw_down[e] bf16 [d, f] (overwritten, zeros for experts with no
+ * tokens), d_topk_prob fp32 [T, k] (gradient of topk_prob). */
+moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* saved, size_t saved_bytes,
+                                 const void* const* w_gate_up, const void* const* w_down, int64_t T, int64_t d,
+                                 int64_t f, int E, int k, moe_precision_t prec, void* dx, void* const* dw_gate_up,
+                                 void* const* dw_down, float* d_topk_prob, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/* Inspection hook (tests): address of a named intermediate inside a saved buffer (which = 0),
+ * a forward workspace (which = 1) or a backward workspace (which = 2) laid out for these
+ * dimensions, given the buffer's base address ``base``; NULL for an unknown name.  Names:
+ * saved: split_sizes poffsets sorted_to_src src_to_sorted prob_perm w1c_q w1c_s w2c_q w2c_s
+ *        xT_q xT_s aT_q aT_s xT aT h
+ * forward workspace: w1_q w1_s w2_q w2_s x_q x_s a_q a_s x_perm a y_perm (+ the routing names
+ *        when training == 0)
+ * backward workspace: dy_q dy_s dyT_q dyT_s dh_q dh_s dhT_q dhT_s dy_perm dyT dh dhT w1T w2T
+ *        dx_perm dp_part
+ * Scales (*_s) are in the tensor-core tile layout described at mxfp8_quantize. */
+void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
+                         int which, void* base, const char* name);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEMX_H */

@@ -1,0 +1,854 @@
+// C ABI of libmoemx (declared in include/moemx.h): argument checks, buffer layout of the
+// saved / workspace regions, TMA tensor maps, and the launch sequence of the fused layer.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "codec.cuh"
+#include "common.cuh"
+#include "gemm.cuh"
+
+using namespace moemx;
+
+struct moe_ctx_s {
+  int device;
+  int num_sms;
+  int* d_status;  // [0] status bits
+  float* dbg_a;
+  float* dbg_dh;
+};
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D map over [rows, inner] (inner contiguous), box 128 rows x 128 bytes, 128-byte swizzle.
+bool map_2d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t rows, uint64_t row_bytes) {
+  const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {fp8 ? 128u : 64u, 128u};
+  cuuint32_t es[2] = {1, 1};
+  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 3-D map over [E, rows, inner] with an arbitrary (16-byte multiple) stride between experts.
+bool map_3d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t rows, uint64_t E,
+            uint64_t row_bytes, uint64_t expert_bytes) {
+  const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[3] = {inner, rows, E};
+  cuuint64_t strides[2] = {row_bytes, expert_bytes};
+  cuuint32_t box[3] = {fp8 ? 128u : 64u, 128u, 1u};
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Bump allocator over a caller buffer (1 KiB granules); with base == nullptr it only measures.
+struct Carve {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(size_t bytes) {
+    off = (off + 1023) & ~size_t(1023);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+struct Dims {
+  int64_t T, d, f, cap, Tk;
+  int E, k;
+  bool mx;
+};
+
+// Everything a training forward leaves for the backward.
+struct Saved {
+  int32_t *split, *poff, *s2src, *src2s;
+  float* pperm;
+  uint8_t *w1c_q, *w1c_s, *w2c_q, *w2c_s;  // MXFP8: weights quantised down the columns, transposed
+  uint8_t *xT_q, *xT_s, *aT_q, *aT_s;      // MXFP8: token-axis quantised x and a, transposed
+  bf16 *xT, *aT;                           // BF16: transposed copies
+  bf16* h;                                 // [cap, 2f] gate/up pre-activations
+};
+void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
+  s.split = c.take<int32_t>(D.E * 4);
+  s.poff = c.take<int32_t>((D.E + 1) * 4);
+  s.s2src = c.take<int32_t>(D.cap * 4);
+  s.src2s = c.take<int32_t>(D.Tk * 4);
+  s.pperm = c.take<float>(D.cap * 4);
+  s.w1c_q = s.w1c_s = s.w2c_q = s.w2c_s = s.xT_q = s.xT_s = s.aT_q = s.aT_s = nullptr;
+  s.xT = s.aT = nullptr;
+  s.h = nullptr;
+  if (!full) return;  // inference: routing bookkeeping only
+  if (D.mx) {
+    s.w1c_q = c.take<uint8_t>(D.E * D.d * 2 * D.f);
+    s.w1c_s = c.take<uint8_t>(D.E * D.d * 2 * D.f / 32);
+    s.w2c_q = c.take<uint8_t>(D.E * D.f * D.d);
+    s.w2c_s = c.take<uint8_t>(D.E * D.f * D.d / 32);
+    s.xT_q = c.take<uint8_t>(D.d * D.cap);
+    s.xT_s = c.take<uint8_t>(D.d * D.cap / 32);
+    s.aT_q = c.take<uint8_t>(D.f * D.cap);
+    s.aT_s = c.take<uint8_t>(D.f * D.cap / 32);
+  } else {
+    s.xT = c.take<bf16>(D.d * D.cap * 2);
+    s.aT = c.take<bf16>(D.f * D.cap * 2);
+  }
+  s.h = c.take<bf16>(D.cap * 2 * D.f * 2);
+}
+
+struct FwdWs {
+  uint8_t *w1_q, *w1_s, *w2_q, *w2_s, *x_q, *x_s, *a_q, *a_s;
+  bf16 *x_perm, *a, *w1_copy, *w2_copy;
+  bf16* y_perm;
+};
+void carve_fwd(Carve& c, const Dims& D, FwdWs& w) {
+  std::memset(&w, 0, sizeof(w));
+  if (D.mx) {
+    w.w1_q = c.take<uint8_t>(D.E * 2 * D.f * D.d);
+    w.w1_s = c.take<uint8_t>(D.E * 2 * D.f * D.d / 32);
+    w.w2_q = c.take<uint8_t>(D.E * D.d * D.f);
+    w.w2_s = c.take<uint8_t>(D.E * D.d * D.f / 32);
+    w.x_q = c.take<uint8_t>(D.cap * D.d);
+    w.x_s = c.take<uint8_t>(D.cap * D.d / 32);
+    w.a_q = c.take<uint8_t>(D.cap * D.f);
+    w.a_s = c.take<uint8_t>(D.cap * D.f / 32);
+  } else {
+    w.x_perm = c.take<bf16>(D.cap * D.d * 2);
+    w.a = c.take<bf16>(D.cap * D.f * 2);
+    w.w1_copy = c.take<bf16>(D.E * 2 * D.f * D.d * 2);
+    w.w2_copy = c.take<bf16>(D.E * D.d * D.f * 2);
+  }
+  w.y_perm = c.take<bf16>(D.cap * D.d * 2);
+}
+
+struct BwdWs {
+  uint8_t *dy_q, *dy_s, *dyT_q, *dyT_s, *dh_q, *dh_s, *dhT_q, *dhT_s;
+  bf16 *dy_perm, *dyT, *dh, *dhT, *w1T, *w2T;
+  bf16* dx_perm;
+  float* dp_part;
+};
+void carve_bwd(Carve& c, const Dims& D, BwdWs& w) {
+  std::memset(&w, 0, sizeof(w));
+  if (D.mx) {
+    w.dy_q = c.take<uint8_t>(D.cap * D.d);
+    w.dy_s = c.take<uint8_t>(D.cap * D.d / 32);
+    w.dyT_q = c.take<uint8_t>(D.d * D.cap);
+    w.dyT_s = c.take<uint8_t>(D.d * D.cap / 32);
+    w.dh_q = c.take<uint8_t>(D.cap * 2 * D.f);
+    w.dh_s = c.take<uint8_t>(D.cap * 2 * D.f / 32);
+    w.dhT_q = c.take<uint8_t>(2 * D.f * D.cap);
+    w.dhT_s = c.take<uint8_t>(2 * D.f * D.cap / 32);
+  } else {
+    w.dy_perm = c.take<bf16>(D.cap * D.d * 2);
+    w.dyT = c.take<bf16>(D.d * D.cap * 2);
+    w.dh = c.take<bf16>(D.cap * 2 * D.f * 2);
+    w.dhT = c.take<bf16>(2 * D.f * D.cap * 2);
+    w.w1T = c.take<bf16>(D.E * D.d * 2 * D.f * 2);
+    w.w2T = c.take<bf16>(D.E * D.f * D.d * 2);
+  }
+  w.dx_perm = c.take<bf16>(D.cap * D.d * 2);
+  w.dp_part = c.take<float>(2 * (D.f / 256) * D.cap * 4);
+}
+
+int64_t capacity_rows(int64_t T, int k, int E) {
+  return round_up(T * k + static_cast<int64_t>(E) * (MOE_ROW_ALIGN - 1), MOE_ROW_ALIGN);
+}
+
+moe_status_t check_dims(int64_t T, int64_t d, int64_t f, int E, int k) {
+  if (T <= 0 || d <= 0 || f <= 0) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > MOE_MAX_EXPERTS || k < 1 || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (d % 256 || f % 256) return MOE_ERR_SHAPE;
+  if (capacity_rows(T, k, E) >= (int64_t(1) << 31) / 2) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+Dims make_dims(int64_t T, int64_t d, int64_t f, int E, int k, moe_precision_t prec) {
+  Dims D;
+  D.T = T;
+  D.d = d;
+  D.f = f;
+  D.E = E;
+  D.k = k;
+  D.Tk = T * k;
+  D.cap = capacity_rows(T, k, E);
+  D.mx = prec == MOE_PREC_MXFP8;
+  return D;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    cudaGetDevice(&prev);
+    if (prev != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (prev >= 0 && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+#define MOE_CUDA(x)                       \
+  do {                                    \
+    if ((x) != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+// Uniform byte stride between consecutive expert pointers (0 if not uniform / not usable by TMA).
+int64_t uniform_stride(const void* const* p, int E, int64_t min_bytes) {
+  if (E == 1) return min_bytes;
+  const int64_t s = reinterpret_cast<const uint8_t*>(p[1]) - reinterpret_cast<const uint8_t*>(p[0]);
+  if (s < min_bytes || (s & 15)) return 0;
+  for (int e = 2; e < E; ++e)
+    if (reinterpret_cast<const uint8_t*>(p[e]) - reinterpret_cast<const uint8_t*>(p[e - 1]) != s) return 0;
+  return s;
+}
+
+QuantArgs quant_args() {
+  QuantArgs a;
+  std::memset(&a, 0, sizeof(a));
+  return a;
+}
+
+GemmArgs gemm_args(moe_ctx_t ctx) {
+  GemmArgs g;
+  std::memset(&g, 0, sizeof(g));
+  g.status = ctx->d_status;
+  return g;
+}
+
+}  // namespace
+
+// ====================================================================================== ABI
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_SHAPE: return "shape breaks an alignment rule";
+    case MOE_ERR_UNSUPPORTED: return "unsupported device or size";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE: return "device-detected error (bad expert index or split_sizes mismatch)";
+    case MOE_ERR_TIMEOUT: return "bounded in-kernel wait expired";
+    case MOE_ERR_WORKSPACE: return "workspace or saved buffer too small";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_ctx_create(moe_ctx_t* out, int device) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return MOE_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return MOE_ERR_UNSUPPORTED;
+  if (!encoder()) return MOE_ERR_CUDA;
+  DeviceGuard guard(device);
+  moe_ctx_s* c = new moe_ctx_s();
+  c->device = device;
+  c->num_sms = prop.multiProcessorCount;
+  c->dbg_a = c->dbg_dh = nullptr;
+  if (cudaMalloc(&c->d_status, 256) != cudaSuccess) {
+    delete c;
+    return MOE_ERR_CUDA;
+  }
+  if (cudaMemset(c->d_status, 0, 256) != cudaSuccess) {
+    cudaFree(c->d_status);
+    delete c;
+    return MOE_ERR_CUDA;
+  }
+  *out = c;
+  return MOE_OK;
+}
+
+moe_status_t moe_ctx_destroy(moe_ctx_t ctx) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->device);
+  cudaFree(ctx->d_status);
+  delete ctx;
+  return MOE_OK;
+}
+
+moe_status_t moe_ctx_set_debug_dump(moe_ctx_t ctx, float* a_f32, float* dh_f32) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  ctx->dbg_a = a_f32;
+  ctx->dbg_dh = dh_f32;
+  return MOE_OK;
+}
+
+moe_status_t moe_get_status(moe_ctx_t ctx, void* stream) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, ctx->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word && cudaMemset(ctx->d_status, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word & kStatusTimeout) return MOE_ERR_TIMEOUT;
+  if (word & kStatusDevice) return MOE_ERR_DEVICE;
+  return MOE_OK;
+}
+
+int64_t moe_capacity_rows(int64_t T, int k, int E) {
+  if (T < 0 || k < 1 || E < 1) return 0;
+  return capacity_rows(T, k, E);
+}
+
+moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t rows, int64_t cols, int flags,
+                            uint8_t* q_row, uint8_t* s_row, uint8_t* q_colT, uint8_t* s_colT, void* stream) {
+  if (!ctx || !x || batch <= 0 || rows <= 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+  const bool row = flags & MXFP8_ROWWISE, col = flags & MXFP8_COLWISE_T, mma = flags & MXFP8_SF_MMA_LAYOUT;
+  if ((flags & ~7) || !(row || col)) return MOE_ERR_INVALID_ARG;
+  if (row && (!q_row || !s_row)) return MOE_ERR_INVALID_ARG;
+  if (col && (!q_colT || !s_colT)) return MOE_ERR_INVALID_ARG;
+  if (cols % 32) return MOE_ERR_SHAPE;
+  if (col && rows % 32) return MOE_ERR_SHAPE;
+  if (mma && (rows % 128 || cols % 128)) return MOE_ERR_SHAPE;
+  if (batch > MOE_MAX_EXPERTS * 256 || rows > (int64_t(1) << 31) / 64 * 64 || cols > (int64_t(1) << 31))
+    return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || (row && !aligned16(q_row)) || (col && !aligned16(q_colT))) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->device);
+  QuantArgs a = quant_args();
+  a.src = static_cast<const bf16*>(x);
+  a.src_batch_stride = rows * cols;
+  a.src_ld = cols;
+  a.rows = rows;
+  a.cols = cols;
+  a.mx = 1;
+  a.do_row = row;
+  a.do_col = col;
+  a.sf_mma = mma;
+  a.q_row = q_row;
+  a.s_row = s_row;
+  a.q_colT = q_colT;
+  a.s_colT = s_colT;
+  MOE_CUDA(launch_quant(a, static_cast<int>(batch), static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status_t mxfp8_dequantize(moe_ctx_t ctx, const uint8_t* q, const uint8_t* s, int64_t rows, int64_t cols,
+                              int sf_mma_layout, float* out, void* stream) {
+  if (!ctx || !q || !s || !out || rows <= 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+  if (cols % 32) return MOE_ERR_SHAPE;
+  if (sf_mma_layout && (rows % 128 || cols % 128)) return MOE_ERR_SHAPE;
+  DeviceGuard guard(ctx->device);
+  MOE_CUDA(launch_dequant(q, s, rows, cols, sf_mma_layout, out, ctx->num_sms, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, const float* topk_prob, int64_t T,
+                         int k, int E, int64_t d, const int32_t* split_sizes_in, int32_t* split_sizes,
+                         int32_t* poffsets, int32_t* sorted_to_src, int32_t* src_to_sorted, float* prob_perm,
+                         void* x_perm, void* stream) {
+  if (!ctx || !topk_idx || !split_sizes || !poffsets || !sorted_to_src || !src_to_sorted) return MOE_ERR_INVALID_ARG;
+  if (T <= 0) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > MOE_MAX_EXPERTS || k < 1 || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (prob_perm && !topk_prob) return MOE_ERR_INVALID_ARG;
+  if ((x_perm != nullptr) != (x != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (x && (d <= 0 || d % 32 || !aligned16(x) || !aligned16(x_perm))) return x && d % 32 ? MOE_ERR_SHAPE : MOE_ERR_INVALID_ARG;
+  const int64_t cap = capacity_rows(T, k, E);
+  if (cap >= (int64_t(1) << 31) / 2) return MOE_ERR_UNSUPPORTED;
+  DeviceGuard guard(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_CUDA(launch_route(topk_idx, topk_prob, static_cast<int>(T * k), E, static_cast<int>(cap), split_sizes_in,
+                        split_sizes, poffsets, sorted_to_src, src_to_sorted, prob_perm, ctx->d_status, st));
+  if (x) {
+    QuantArgs a = quant_args();
+    a.src = static_cast<const bf16*>(x);
+    a.src_ld = d;
+    a.sorted_to_src = sorted_to_src;
+    a.k = k;
+    a.rows = cap;
+    a.cols = d;
+    a.mx = 0;
+    a.do_row = 1;
+    a.o_row = static_cast<bf16*>(x_perm);
+    MOE_CUDA(launch_quant(a, 1, st));
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_unpermute(moe_ctx_t ctx, const void* y_perm, const int32_t* src_to_sorted, const float* probs,
+                           int64_t T, int k, int64_t d, void* y, void* stream) {
+  if (!ctx || !y_perm || !src_to_sorted || !y || T <= 0 || d <= 0) return MOE_ERR_INVALID_ARG;
+  if (k < 1 || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (d % 8) return MOE_ERR_SHAPE;
+  if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->device);
+  MOE_CUDA(launch_unpermute(static_cast<const bf16*>(y_perm), src_to_sorted, probs, T, k, d, static_cast<bf16*>(y),
+                            ctx->num_sms, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+size_t moe_saved_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec) {
+  if (check_dims(T, d, f, E, k) != MOE_OK) return 0;
+  Dims D = make_dims(T, d, f, E, k, prec);
+  Carve c(nullptr);
+  Saved s;
+  carve_saved(c, D, s);
+  return c.off + 1024;
+}
+
+size_t moe_fwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training) {
+  if (check_dims(T, d, f, E, k) != MOE_OK) return 0;
+  Dims D = make_dims(T, d, f, E, k, prec);
+  Carve c(nullptr);
+  FwdWs w;
+  carve_fwd(c, D, w);
+  if (!training) {  // routing bookkeeping lives in the workspace when nothing is saved
+    Saved s;
+    carve_saved(c, D, s, false);
+  }
+  return c.off + 1024;
+}
+
+size_t moe_bwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec) {
+  if (check_dims(T, d, f, E, k) != MOE_OK) return 0;
+  Dims D = make_dims(T, d, f, E, k, prec);
+  Carve c(nullptr);
+  BwdWs w;
+  carve_bwd(c, D, w);
+  return c.off + 1024;
+}
+
+moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, const float* topk_prob,
+                                 const int32_t* split_sizes, const void* const* w_gate_up,
+                                 const void* const* w_down, int64_t T, int64_t d, int64_t f, int E, int k,
+                                 moe_precision_t prec, int training, void* y, void* saved, size_t saved_bytes,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ctx || !x || !topk_idx || !topk_prob || !w_gate_up || !w_down || !y || !workspace) return MOE_ERR_INVALID_ARG;
+  if (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8) return MOE_ERR_INVALID_ARG;
+  const moe_status_t dc = check_dims(T, d, f, E, k);
+  if (dc != MOE_OK) return dc;
+  if (training && !saved) return MOE_ERR_INVALID_ARG;
+  for (int e = 0; e < E; ++e)
+    if (!w_gate_up[e] || !w_down[e] || !aligned16(w_gate_up[e]) || !aligned16(w_down[e])) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < moe_fwd_workspace_size(T, k, E, d, f, prec, training)) return MOE_ERR_WORKSPACE;
+  if (training && saved_bytes < moe_saved_size(T, k, E, d, f, prec)) return MOE_ERR_WORKSPACE;
+
+  DeviceGuard guard(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Dims D = make_dims(T, d, f, E, k, prec);
+  Carve cw(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(workspace), 1024)));
+  FwdWs w;
+  carve_fwd(cw, D, w);
+  Saved s;
+  if (training) {
+    Carve cs(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(saved), 1024)));
+    carve_saved(cs, D, s);
+  } else {
+    carve_saved(cw, D, s, false);
+  }
+
+  // 1. routing: counts, padded offsets, stable permutation, per-row probabilities
+  MOE_CUDA(launch_route(topk_idx, topk_prob, static_cast<int>(D.Tk), E, static_cast<int>(D.cap), split_sizes, s.split,
+                        s.poff, s.s2src, s.src2s, s.pperm, ctx->d_status, st));
+
+  // 2. operands of the gate_up GEMM
+  const void* w1_base;
+  const void* w2_base;
+  int64_t w1_stride, w2_stride;  // bytes between experts
+  if (D.mx) {
+    // 16-bit masters -> MXFP8 every step: row-wise (K = d / f of the forward GEMMs) and, for the
+    // backward, down the columns (K = 2f / d of the dgrad GEMMs), from one read of each weight.
+    QuantArgs a = quant_args();
+    for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_gate_up[e];
+    a.src_ld = d;
+    a.rows = 2 * f;
+    a.cols = d;
+    a.mx = 1;
+    a.sf_mma = 1;
+    a.do_row = 1;
+    a.q_row = w.w1_q;
+    a.s_row = w.w1_s;
+    a.do_col = training;
+    a.q_colT = s.w1c_q;
+    a.s_colT = s.w1c_s;
+    MOE_CUDA(launch_quant(a, E, st));
+    for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
+    a.src_ld = f;
+    a.rows = d;
+    a.cols = f;
+    a.q_row = w.w2_q;
+    a.s_row = w.w2_s;
+    a.q_colT = s.w2c_q;
+    a.s_colT = s.w2c_s;
+    MOE_CUDA(launch_quant(a, E, st));
+    w1_base = w.w1_q;
+    w1_stride = 2 * f * d;
+    w2_base = w.w2_q;
+    w2_stride = d * f;
+
+    // x: gather by expert + row-wise MXFP8 (K = d) and, for wgrad, token-axis MXFP8 transposed
+    QuantArgs xa = quant_args();
+    xa.src = static_cast<const bf16*>(x);
+    xa.src_ld = d;
+    xa.sorted_to_src = s.s2src;
+    xa.k = k;
+    xa.rows = D.cap;
+    xa.cols = d;
+    xa.mx = 1;
+    xa.sf_mma = 1;
+    xa.do_row = 1;
+    xa.q_row = w.x_q;
+    xa.s_row = w.x_s;
+    xa.do_col = training;
+    xa.q_colT = s.xT_q;
+    xa.s_colT = s.xT_s;
+    MOE_CUDA(launch_quant(xa, 1, st));
+  } else {
+    w1_stride = uniform_stride(w_gate_up, E, 2 * f * d * 2);
+    w2_stride = uniform_stride(w_down, E, d * f * 2);
+    w1_base = w_gate_up[0];
+    w2_base = w_down[0];
+    QuantArgs a = quant_args();
+    a.mx = 0;
+    a.do_row = 1;
+    if (!w1_stride) {  // experts not evenly spaced: gather into one [E, 2f, d] tensor
+      for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_gate_up[e];
+      a.src_ld = d;
+      a.rows = 2 * f;
+      a.cols = d;
+      a.o_row = w.w1_copy;
+      MOE_CUDA(launch_quant(a, E, st));
+      w1_base = w.w1_copy;
+      w1_stride = 2 * f * d * 2;
+    }
+    if (!w2_stride) {
+      for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
+      a.src_ld = f;
+      a.rows = d;
+      a.cols = f;
+      a.o_row = w.w2_copy;
+      MOE_CUDA(launch_quant(a, E, st));
+      w2_base = w.w2_copy;
+      w2_stride = d * f * 2;
+    }
+    QuantArgs xa = quant_args();
+    xa.src = static_cast<const bf16*>(x);
+    xa.src_ld = d;
+    xa.sorted_to_src = s.s2src;
+    xa.k = k;
+    xa.rows = D.cap;
+    xa.cols = d;
+    xa.mx = 0;
+    xa.do_row = 1;
+    xa.o_row = w.x_perm;
+    xa.do_col = training;
+    xa.o_colT = s.xT;
+    MOE_CUDA(launch_quant(xa, 1, st));
+  }
+
+  // 3. gate_up GEMM + ScaledSwiGLU + requantisation of a
+  {
+    GemmArgs g = gemm_args(ctx);
+    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.x_q) : w.x_perm, D.mx, d, D.cap,
+                           d * (D.mx ? 1 : 2)) &&
+                    map_3d(&g.tmap_b, w1_base, D.mx, d, 2 * f, E, d * (D.mx ? 1 : 2), w1_stride);
+    if (!ok) return MOE_ERR_CUDA;
+    g.kgrouped = 0;
+    g.E = E;
+    g.K = static_cast<int>(d);
+    g.n_tiles = static_cast<int>(f / 128);
+    g.gate_up_half = static_cast<int>(f);
+    g.poffsets = s.poff;
+    g.sfa = w.x_s;
+    g.sfa_kb4 = d / 128;
+    g.sfb = w.w1_s;
+    g.sfb_kb4 = d / 128;
+    g.sfb_expert_rows = 2 * f;
+    EpiArgs& ep = g.epi;
+    ep.f = f;
+    ep.cap = D.cap;
+    ep.p_perm = s.pperm;
+    ep.h = training ? s.h : nullptr;
+    ep.dump = ctx->dbg_a;
+    if (D.mx) {
+      ep.q_row = w.a_q;
+      ep.s_row = w.a_s;
+      ep.q_colT = training ? s.aT_q : nullptr;
+      ep.s_colT = training ? s.aT_s : nullptr;
+    } else {
+      ep.o_row = w.a;
+      ep.o_colT = training ? s.aT : nullptr;
+    }
+    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_SWIGLU, ctx->num_sms, st));
+  }
+  // 4. down GEMM
+  {
+    GemmArgs g = gemm_args(ctx);
+    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.a_q) : w.a, D.mx, f, D.cap,
+                           f * (D.mx ? 1 : 2)) &&
+                    map_3d(&g.tmap_b, w2_base, D.mx, f, d, E, f * (D.mx ? 1 : 2), w2_stride);
+    if (!ok) return MOE_ERR_CUDA;
+    g.kgrouped = 0;
+    g.E = E;
+    g.K = static_cast<int>(f);
+    g.n_tiles = static_cast<int>(d / 256);
+    g.poffsets = s.poff;
+    g.sfa = w.a_s;
+    g.sfa_kb4 = f / 128;
+    g.sfb = w.w2_s;
+    g.sfb_kb4 = f / 128;
+    g.sfb_expert_rows = d;
+    g.epi.out = w.y_perm;
+    g.epi.ldo = d;
+    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+  }
+  // 5. combine (probabilities were applied in ScaledSwiGLU)
+  MOE_CUDA(launch_unpermute(w.y_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(y), ctx->num_sms, st));
+  return MOE_OK;
+}
+
+moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* saved, size_t saved_bytes,
+                                 const void* const* w_gate_up, const void* const* w_down, int64_t T, int64_t d,
+                                 int64_t f, int E, int k, moe_precision_t prec, void* dx, void* const* dw_gate_up,
+                                 void* const* dw_down, float* d_topk_prob, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!ctx || !dy || !saved || !w_gate_up || !w_down || !dx || !dw_gate_up || !dw_down || !d_topk_prob || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8) return MOE_ERR_INVALID_ARG;
+  const moe_status_t dc = check_dims(T, d, f, E, k);
+  if (dc != MOE_OK) return dc;
+  for (int e = 0; e < E; ++e)
+    if (!w_gate_up[e] || !w_down[e] || !dw_gate_up[e] || !dw_down[e] || !aligned16(dw_gate_up[e]) ||
+        !aligned16(dw_down[e]) || !aligned16(w_gate_up[e]) || !aligned16(w_down[e]))
+      return MOE_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(dx)) return MOE_ERR_INVALID_ARG;
+  if (saved_bytes < moe_saved_size(T, k, E, d, f, prec)) return MOE_ERR_WORKSPACE;
+  if (workspace_bytes < moe_bwd_workspace_size(T, k, E, d, f, prec)) return MOE_ERR_WORKSPACE;
+
+  DeviceGuard guard(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Dims D = make_dims(T, d, f, E, k, prec);
+  Saved s;
+  Carve cs(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(saved), 1024)));
+  carve_saved(cs, D, s);
+  BwdWs w;
+  Carve cw(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(workspace), 1024)));
+  carve_bwd(cw, D, w);
+
+  // 1. dy gathered by expert: row-wise (K = d, dgrad of down) and token-axis transposed (wgrad of down)
+  {
+    QuantArgs a = quant_args();
+    a.src = static_cast<const bf16*>(dy);
+    a.src_ld = d;
+    a.sorted_to_src = s.s2src;
+    a.k = k;
+    a.rows = D.cap;
+    a.cols = d;
+    a.do_row = 1;
+    a.do_col = 1;
+    if (D.mx) {
+      a.mx = 1;
+      a.sf_mma = 1;
+      a.q_row = w.dy_q;
+      a.s_row = w.dy_s;
+      a.q_colT = w.dyT_q;
+      a.s_colT = w.dyT_s;
+    } else {
+      a.o_row = w.dy_perm;
+      a.o_colT = w.dyT;
+    }
+    MOE_CUDA(launch_quant(a, 1, st));
+  }
+  const void* w1c;  // B of dgrad of gate_up: [E, d, 2f]
+  const void* w2c;  // B of dgrad of down:    [E, f, d]
+  if (D.mx) {
+    w1c = s.w1c_q;
+    w2c = s.w2c_q;
+  } else {
+    QuantArgs a = quant_args();
+    a.mx = 0;
+    a.do_col = 1;
+    for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_gate_up[e];
+    a.src_ld = d;
+    a.rows = 2 * f;
+    a.cols = d;
+    a.o_colT = w.w1T;
+    MOE_CUDA(launch_quant(a, E, st));
+    for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
+    a.src_ld = f;
+    a.rows = d;
+    a.cols = f;
+    a.o_colT = w.w2T;
+    MOE_CUDA(launch_quant(a, E, st));
+    w1c = w.w1T;
+    w2c = w.w2T;
+  }
+  const int es = D.mx ? 1 : 2;
+  // 2. dgrad of down + ScaledSwiGLU backward: dh = [dg, du] requantised both ways, dp partials
+  {
+    GemmArgs g = gemm_args(ctx);
+    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dy_q) : w.dy_perm, D.mx, d, D.cap, d * es) &&
+                    map_3d(&g.tmap_b, w2c, D.mx, d, f, E, d * es, f * d * es);
+    if (!ok) return MOE_ERR_CUDA;
+    g.kgrouped = 0;
+    g.E = E;
+    g.K = static_cast<int>(d);
+    g.n_tiles = static_cast<int>(f / 256);
+    g.poffsets = s.poff;
+    g.sfa = w.dy_s;
+    g.sfa_kb4 = d / 128;
+    g.sfb = s.w2c_s;
+    g.sfb_kb4 = d / 128;
+    g.sfb_expert_rows = f;
+    EpiArgs& ep = g.epi;
+    ep.f = f;
+    ep.cap = D.cap;
+    ep.p_perm = s.pperm;
+    ep.h = s.h;
+    ep.dump = ctx->dbg_dh;
+    ep.dp_part = w.dp_part;
+    if (D.mx) {
+      ep.q_row = w.dh_q;
+      ep.s_row = w.dh_s;
+      ep.q_colT = w.dhT_q;
+      ep.s_colT = w.dhT_s;
+    } else {
+      ep.o_row = w.dh;
+      ep.o_colT = w.dhT;
+    }
+    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_DSWIGLU, ctx->num_sms, st));
+  }
+  // 3. wgrad of down: dW2_e [d, f] = dy_e^T a_e (K = the expert's tokens)
+  {
+    GemmArgs g = gemm_args(ctx);
+    const bool ok =
+        map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dyT_q) : w.dyT, D.mx, D.cap, d, D.cap * es) &&
+        map_2d(&g.tmap_b, D.mx ? static_cast<const void*>(s.aT_q) : s.aT, D.mx, D.cap, f, D.cap * es);
+    if (!ok) return MOE_ERR_CUDA;
+    g.kgrouped = 1;
+    g.E = E;
+    g.m_tiles = static_cast<int>(d / 128);
+    g.n_tiles = static_cast<int>(f / 256);
+    g.poffsets = s.poff;
+    g.sfa = w.dyT_s;
+    g.sfa_kb4 = D.cap / 128;
+    g.sfb = s.aT_s;
+    g.sfb_kb4 = D.cap / 128;
+    g.epi.ldo = f;
+    for (int e = 0; e < E; ++e) g.epi.out_ptrs.p[e] = dw_down[e];
+    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+  }
+  // 4. dgrad of gate_up: dx_perm = dh W1 (K = 2f)
+  {
+    GemmArgs g = gemm_args(ctx);
+    const bool ok =
+        map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dh_q) : w.dh, D.mx, 2 * f, D.cap, 2 * f * es) &&
+        map_3d(&g.tmap_b, w1c, D.mx, 2 * f, d, E, 2 * f * es, 2 * f * d * es);
+    if (!ok) return MOE_ERR_CUDA;
+    g.kgrouped = 0;
+    g.E = E;
+    g.K = static_cast<int>(2 * f);
+    g.n_tiles = static_cast<int>(d / 256);
+    g.poffsets = s.poff;
+    g.sfa = w.dh_s;
+    g.sfa_kb4 = 2 * f / 128;
+    g.sfb = s.w1c_s;
+    g.sfb_kb4 = 2 * f / 128;
+    g.sfb_expert_rows = d;
+    g.epi.out = w.dx_perm;
+    g.epi.ldo = d;
+    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+  }
+  // 5. wgrad of gate_up: dW1_e [2f, d] = dh_e^T x_e
+  {
+    GemmArgs g = gemm_args(ctx);
+    const bool ok =
+        map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dhT_q) : w.dhT, D.mx, D.cap, 2 * f, D.cap * es) &&
+        map_2d(&g.tmap_b, D.mx ? static_cast<const void*>(s.xT_q) : s.xT, D.mx, D.cap, d, D.cap * es);
+    if (!ok) return MOE_ERR_CUDA;
+    g.kgrouped = 1;
+    g.E = E;
+    g.m_tiles = static_cast<int>(2 * f / 128);
+    g.n_tiles = static_cast<int>(d / 256);
+    g.poffsets = s.poff;
+    g.sfa = w.dhT_s;
+    g.sfa_kb4 = D.cap / 128;
+    g.sfb = s.xT_s;
+    g.sfb_kb4 = D.cap / 128;
+    g.epi.ldo = d;
+    for (int e = 0; e < E; ++e) g.epi.out_ptrs.p[e] = dw_gate_up[e];
+    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+  }
+  // 6. combine dx, reduce the probability gradient
+  MOE_CUDA(launch_unpermute(w.dx_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(dx), ctx->num_sms, st));
+  MOE_CUDA(launch_dprob_reduce(w.dp_part, static_cast<int>(2 * (f / 256)), D.cap, s.src2s, D.Tk, d_topk_prob, st));
+  return MOE_OK;
+}
+
+void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
+                         int which, void* base, const char* name) {
+  if (!base || !name || check_dims(T, d, f, E, k) != MOE_OK) return nullptr;
+  const Dims D = make_dims(T, d, f, E, k, prec);
+  Carve c(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(base), 1024)));
+  struct Named {
+    const char* n;
+    void* p;
+  };
+  if (which == 0 || (which == 1 && !training)) {
+    Saved s;
+    if (which == 1) {
+      FwdWs w;
+      carve_fwd(c, D, w);
+    }
+    carve_saved(c, D, s, which == 0);
+    const Named tab[] = {{"split_sizes", s.split}, {"poffsets", s.poff}, {"sorted_to_src", s.s2src},
+                         {"src_to_sorted", s.src2s}, {"prob_perm", s.pperm}, {"w1c_q", s.w1c_q},
+                         {"w1c_s", s.w1c_s}, {"w2c_q", s.w2c_q}, {"w2c_s", s.w2c_s}, {"xT_q", s.xT_q},
+                         {"xT_s", s.xT_s}, {"aT_q", s.aT_q}, {"aT_s", s.aT_s}, {"xT", s.xT}, {"aT", s.aT},
+                         {"h", s.h}};
+    for (const Named& e : tab)
+      if (!std::strcmp(e.n, name) && e.p) return e.p;
+    if (which == 0) return nullptr;
+    c = Carve(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(base), 1024)));
+  }
+  if (which == 1) {
+    FwdWs w;
+    carve_fwd(c, D, w);
+    const Named tab[] = {{"w1_q", w.w1_q}, {"w1_s", w.w1_s}, {"w2_q", w.w2_q}, {"w2_s", w.w2_s},
+                         {"x_q", w.x_q},   {"x_s", w.x_s},   {"a_q", w.a_q},   {"a_s", w.a_s},
+                         {"x_perm", w.x_perm}, {"a", w.a}, {"y_perm", w.y_perm}};
+    for (const Named& e : tab)
+      if (!std::strcmp(e.n, name) && e.p) return e.p;
+    return nullptr;
+  }
+  if (which == 2) {
+    BwdWs w;
+    carve_bwd(c, D, w);
+    const Named tab[] = {{"dy_q", w.dy_q},   {"dy_s", w.dy_s},     {"dyT_q", w.dyT_q}, {"dyT_s", w.dyT_s},
+                         {"dh_q", w.dh_q},   {"dh_s", w.dh_s},     {"dhT_q", w.dhT_q}, {"dhT_s", w.dhT_s},
+                         {"dy_perm", w.dy_perm}, {"dyT", w.dyT},   {"dh", w.dh},       {"dhT", w.dhT},
+                         {"w1T", w.w1T},     {"w2T", w.w2T},       {"dx_perm", w.dx_perm},
+                         {"dp_part", w.dp_part}};
+    for (const Named& e : tab)
+      if (!std::strcmp(e.n, name) && e.p) return e.p;
+  }
+  return nullptr;
+}
+
+}  // extern "C"

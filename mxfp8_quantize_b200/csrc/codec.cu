@@ -1,0 +1,362 @@
+// HBM-bound kernels of the grouped MoE MLP: routing bookkeeping, MXFP8 quantisation (with the
+// token gather fused in), the bf16 gather/transpose used by the BF16 path, the combine of
+// expert rows back to tokens, and the reduction of the routing-probability gradient.
+#include <cuda_fp8.h>
+
+#include "codec.cuh"
+
+namespace moemx {
+
+// ------------------------------------------------------------------------------------------
+// Routing: stable counting sort of the T*k slots by expert (sitech.ge "Grouped experts instead
+// of a Python loop": per-expert token counts drive one grouped call).  One CTA of 1024 threads;
+// warp w owns a contiguous run of slots, so counting per (warp, expert) and an exclusive scan
+// over warps gives every slot its stable position without atomics.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024, 1)
+route_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_prob, int Tk, int E,
+             int capacity, const int32_t* __restrict__ split_in, int32_t* __restrict__ split_out,
+             int32_t* __restrict__ poffsets, int32_t* __restrict__ sorted_to_src, int32_t* __restrict__ src_to_sorted,
+             float* __restrict__ prob_perm, int* __restrict__ status) {
+  extern __shared__ int32_t sm[];      // [32][E] per-warp counts, then running bases
+  __shared__ int32_t s_poff[MOE_MAX_EXPERTS + 1];
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int32_t* wcnt = sm;
+
+  for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+  if (tid == 0) s_bad = 0;
+  for (int i = tid; i < capacity; i += blockDim.x) {
+    sorted_to_src[i] = -1;
+    if (prob_perm) prob_perm[i] = 0.f;
+  }
+  __syncthreads();
+
+  const int per_warp = static_cast<int>(round_up(ceil_div(Tk, 32), 32));
+  const int lo = warp * per_warp;
+  const int hi = min(Tk, lo + per_warp);
+  const unsigned lt_mask = (1u << lane) - 1u;
+
+  // pass 1: per-warp histograms
+  for (int base = lo; base < hi; base += 32) {
+    const int s = base + lane;
+    int e = -1;
+    if (s < hi) {
+      e = topk_idx[s];
+      if (e < 0 || e >= E) {
+        s_bad = 1;
+        e = -1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (peers & lt_mask) == 0) wcnt[warp * E + e] += __popc(peers);
+  }
+  __syncthreads();
+
+  // exclusive scan over warps per expert; totals
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = wcnt[w * E + e];
+      wcnt[w * E + e] = run;
+      run += c;
+    }
+    split_out[e] = run;
+    if (split_in && split_in[e] != run) s_bad = 1;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      s_poff[e] = acc;
+      acc += static_cast<int>(round_up(split_out[e], MOE_ROW_ALIGN));
+    }
+    s_poff[E] = acc;
+  }
+  __syncthreads();
+  for (int e = tid; e <= E; e += blockDim.x) poffsets[e] = s_poff[e];
+  if (tid == 0 && s_bad) atomicOr(status, kStatusDevice);
+
+  // pass 2: positions
+  for (int base = lo; base < hi; base += 32) {
+    const int s = base + lane;
+    int e = -1;
+    if (s < hi) {
+      e = topk_idx[s];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    int pos = -1;
+    if (e >= 0) pos = s_poff[e] + wcnt[warp * E + e] + __popc(peers & lt_mask);
+    __syncwarp();
+    if (e >= 0 && (peers & lt_mask) == 0) wcnt[warp * E + e] += __popc(peers);
+    __syncwarp();
+    if (e >= 0) {
+      sorted_to_src[pos] = s;
+      src_to_sorted[s] = pos;
+      if (prob_perm) prob_perm[pos] = topk_prob[s];
+    } else if (s < hi) {
+      src_to_sorted[s] = -1;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Quantise / gather / transpose tiles of 64 rows x 128 columns (256 threads).
+//   MXFP8 mode: row-wise codes + scales (blocks of 32 along a row) and column-wise codes +
+//               scales (blocks of 32 down a column) written transposed, from one read of x.
+//   BF16 mode:  the gathered rows copied, and/or written transposed.
+// The source row of output row r is r itself, or, when ``sorted_to_src`` is given, token
+// sorted_to_src[r] / k (padding rows, -1, read as zeros).
+// ------------------------------------------------------------------------------------------
+namespace {
+constexpr int QT_ROWS = 64;
+constexpr int QT_COLS = 128;
+constexpr int QT_PITCH = QT_COLS + 8;  // bf16 elements per smem row (padding against bank conflicts)
+
+__device__ __forceinline__ uint32_t abs_bits_bf16x2_max(uint32_t w, uint32_t m) {
+  const uint32_t lo = (w & 0x7FFFu) << 16;
+  const uint32_t hi = (w & 0x7FFF0000u);
+  return max(m, max(lo, hi));
+}
+
+// E4M3 codes of 8 values, packed little-endian into two 32-bit words.
+__device__ __forceinline__ uint2 e4m3x8(const float* v) {
+  uint2 out;
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * i], v[2 * i + 1]), __NV_SATFINITE, __NV_E4M3);
+    w[i] = static_cast<uint32_t>(p);
+  }
+  out.x = w[0] | (w[1] << 16);
+  out.y = w[2] | (w[3] << 16);
+  return out;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(256)
+quant_tile_kernel(QuantArgs a) {
+  __shared__ __align__(16) bf16 tile[QT_ROWS * QT_PITCH];
+  const int tid = threadIdx.x;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * QT_ROWS;
+  const int64_t col0 = static_cast<int64_t>(blockIdx.y) * QT_COLS;
+  const int b = blockIdx.z;
+  const int64_t R = a.rows, C = a.cols, KBr = C / 32, KBc = R / 32;
+
+  const bf16* src = a.src_ptrs.p[0] ? static_cast<const bf16*>(a.src_ptrs.p[b])
+                                    : static_cast<const bf16*>(a.src) + static_cast<int64_t>(b) * a.src_batch_stride;
+
+  // ---- load 64 x 128 (4 chunks of 8 bf16 per thread), row-wise quantise on the fly
+  const int cchunk = tid & 15;
+  const int64_t col = col0 + cchunk * 8;
+  const bool col_ok = col < C;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int lr = (tid >> 4) + 16 * i;
+    const int64_t r = row0 + lr;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    bool valid_row = r < R;
+    if (valid_row && col_ok) {
+      int64_t sr = r;
+      bool zero = false;
+      if (a.sorted_to_src) {
+        const int32_t s = a.sorted_to_src[r];
+        zero = s < 0;
+        sr = zero ? 0 : static_cast<int64_t>(s / a.k);
+      }
+      if (!zero) v = __ldg(reinterpret_cast<const uint4*>(src + sr * a.src_ld + col));
+    }
+    *reinterpret_cast<uint4*>(&tile[lr * QT_PITCH + cchunk * 8]) = v;
+
+    if (a.do_row) {
+      if (a.mx) {
+        uint32_t m = 0;
+        m = abs_bits_bf16x2_max(v.x, m);
+        m = abs_bits_bf16x2_max(v.y, m);
+        m = abs_bits_bf16x2_max(v.z, m);
+        m = abs_bits_bf16x2_max(v.w, m);
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        const uint32_t sb = e8m0_from_amax_bits(m);
+        const float inv = e8m0_inv_scale(sb);
+        if (valid_row && col_ok) {
+          float f[8];
+          const bf16* h = reinterpret_cast<const bf16*>(&v);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] = __bfloat162float(h[j]) * inv;
+          const uint2 q = e4m3x8(f);
+          uint8_t* qrow = a.q_row + (static_cast<int64_t>(b) * R + r) * C + col;
+          *reinterpret_cast<uint2*>(qrow) = q;
+          if ((cchunk & 3) == 0) {
+            const int64_t kb = col / 32;
+            const int64_t off = a.sf_mma ? sf_mma_offset(r, kb, KBr) : r * KBr + kb;
+            a.s_row[static_cast<int64_t>(b) * R * KBr + off] = static_cast<uint8_t>(sb);
+          }
+        }
+      } else if (valid_row && col_ok) {
+        *reinterpret_cast<uint4*>(a.o_row + (static_cast<int64_t>(b) * R + r) * C + col) = v;
+      }
+    }
+  }
+  if (!a.do_col) return;
+  __syncthreads();
+
+  // ---- column-wise: thread -> (column c, 32-row block rb)
+  const int c = tid & 127;
+  const int rb = tid >> 7;
+  const int64_t gc = col0 + c;
+  const int64_t gr = row0 + rb * 32;
+  if (gc >= C || gr >= R) return;
+  float f[32];
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const bf16 h = tile[(rb * 32 + i) * QT_PITCH + c];
+    f[i] = __bfloat162float(h);
+    m = max(m, __float_as_uint(f[i]) & 0x7FFFFFFFu);
+  }
+  if (a.mx) {
+    const uint32_t sb = e8m0_from_amax_bits(m);
+    const float inv = e8m0_inv_scale(sb);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) f[i] *= inv;
+    uint8_t* qc = a.q_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
+    uint4 w0, w1;
+    uint2 q0 = e4m3x8(f), q1 = e4m3x8(f + 8), q2 = e4m3x8(f + 16), q3 = e4m3x8(f + 24);
+    w0 = make_uint4(q0.x, q0.y, q1.x, q1.y);
+    w1 = make_uint4(q2.x, q2.y, q3.x, q3.y);
+    reinterpret_cast<uint4*>(qc)[0] = w0;
+    reinterpret_cast<uint4*>(qc)[1] = w1;
+    const int64_t kb = gr / 32;
+    const int64_t off = a.sf_mma ? sf_mma_offset(gc, kb, KBc) : gc * KBc + kb;
+    a.s_colT[static_cast<int64_t>(b) * C * KBc + off] = static_cast<uint8_t>(sb);
+  } else {
+    bf16* oc = a.o_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 w;
+      bf16* hw = reinterpret_cast<bf16*>(&w);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) hw[j] = tile[(rb * 32 + 8 * i + j) * QT_PITCH + c];
+      reinterpret_cast<uint4*>(oc)[i] = w;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Combine: y[t] = bf16(sum_j w_j * fp32(rows[row(t, j)])), j ascending, fp32 products and sums.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+unpermute_kernel(const bf16* __restrict__ rows, const int32_t* __restrict__ src_to_sorted,
+                 const float* __restrict__ probs, int64_t T, int k, int64_t d, bf16* __restrict__ y) {
+  const int64_t chunks = d / 8;
+  const int64_t total = T * chunks;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = i / chunks;
+    const int64_t c = (i - t * chunks) * 8;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int64_t r = src_to_sorted[t * k + j];
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(rows + r * d + c));
+      const bf16* h = reinterpret_cast<const bf16*>(&v);
+      if (probs) {
+        const float w = probs[t * k + j];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = __fadd_rn(acc[q], __fmul_rn(w, __bfloat162float(h[q])));
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = __fadd_rn(acc[q], __bfloat162float(h[q]));
+      }
+    }
+    uint4 o;
+    bf16* ho = reinterpret_cast<bf16*>(&o);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) ho[q] = __float2bfloat16_rn(acc[q]);
+    *reinterpret_cast<uint4*>(y + t * d + c) = o;
+  }
+}
+
+// d_topk_prob[t][j] = sum over n-tiles (ascending) of the partial row sums of the
+// ScaledSwiGLU probability gradient, read at row(t, j).
+__global__ void dprob_reduce_kernel(const float* __restrict__ part, int n_parts, int64_t part_stride,
+                                    const int32_t* __restrict__ src_to_sorted, int64_t Tk,
+                                    float* __restrict__ d_prob) {
+  for (int64_t s = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; s < Tk;
+       s += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = src_to_sorted[s];
+    float acc = 0.f;
+    for (int n = 0; n < n_parts; ++n) acc = __fadd_rn(acc, part[n * part_stride + r]);
+    d_prob[s] = acc;
+  }
+}
+
+// Row-wise MXFP8 -> fp32 (tests).
+__global__ void dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ s, int64_t R, int64_t C,
+                               int sf_mma, float* __restrict__ out) {
+  const int64_t KB = C / 32;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < R * C;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / C, c = i - r * C;
+    const int64_t kb = c / 32;
+    const uint8_t sb = s[sf_mma ? sf_mma_offset(r, kb, KB) : r * KB + kb];
+    const __nv_fp8_e4m3 v = *reinterpret_cast<const __nv_fp8_e4m3*>(q + i);
+    const float scale = sb == 255 ? __uint_as_float(0x7FC00000u) : (sb == 0 ? 0x1p-127f : __uint_as_float(static_cast<uint32_t>(sb) << 23));
+    out[i] = static_cast<float>(v) * scale;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// launchers
+// ------------------------------------------------------------------------------------------
+cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk, int E, int capacity,
+                         const int32_t* split_in, int32_t* split_out, int32_t* poffsets, int32_t* sorted_to_src,
+                         int32_t* src_to_sorted, float* prob_perm, int* status, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(32) * E * sizeof(int32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  route_kernel<<<1, 1024, smem, st>>>(topk_idx, topk_prob, Tk, E, capacity, split_in, split_out, poffsets,
+                                       sorted_to_src, src_to_sorted, prob_perm, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant(const QuantArgs& a, int batch, cudaStream_t st) {
+  if (a.rows == 0 || a.cols == 0 || batch == 0) return cudaSuccess;
+  dim3 grid(static_cast<unsigned>(ceil_div(a.rows, QT_ROWS)), static_cast<unsigned>(ceil_div(a.cols, QT_COLS)),
+            static_cast<unsigned>(batch));
+  quant_tile_kernel<<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute(const bf16* rows, const int32_t* src_to_sorted, const float* probs, int64_t T, int k,
+                             int64_t d, bf16* y, int num_sms, cudaStream_t st) {
+  const int64_t total = T * (d / 8);
+  if (total == 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), static_cast<int64_t>(num_sms) * 16);
+  unpermute_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(rows, src_to_sorted, probs, T, k, d, y);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_stride, const int32_t* src_to_sorted,
+                                int64_t Tk, float* d_prob, cudaStream_t st) {
+  if (Tk == 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>(ceil_div(Tk, 256), 4096);
+  dprob_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(part, n_parts, part_stride, src_to_sorted, Tk,
+                                                                      d_prob);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(const uint8_t* q, const uint8_t* s, int64_t R, int64_t C, int sf_mma, float* out,
+                           int num_sms, cudaStream_t st) {
+  if (R * C == 0) return cudaSuccess;
+  const int64_t blocks = std::min<int64_t>(ceil_div(R * C, 256), static_cast<int64_t>(num_sms) * 16);
+  dequant_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(q, s, R, C, sf_mma, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moemx

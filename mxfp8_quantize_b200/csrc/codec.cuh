@@ -1,0 +1,41 @@
+// Declarations of the HBM-bound kernels' launchers (codec.cu).
+#pragma once
+#include "common.cuh"
+
+namespace moemx {
+
+struct PtrArray {
+  const void* p[MOE_MAX_EXPERTS];
+};
+
+// One quantise / gather / transpose pass over a [batch, rows, cols] bf16 source.
+struct QuantArgs {
+  const bf16* src;             // batch 0 source (when src_ptrs.p[0] is null)
+  int64_t src_batch_stride;    // elements between batches of ``src``
+  int64_t src_ld;              // elements between source rows
+  PtrArray src_ptrs;           // per-batch sources (expert weights), or all null
+  const int32_t* sorted_to_src;  // gather: output row r reads token sorted_to_src[r] / k (-1: zeros)
+  int k;
+  int64_t rows, cols;          // output rows and columns per batch
+  int mx;                      // 1: MXFP8 codes + scales; 0: bf16 copies
+  int do_row, do_col, sf_mma;
+  uint8_t* q_row;
+  uint8_t* s_row;
+  uint8_t* q_colT;
+  uint8_t* s_colT;
+  bf16* o_row;
+  bf16* o_colT;
+};
+
+cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk, int E, int capacity,
+                         const int32_t* split_in, int32_t* split_out, int32_t* poffsets, int32_t* sorted_to_src,
+                         int32_t* src_to_sorted, float* prob_perm, int* status, cudaStream_t st);
+cudaError_t launch_quant(const QuantArgs& a, int batch, cudaStream_t st);
+cudaError_t launch_unpermute(const bf16* rows, const int32_t* src_to_sorted, const float* probs, int64_t T, int k,
+                             int64_t d, bf16* y, int num_sms, cudaStream_t st);
+cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_stride, const int32_t* src_to_sorted,
+                                int64_t Tk, float* d_prob, cudaStream_t st);
+cudaError_t launch_dequant(const uint8_t* q, const uint8_t* s, int64_t R, int64_t C, int sf_mma, float* out,
+                           int num_sms, cudaStream_t st);
+
+}  // namespace moemx

@@ -1,0 +1,57 @@
+// Grouped GEMM on the sm_100a tensor cores (tcgen05) with fused epilogues.
+#pragma once
+#include <cuda.h>
+
+#include "codec.cuh"
+
+namespace moemx {
+
+enum EpiKind : int {
+  EPI_STORE = 0,    // fp32 accumulator -> bf16 rows
+  EPI_SWIGLU = 1,   // gate/up accumulator -> a = silu(g)*u*p, requantised (ScaledSwiGLU)
+  EPI_DSWIGLU = 2,  // da accumulator + saved h -> dh = [dg, du] requantised, dp partial sums
+};
+
+struct EpiArgs {
+  // EPI_STORE
+  bf16* out;          // M-grouped: [rows, ldo]
+  int64_t ldo;
+  PtrArray out_ptrs;  // K-grouped: per-expert outputs [M, ldo]
+  // EPI_SWIGLU / EPI_DSWIGLU
+  int64_t f;          // ffn width
+  int64_t cap;        // padded row capacity (token axis of the transposed outputs)
+  const float* p_perm;
+  bf16* h;            // [cap, 2f] saved gate/up pre-activations (written by SWIGLU, read by DSWIGLU)
+  uint8_t* q_row;     // MXFP8 row-wise codes ([cap, f] for a, [cap, 2f] for dh)
+  uint8_t* s_row;     // their scales, tensor-core tile layout
+  uint8_t* q_colT;    // MXFP8 codes transposed ([f, cap] / [2f, cap])
+  uint8_t* s_colT;
+  bf16* o_row;        // BF16 path equivalents
+  bf16* o_colT;
+  float* dump;        // debug: fp32 values before quantisation
+  float* dp_part;     // DSWIGLU: [2 * n_tiles, cap] partial sums of the probability gradient
+};
+
+struct GemmArgs {
+  CUtensorMap tmap_a;  // A: 2-D [rows, K] K-contiguous, box 128 rows x 128 bytes, 128B swizzle
+  CUtensorMap tmap_b;  // B: 3-D [E, rows, K] (M-grouped) or 2-D [rows, K] (K-grouped)
+  int kgrouped;        // 0: M grouped by expert (rows of A = expert segments); 1: K grouped (wgrad)
+  int E;
+  int K;               // M-grouped reduction length
+  int n_tiles;         // output tiles along N per expert
+  int m_tiles;         // K-grouped: M / 128
+  int gate_up_half;    // M-grouped SWIGLU: f (B rows of the up half start at f); else 0
+  const int32_t* poffsets;
+  const uint8_t* sfa;  // MXFP8 scales of A / B in the tile layout
+  int64_t sfa_kb4;     // 128-wide K blocks per 128-row block of A's scales
+  const uint8_t* sfb;
+  int64_t sfb_kb4;
+  int64_t sfb_expert_rows;  // rows of B per expert (M-grouped), for the scale tile index
+  int* status;
+  EpiArgs epi;
+};
+
+// Launch one grouped GEMM.  ``mx``: MXFP8 (kind::mxf8f6f4) or BF16 (kind::f16).
+cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st);
+
+}  // namespace moemx
