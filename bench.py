@@ -1,0 +1,404 @@
+"""Benchmark of the grouped MoE expert MLP (forward + backward) on B200.
+
+A step is one training pass of the whole hot path over one batch of synthetic input: per-step
+MXFP8 quantisation of the bf16 master weights, routing, permute + quantise, the gate_up GEMM
+with the fused ScaledSwiGLU requantisation, the down GEMM, the combine, and the backward
+(dgrad + dSwiGLU, both wgrads, dgrad of gate_up, combine of dx, probability gradient).
+
+Default workload: the Mixtral-8x7B layer shape in MXFP8 (T=8192 tokens, d=4096, f=14336,
+E=8 experts, top-2).  ``value`` is algorithmic TFLOP/s (18*T*k*d*f per step, padding excluded)
+with inputs resident in HBM; ``e2e`` is the same metric through the public API with host
+buffers (inputs copied in from pinned memory and outputs copied back inside the timed region).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+With --gpus N > 1 (under torchrun) every rank runs an independent replica of the layer (the
+single-layer path has no exchange step), and the job value is the sum over ranks with the time
+taken as the max over ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from mxfp8_quantize_b200 import workloads  # noqa: E402
+
+METRIC = "grouped MoE MLP fwd+bwd TFLOP/s and tokens/s (MXFP8, BF16) vs tensor peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------------------ per-kernel work
+def kernel_work(cfg, name):
+    """(kind, algorithmic amount per launch): FLOPs for GEMMs, bytes for the HBM-bound kernels."""
+    Tk, T, d, f, E, k = cfg.Tk, cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
+    mx = cfg.precision == "mxfp8"
+    q = 1.0 + 1.0 / 32  # bytes per quantised element (code + its share of a scale)
+    gemm = {
+        "gemm_gate_up_swiglu": 2.0 * Tk * d * 2 * f,
+        "gemm_down": 2.0 * Tk * f * d,
+        "gemm_dgrad_down_dswiglu": 2.0 * Tk * d * f,
+        "gemm_wgrad_down": 2.0 * Tk * d * f,
+        "gemm_dgrad_gate_up": 2.0 * Tk * 2 * f * d,
+        "gemm_wgrad_gate_up": 2.0 * Tk * 2 * f * d,
+    }
+    if name in gemm:
+        return "tensor", gemm[name]
+    out_b = 2 * q if mx else 4.0  # row + column outputs per element
+    hbm = {
+        "quantize_w_gate_up": E * 2 * f * d * (2 + out_b),
+        "quantize_w_down": E * d * f * (2 + out_b),
+        "permute_quantize_x": T * d * 2 + Tk * d * out_b,
+        "permute_x": T * d * 2 + Tk * d * out_b,
+        "gather_quantize_dy": T * d * 2 + Tk * d * out_b,
+        "transpose_w_gate_up": E * 2 * f * d * 4,
+        "transpose_w_down": E * d * f * 4,
+        "unpermute_y": Tk * d * 2 + T * d * 2 + Tk * 4,
+        "unpermute_dx": Tk * d * 2 + T * d * 2 + Tk * 4,
+        "route": Tk * 4 * 3,
+        "dprob_reduce": Tk * 4 * 2,
+    }
+    return "hbm", hbm.get(name, 0.0)
+
+
+# ------------------------------------------------------------------------------ clocks
+REASON_FIELDS = ["clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                 "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," + ",".join(REASON_FIELDS)
+        try:
+            self.f = open(self.path, "w")
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100",
+                                       "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        for line in open(self.path):
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) < 5 + len(REASON_FIELDS):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(REASON_FIELDS, parts[5:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name.split(".")[1])
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(cfg, m_tokens: int, f_slab: int):
+    """A bounded slice of the workload for the CPU oracle: expert 0 of the layer with the first
+    ``m_tokens`` slots routed to it and a slab of ``f_slab`` ffn columns (gate and up halves),
+    forward + backward with the workload's precision.  Returns (callable, flops, description)."""
+    from mxfp8_quantize_b200.workloads import _normal_bf16
+    rng = np.random.default_rng(cfg.seed)
+    d = cfg.d
+    std1 = cfg.w_std if cfg.w_std is not None else 1.0 / np.sqrt(d)
+    std2 = cfg.w_std if cfg.w_std is not None else 1.0 / np.sqrt(cfg.f)
+    x = _normal_bf16(rng, (m_tokens, d), 1.0).float().numpy()
+    w1 = _normal_bf16(rng, (1, 2 * f_slab, d), float(std1)).float().numpy()
+    w2 = _normal_bf16(rng, (1, d, f_slab), float(std2)).float().numpy()
+    dy = _normal_bf16(rng, (m_tokens, d), 1.0).float().numpy()
+    prob = rng.uniform(0.05, 0.95, (m_tokens, 1)).astype(np.float32)
+    idx = np.zeros((m_tokens, 1), dtype=np.int32)
+
+    def run():
+        from oracle import moe as omoe
+        y, st = omoe.forward(x, idx, prob, w1, w2, cfg.precision)
+        omoe.backward(dy, st, w1, w2)
+
+    flops = 18.0 * m_tokens * d * f_slab
+    desc = (f"oracle fwd+bwd ({cfg.precision}) of one expert of the {cfg.name} layer: {m_tokens} routed slots, "
+            f"d={d}, a {f_slab}-column ffn slab (gate+up {2 * f_slab} rows), incl. that slab's weight quantisation")
+    return run, flops, desc
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def time_oracle(cfg, m_tokens, f_slab, repeats):
+    run, flops, desc = oracle_sample(cfg, m_tokens, f_slab)
+    ts = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        run()
+        ts.append(time.perf_counter() - t0)
+    return flops, ts, desc
+
+
+# ------------------------------------------------------------------------------ GPU arm
+def run_ours(args, cfg, rank, world, local_rank):
+    import mxfp8_quantize_b200 as moe
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = workloads.make_inputs(cfg, with_dy=True)
+    x = inp["x"].to(dev)
+    idx = inp["topk_idx"].to(dev)
+    prob = inp["topk_prob"].to(dev)
+    dy = inp["dy"].to(dev)
+    w1 = inp["w_gate_up"].to(dev)
+    w2 = inp["w_down"].to(dev)
+    T, d, f, E, k = cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
+    sz = moe.sizes(T, d, f, E, k, cfg.precision, True)
+    fws = torch.empty(sz["fwd_ws"], dtype=torch.uint8, device=dev)
+    bws = torch.empty(sz["bwd_ws"], dtype=torch.uint8, device=dev)
+    saved = moe.Saved(torch.empty(sz["saved"], dtype=torch.uint8, device=dev), (T, d, f, E, k, cfg.precision))
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty_like(y)
+    dw1 = torch.empty_like(w1)
+    dw2 = torch.empty_like(w2)
+    dp = torch.empty((T, k), dtype=torch.float32, device=dev)
+
+    def step(xi, idxi, probi, dyi):
+        moe.moe_grouped_mlp_fwd(xi, idxi, probi, w1, w2, precision=cfg.precision, training=True, workspace=fws,
+                                saved=saved, y=y)
+        moe.moe_grouped_mlp_bwd(dyi, saved, w1, w2, workspace=bws, dx=dx, dw_gate_up=dw1, dw_down=dw2,
+                                d_topk_prob=dp)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step(x, idx, prob, dy)
+    moe.get_status(local_rank)
+
+    # ---- timed region: device-resident inputs; every kernel bracketed by events on its stream
+    records = []
+    stream = torch.cuda.current_stream(dev)
+
+    def hook(name, after):
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        records.append((name, after, ev))
+
+    clocks = ClockSampler(local_rank if world > 1 else (torch.cuda.current_device()))
+    barrier()
+    torch.cuda.synchronize(dev)
+    moe.set_launch_hook(local_rank, hook)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(x, idx, prob, dy)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    moe.set_launch_hook(local_rank, None)
+    barrier()
+    clk = clocks.stop()
+    moe.get_status(local_rank)
+    ms = t0.elapsed_time(t1) / args.steps
+    launches = sum(1 for r in records if not r[1])
+
+    # per-kernel averages
+    per = {}
+    open_ev = {}
+    for name, after, ev in records:
+        if not after:
+            open_ev[name] = ev
+        else:
+            per.setdefault(name, []).append(open_ev.pop(name).elapsed_time(ev))
+    kern = {}
+    peaks, peak_src = load_peaks()
+    mx = cfg.precision == "mxfp8"
+    tensor_peak = peaks["bf16_tflops_sustained"] * (2.0 if mx else 1.0)
+    for name, v in per.items():
+        avg = float(np.mean(v))
+        kind, work = kernel_work(cfg, name)
+        if kind == "tensor":
+            ach = work / (avg * 1e-3) / 1e12
+            kern[name] = {"ms": round(avg, 4), "launches": len(v), "tflops": round(ach, 1),
+                          "frac": round(ach / tensor_peak, 4)}
+        else:
+            ach = work / (avg * 1e-3) / 1e9
+            kern[name] = {"ms": round(avg, 4), "launches": len(v), "gbs": round(ach, 1),
+                          "frac": round(ach / peaks["hbm_gbs"], 4)}
+    dom = max(per, key=lambda n: sum(per[n]))
+    kind, work = kernel_work(cfg, dom)
+    avg = float(np.mean(per[dom]))
+    if kind == "tensor":
+        achieved, peak, unit = work / (avg * 1e-3) / 1e12, tensor_peak, "TFLOP/s"
+    else:
+        achieved, peak, unit = work / (avg * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        traffic = json.load(open(tpath)).get(cfg.name, {}).get(dom)
+    roofline = {"bound": kind, "kernel": dom, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": (f"{peak_src}: bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s"
+                                + (" x 2 (nominal fp8/bf16 ratio)" if mx and kind == "tensor" else "")
+                                if kind == "tensor" else f"{peak_src}: HBM copy {peaks['hbm_gbs']} GB/s")}
+
+    # ---- e2e: through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hx = inp["x"].pin_memory()
+        hidx = inp["topk_idx"].pin_memory()
+        hprob = inp["topk_prob"].pin_memory()
+        hdy = inp["dy"].pin_memory()
+        oy = torch.empty_like(hx).pin_memory()
+        odx = torch.empty_like(hx).pin_memory()
+        odp = torch.empty((T, k), dtype=torch.float32).pin_memory()
+        dx_in = torch.empty_like(x)
+        didx = torch.empty_like(idx)
+        dprob = torch.empty_like(prob)
+        ddy = torch.empty_like(dy)
+        h2d = sum(t.numel() * t.element_size() for t in (hx, hidx, hprob, hdy))
+        d2h = sum(t.numel() * t.element_size() for t in (oy, odx, odp))
+        n2 = max(1, min(args.steps, 20))
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n2):
+            dx_in.copy_(hx, non_blocking=True)
+            didx.copy_(hidx, non_blocking=True)
+            dprob.copy_(hprob, non_blocking=True)
+            ddy.copy_(hdy, non_blocking=True)
+            step(dx_in, didx, dprob, ddy)
+            oy.copy_(y, non_blocking=True)
+            odx.copy_(dx, non_blocking=True)
+            odp.copy_(dp, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms_e2e = e0.elapsed_time(e1) / n2
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": round(world * cfg.flops_fwd_bwd() / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "ms_per_step": round(ms_e2e, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "tokens_per_s": round(world * T / (ms_e2e * 1e-3), 1)}
+
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return dict(ms=ms, kernels=kern, roofline=roofline, clocks=clk, e2e=e2e, launches=launches)
+
+
+def config_desc(cfg):
+    return {"workload": f"{cfg.name}: T={cfg.T} d={cfg.d} f={cfg.f} E={cfg.E} top-{cfg.k}, {cfg.precision} "
+                        f"fwd+bwd incl. per-step weight quantisation, {cfg.routing} routing",
+            "tokens": cfg.T, "d": cfg.d, "f": cfg.f, "experts": cfg.E, "top_k": cfg.k,
+            "l2": "inputs larger than L2 (bf16 master weights and their MXFP8 copies are GBs)",
+            "parallelism": "replicas (one independent layer per GPU)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="mixtral_mxfp8", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling cases)")
+    ap.add_argument("--experts", type=int, default=None, help="override E (profiling cases)")
+    args = ap.parse_args()
+    cfg = workloads.CONFIGS[args.config]
+    if args.tokens or args.experts:
+        cfg = workloads.scaled_config(cfg, T=args.tokens or cfg.T, E=args.experts or cfg.E,
+                                      name=f"{cfg.name}[T={args.tokens or cfg.T},E={args.experts or cfg.E}]")
+    if not cfg.backward:
+        cfg = workloads.scaled_config(cfg, backward=True)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        # per step: a bounded slice sized so that the whole run stays within a few minutes
+        m, fs = 256, 256
+        for _ in range(args.warmup):
+            time_oracle(cfg, m, fs, 1)
+        flops, ts, desc = time_oracle(cfg, m, fs, args.steps)
+        sec = float(np.sum(ts))
+        val = flops * args.steps / sec / 1e12
+        line = {"metric": METRIC, "value": round(val, 5), "unit": "TFLOP/s", "impl": "reference",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1e3 * sec / args.steps, 2), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_desc(cfg),
+                "cpu_baseline": {"value": round(val, 5), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": round(val, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    res = run_ours(args, cfg, rank, world, local_rank)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    tflops = world * cfg.flops_fwd_bwd() / (res["ms"] * 1e-3) / 1e12
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        flops, ts, desc = time_oracle(cfg, 2048, 512, 2)
+        cpu = {"value": round(flops / float(np.median(ts)) / 1e12, 5), "unit": "TFLOP/s", "cores": cpu_threads(),
+               "kind": "oracle", "sample": desc + f"; median of {len(ts)} runs of {float(np.median(ts)):.1f} s"}
+    line = {"metric": METRIC, "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(res["ms"], 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "mxfp8-e4m3 (fp32 accumulate)" if cfg.precision == "mxfp8" else "bf16",
+            "data": "synthetic", "config": config_desc(cfg),
+            "tokens_per_s": round(world * cfg.T / (res["ms"] * 1e-3), 1),
+            "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["launches"],
+            "clocks": res["clocks"], "kernels": res["kernels"]}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

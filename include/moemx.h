@@ -82,6 +82,13 @@ moe_status_t moe_ctx_set_debug_dump(moe_ctx_t ctx, float* a_f32, float* dh_f32);
 
 const char* moe_status_string(moe_status_t s);
 
+/* Launch hook (profiling).  When set, the fused-layer and codec entry points call
+ * hook(user, kernel_name, 0, stream) just before and hook(user, kernel_name, 1, stream) just
+ * after enqueueing each of their kernels, on the host thread that made the call, so a caller can
+ * record CUDA events around every kernel on the stream it runs on.  NULL switches it off. */
+typedef void (*moe_launch_hook_t)(void* user, const char* kernel, int after, void* stream);
+moe_status_t moe_ctx_set_launch_hook(moe_ctx_t ctx, moe_launch_hook_t hook, void* user);
+
 /* ---------------------------------------------------------------------------------------
  * mxfp8_quantize: bf16 -> MXFP8 (sitech.ge "Memory and quantization overhead": one scale per
  * block of 32 consecutive values; ai4snews paragraph 2).

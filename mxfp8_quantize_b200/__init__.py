@@ -29,7 +29,9 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "unsupported", 4: "cuda
 EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_get_status", "moe_ctx_set_debug_dump", "moe_status_string",
            "mxfp8_quantize", "mxfp8_dequantize", "moe_capacity_rows", "moe_permute", "moe_unpermute",
            "moe_saved_size", "moe_fwd_workspace_size", "moe_bwd_workspace_size", "moe_grouped_mlp_fwd",
-           "moe_grouped_mlp_bwd", "moe_buffer_address"]
+           "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook"]
+
+LAUNCH_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
 
 class MoeError(RuntimeError):
@@ -71,6 +73,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                         c_int, c_int, c_vp, c_vp, c_size, c_vp, c_size, c_vp]),
         "moe_grouped_mlp_bwd": (c_int, [c_vp, c_vp, c_vp, c_size, c_vp, c_vp, c_i64, c_i64, c_i64, c_int, c_int,
                                         c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
+        "moe_ctx_set_launch_hook": (c_int, [c_vp, LAUNCH_HOOK, c_vp]),
         "moe_buffer_address": (c_vp, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int, c_int, c_vp,
                                       ctypes.c_char_p]),
     }
@@ -120,6 +123,22 @@ def get_status(device: int = 0):
 def set_debug_dump(device: int, a_f32: Optional[torch.Tensor], dh_f32: Optional[torch.Tensor]):
     L = load_library()
     _check("moe_ctx_set_debug_dump", L.moe_ctx_set_debug_dump(context(device), _ptr(a_f32), _ptr(dh_f32)))
+
+
+_hooks = {}
+
+
+def set_launch_hook(device: int, fn):
+    """fn(kernel_name: str, after: bool) is called around every kernel the library enqueues on
+    ``device`` (None switches it off).  Used to time kernels with CUDA events."""
+    L = load_library()
+    if fn is None:
+        _hooks.pop(device, None)
+        _check("moe_ctx_set_launch_hook", L.moe_ctx_set_launch_hook(context(device), LAUNCH_HOOK(), None))
+        return
+    cb = LAUNCH_HOOK(lambda user, name, after, stream: fn(name.decode(), bool(after)))
+    _hooks[device] = cb
+    _check("moe_ctx_set_launch_hook", L.moe_ctx_set_launch_hook(context(device), cb, None))
 
 
 def capacity_rows(T: int, k: int, E: int) -> int:

@@ -19,6 +19,8 @@ struct moe_ctx_s {
   int* d_status;  // [0] status bits
   float* dbg_a;
   float* dbg_dh;
+  moe_launch_hook_t hook;
+  void* hook_user;
 };
 
 namespace {
@@ -215,6 +217,15 @@ struct DeviceGuard {
     if ((x) != cudaSuccess) return MOE_ERR_CUDA; \
   } while (0)
 
+// Enqueue one kernel, calling the context's launch hook around it.
+#define MOE_LAUNCH(ctx, name, st, x)                                          \
+  do {                                                                        \
+    if ((ctx)->hook) (ctx)->hook((ctx)->hook_user, name, 0, (void*)(st));     \
+    const cudaError_t moe_launch_err_ = (x);                                  \
+    if ((ctx)->hook) (ctx)->hook((ctx)->hook_user, name, 1, (void*)(st));     \
+    if (moe_launch_err_ != cudaSuccess) return MOE_ERR_CUDA;                  \
+  } while (0)
+
 // Uniform byte stride between consecutive expert pointers (0 if not uniform / not usable by TMA).
 int64_t uniform_stride(const void* const* p, int E, int64_t min_bytes) {
   if (E == 1) return min_bytes;
@@ -270,6 +281,8 @@ moe_status_t moe_ctx_create(moe_ctx_t* out, int device) {
   c->device = device;
   c->num_sms = prop.multiProcessorCount;
   c->dbg_a = c->dbg_dh = nullptr;
+  c->hook = nullptr;
+  c->hook_user = nullptr;
   if (cudaMalloc(&c->d_status, 256) != cudaSuccess) {
     delete c;
     return MOE_ERR_CUDA;
@@ -295,6 +308,13 @@ moe_status_t moe_ctx_set_debug_dump(moe_ctx_t ctx, float* a_f32, float* dh_f32) 
   if (!ctx) return MOE_ERR_INVALID_ARG;
   ctx->dbg_a = a_f32;
   ctx->dbg_dh = dh_f32;
+  return MOE_OK;
+}
+
+moe_status_t moe_ctx_set_launch_hook(moe_ctx_t ctx, moe_launch_hook_t hook, void* user) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  ctx->hook = hook;
+  ctx->hook_user = user;
   return MOE_OK;
 }
 
@@ -344,7 +364,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
   a.s_row = s_row;
   a.q_colT = q_colT;
   a.s_colT = s_colT;
-  MOE_CUDA(launch_quant(a, static_cast<int>(batch), static_cast<cudaStream_t>(stream)));
+  MOE_LAUNCH(ctx, "mxfp8_quantize", stream, launch_quant(a, static_cast<int>(batch), static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 
@@ -354,7 +374,7 @@ moe_status_t mxfp8_dequantize(moe_ctx_t ctx, const uint8_t* q, const uint8_t* s,
   if (cols % 32) return MOE_ERR_SHAPE;
   if (sf_mma_layout && (rows % 128 || cols % 128)) return MOE_ERR_SHAPE;
   DeviceGuard guard(ctx->device);
-  MOE_CUDA(launch_dequant(q, s, rows, cols, sf_mma_layout, out, ctx->num_sms, static_cast<cudaStream_t>(stream)));
+  MOE_LAUNCH(ctx, "mxfp8_dequantize", stream, launch_dequant(q, s, rows, cols, sf_mma_layout, out, ctx->num_sms, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 
@@ -372,7 +392,7 @@ moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, 
   if (cap >= (int64_t(1) << 31) / 2) return MOE_ERR_UNSUPPORTED;
   DeviceGuard guard(ctx->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  MOE_CUDA(launch_route(topk_idx, topk_prob, static_cast<int>(T * k), E, static_cast<int>(cap), split_sizes_in,
+  MOE_LAUNCH(ctx, "route", st, launch_route(topk_idx, topk_prob, static_cast<int>(T * k), E, static_cast<int>(cap), split_sizes_in,
                         split_sizes, poffsets, sorted_to_src, src_to_sorted, prob_perm, ctx->d_status, st));
   if (x) {
     QuantArgs a = quant_args();
@@ -385,7 +405,7 @@ moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, 
     a.mx = 0;
     a.do_row = 1;
     a.o_row = static_cast<bf16*>(x_perm);
-    MOE_CUDA(launch_quant(a, 1, st));
+    MOE_LAUNCH(ctx, "permute_x", st, launch_quant(a, 1, st));
   }
   return MOE_OK;
 }
@@ -397,7 +417,7 @@ moe_status_t moe_unpermute(moe_ctx_t ctx, const void* y_perm, const int32_t* src
   if (d % 8) return MOE_ERR_SHAPE;
   if (!aligned16(y_perm) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->device);
-  MOE_CUDA(launch_unpermute(static_cast<const bf16*>(y_perm), src_to_sorted, probs, T, k, d, static_cast<bf16*>(y),
+  MOE_LAUNCH(ctx, "unpermute", stream, launch_unpermute(static_cast<const bf16*>(y_perm), src_to_sorted, probs, T, k, d, static_cast<bf16*>(y),
                             ctx->num_sms, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
@@ -464,7 +484,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
   }
 
   // 1. routing: counts, padded offsets, stable permutation, per-row probabilities
-  MOE_CUDA(launch_route(topk_idx, topk_prob, static_cast<int>(D.Tk), E, static_cast<int>(D.cap), split_sizes, s.split,
+  MOE_LAUNCH(ctx, "route", st, launch_route(topk_idx, topk_prob, static_cast<int>(D.Tk), E, static_cast<int>(D.cap), split_sizes, s.split,
                         s.poff, s.s2src, s.src2s, s.pperm, ctx->d_status, st));
 
   // 2. operands of the gate_up GEMM
@@ -487,7 +507,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     a.do_col = training;
     a.q_colT = s.w1c_q;
     a.s_colT = s.w1c_s;
-    MOE_CUDA(launch_quant(a, E, st));
+    MOE_LAUNCH(ctx, "quantize_w_gate_up", st, launch_quant(a, E, st));
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
     a.src_ld = f;
     a.rows = d;
@@ -496,7 +516,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     a.s_row = w.w2_s;
     a.q_colT = s.w2c_q;
     a.s_colT = s.w2c_s;
-    MOE_CUDA(launch_quant(a, E, st));
+    MOE_LAUNCH(ctx, "quantize_w_down", st, launch_quant(a, E, st));
     w1_base = w.w1_q;
     w1_stride = 2 * f * d;
     w2_base = w.w2_q;
@@ -518,7 +538,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.do_col = training;
     xa.q_colT = s.xT_q;
     xa.s_colT = s.xT_s;
-    MOE_CUDA(launch_quant(xa, 1, st));
+    MOE_LAUNCH(ctx, "permute_quantize_x", st, launch_quant(xa, 1, st));
   } else {
     w1_stride = uniform_stride(w_gate_up, E, 2 * f * d * 2);
     w2_stride = uniform_stride(w_down, E, d * f * 2);
@@ -533,7 +553,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       a.rows = 2 * f;
       a.cols = d;
       a.o_row = w.w1_copy;
-      MOE_CUDA(launch_quant(a, E, st));
+      MOE_LAUNCH(ctx, "gather_w_gate_up", st, launch_quant(a, E, st));
       w1_base = w.w1_copy;
       w1_stride = 2 * f * d * 2;
     }
@@ -543,7 +563,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       a.rows = d;
       a.cols = f;
       a.o_row = w.w2_copy;
-      MOE_CUDA(launch_quant(a, E, st));
+      MOE_LAUNCH(ctx, "gather_w_down", st, launch_quant(a, E, st));
       w2_base = w.w2_copy;
       w2_stride = d * f * 2;
     }
@@ -559,7 +579,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.o_row = w.x_perm;
     xa.do_col = training;
     xa.o_colT = s.xT;
-    MOE_CUDA(launch_quant(xa, 1, st));
+    MOE_LAUNCH(ctx, "permute_x", st, launch_quant(xa, 1, st));
   }
 
   // 3. gate_up GEMM + ScaledSwiGLU + requantisation of a
@@ -595,7 +615,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       ep.o_row = w.a;
       ep.o_colT = training ? s.aT : nullptr;
     }
-    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_SWIGLU, ctx->num_sms, st));
+    MOE_LAUNCH(ctx, "gemm_gate_up_swiglu", st, launch_grouped_gemm(g, D.mx, EPI_SWIGLU, ctx->num_sms, st));
   }
   // 4. down GEMM
   {
@@ -616,10 +636,10 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     g.sfb_expert_rows = d;
     g.epi.out = w.y_perm;
     g.epi.ldo = d;
-    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+    MOE_LAUNCH(ctx, "gemm_down", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
   }
   // 5. combine (probabilities were applied in ScaledSwiGLU)
-  MOE_CUDA(launch_unpermute(w.y_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(y), ctx->num_sms, st));
+  MOE_LAUNCH(ctx, "unpermute_y", st, launch_unpermute(w.y_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(y), ctx->num_sms, st));
   return MOE_OK;
 }
 
@@ -673,7 +693,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
       a.o_row = w.dy_perm;
       a.o_colT = w.dyT;
     }
-    MOE_CUDA(launch_quant(a, 1, st));
+    MOE_LAUNCH(ctx, "gather_quantize_dy", st, launch_quant(a, 1, st));
   }
   const void* w1c;  // B of dgrad of gate_up: [E, d, 2f]
   const void* w2c;  // B of dgrad of down:    [E, f, d]
@@ -689,13 +709,13 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     a.rows = 2 * f;
     a.cols = d;
     a.o_colT = w.w1T;
-    MOE_CUDA(launch_quant(a, E, st));
+    MOE_LAUNCH(ctx, "transpose_w_gate_up", st, launch_quant(a, E, st));
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
     a.src_ld = f;
     a.rows = d;
     a.cols = f;
     a.o_colT = w.w2T;
-    MOE_CUDA(launch_quant(a, E, st));
+    MOE_LAUNCH(ctx, "transpose_w_down", st, launch_quant(a, E, st));
     w1c = w.w1T;
     w2c = w.w2T;
   }
@@ -732,7 +752,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
       ep.o_row = w.dh;
       ep.o_colT = w.dhT;
     }
-    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_DSWIGLU, ctx->num_sms, st));
+    MOE_LAUNCH(ctx, "gemm_dgrad_down_dswiglu", st, launch_grouped_gemm(g, D.mx, EPI_DSWIGLU, ctx->num_sms, st));
   }
   // 3. wgrad of down: dW2_e [d, f] = dy_e^T a_e (K = the expert's tokens)
   {
@@ -752,7 +772,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     g.sfb_kb4 = D.cap / 128;
     g.epi.ldo = f;
     for (int e = 0; e < E; ++e) g.epi.out_ptrs.p[e] = dw_down[e];
-    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+    MOE_LAUNCH(ctx, "gemm_wgrad_down", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
   }
   // 4. dgrad of gate_up: dx_perm = dh W1 (K = 2f)
   {
@@ -773,7 +793,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     g.sfb_expert_rows = d;
     g.epi.out = w.dx_perm;
     g.epi.ldo = d;
-    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+    MOE_LAUNCH(ctx, "gemm_dgrad_gate_up", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
   }
   // 5. wgrad of gate_up: dW1_e [2f, d] = dh_e^T x_e
   {
@@ -793,11 +813,11 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     g.sfb_kb4 = D.cap / 128;
     g.epi.ldo = d;
     for (int e = 0; e < E; ++e) g.epi.out_ptrs.p[e] = dw_gate_up[e];
-    MOE_CUDA(launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+    MOE_LAUNCH(ctx, "gemm_wgrad_gate_up", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
   }
   // 6. combine dx, reduce the probability gradient
-  MOE_CUDA(launch_unpermute(w.dx_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(dx), ctx->num_sms, st));
-  MOE_CUDA(launch_dprob_reduce(w.dp_part, static_cast<int>(2 * (f / 256)), D.cap, s.src2s, D.Tk, d_topk_prob, st));
+  MOE_LAUNCH(ctx, "unpermute_dx", st, launch_unpermute(w.dx_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(dx), ctx->num_sms, st));
+  MOE_LAUNCH(ctx, "dprob_reduce", st, launch_dprob_reduce(w.dp_part, static_cast<int>(2 * (f / 256)), D.cap, s.src2s, D.Tk, d_topk_prob, st));
   return MOE_OK;
 }
 
