@@ -52,11 +52,11 @@ bool map_2d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t
 }
 // 3-D map over [E, rows, inner] with an arbitrary (16-byte multiple) stride between experts.
 bool map_3d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t rows, uint64_t E,
-            uint64_t row_bytes, uint64_t expert_bytes) {
+            uint64_t row_bytes, uint64_t expert_bytes, uint32_t box_rows = 128) {
   const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cuuint64_t dims[3] = {inner, rows, E};
   cuuint64_t strides[2] = {row_bytes, expert_bytes};
-  cuuint32_t box[3] = {fp8 ? 128u : 64u, 128u, 1u};
+  cuuint32_t box[3] = {fp8 ? 128u : 64u, box_rows, 1u};
   cuuint32_t es[3] = {1, 1, 1};
   return g_encode(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -507,7 +507,9 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     a.do_col = training;
     a.q_colT = s.w1c_q;
     a.s_colT = s.w1c_s;
+    a.gate_up_half = f;  // row-wise copy in 256-row groups of 128 gate + 128 up rows (one B tile each)
     MOE_LAUNCH(ctx, "quantize_w_gate_up", st, launch_quant(a, E, st));
+    a.gate_up_half = 0;
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
     a.src_ld = f;
     a.rows = d;
@@ -585,6 +587,8 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
   // 3. gate_up GEMM + ScaledSwiGLU + requantisation of a
   {
     GemmArgs g = gemm_args(ctx);
+    // MXFP8: the quantised copy is gate/up interleaved, two 128-row boxes per tile; BF16 reads the
+    // unpermuted weights as a 128-row gate box plus the matching 128-row up box.
     const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.x_q) : w.x_perm, D.mx, d, D.cap,
                            d * (D.mx ? 1 : 2)) &&
                     map_3d(&g.tmap_b, w1_base, D.mx, d, 2 * f, E, d * (D.mx ? 1 : 2), w1_stride);
@@ -593,7 +597,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     g.E = E;
     g.K = static_cast<int>(d);
     g.n_tiles = static_cast<int>(f / 128);
-    g.gate_up_half = static_cast<int>(f);
+    g.gate_up_half = D.mx ? 0 : static_cast<int>(f);
     g.poffsets = s.poff;
     g.sfa = w.x_s;
     g.sfa_kb4 = d / 128;

@@ -102,17 +102,19 @@ route_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ top
 }
 
 // ------------------------------------------------------------------------------------------
-// Quantise / gather / transpose tiles of 64 rows x 128 columns (256 threads).
+// Quantise / gather / transpose tiles of 128 rows x 128 columns (256 threads).
 //   MXFP8 mode: row-wise codes + scales (blocks of 32 along a row) and column-wise codes +
 //               scales (blocks of 32 down a column) written transposed, from one read of x.
 //   BF16 mode:  the gathered rows copied, and/or written transposed.
 // The source row of output row r is r itself, or, when ``sorted_to_src`` is given, token
-// sorted_to_src[r] / k (padding rows, -1, read as zeros).
+// sorted_to_src[r] / k (padding rows, -1, read as zeros).  Every thread issues its 8 loads before
+// using any; the column pass writes whole 128-byte lines of the transposed output.
 // ------------------------------------------------------------------------------------------
 namespace {
-constexpr int QT_ROWS = 64;
+constexpr int QT_ROWS = 128;
 constexpr int QT_COLS = 128;
 constexpr int QT_PITCH = QT_COLS + 8;  // bf16 elements per smem row (padding against bank conflicts)
+constexpr int QT_LOADS = QT_ROWS * QT_COLS / 8 / 256;
 
 __device__ __forceinline__ uint32_t abs_bits_bf16x2_max(uint32_t w, uint32_t m) {
   const uint32_t lo = (w & 0x7FFFu) << 16;
@@ -147,17 +149,16 @@ quant_tile_kernel(QuantArgs a) {
   const bf16* src = a.src_ptrs.p[0] ? static_cast<const bf16*>(a.src_ptrs.p[b])
                                     : static_cast<const bf16*>(a.src) + static_cast<int64_t>(b) * a.src_batch_stride;
 
-  // ---- load 64 x 128 (4 chunks of 8 bf16 per thread), row-wise quantise on the fly
+  // ---- load 128 x 128: 8 chunks of 8 bf16 per thread, all issued before any use
   const int cchunk = tid & 15;
   const int64_t col = col0 + cchunk * 8;
   const bool col_ok = col < C;
+  uint4 v[QT_LOADS];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int lr = (tid >> 4) + 16 * i;
-    const int64_t r = row0 + lr;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    bool valid_row = r < R;
-    if (valid_row && col_ok) {
+  for (int i = 0; i < QT_LOADS; ++i) {
+    const int64_t r = row0 + (tid >> 4) + 16 * i;
+    v[i] = make_uint4(0, 0, 0, 0);
+    if (r < R && col_ok) {
       int64_t sr = r;
       bool zero = false;
       if (a.sorted_to_src) {
@@ -165,81 +166,93 @@ quant_tile_kernel(QuantArgs a) {
         zero = s < 0;
         sr = zero ? 0 : static_cast<int64_t>(s / a.k);
       }
-      if (!zero) v = __ldg(reinterpret_cast<const uint4*>(src + sr * a.src_ld + col));
+      if (!zero) v[i] = __ldg(reinterpret_cast<const uint4*>(src + sr * a.src_ld + col));
     }
-    *reinterpret_cast<uint4*>(&tile[lr * QT_PITCH + cchunk * 8]) = v;
-
+  }
+  // ---- row-wise outputs (and the smem copy for the column pass)
+#pragma unroll
+  for (int i = 0; i < QT_LOADS; ++i) {
+    const int lr = (tid >> 4) + 16 * i;
+    const int64_t r = row0 + lr;
+    const bool valid_row = r < R;
+    // destination row: identity, or the gate/up interleaving (128 rows from each half per 256-row group)
+    int64_t dr = r;
+    if (a.gate_up_half) {
+      const int64_t hf = a.gate_up_half;
+      dr = r < hf ? (r / 128) * 256 + (r % 128) : ((r - hf) / 128) * 256 + 128 + ((r - hf) % 128);
+    }
+    if (a.do_col) *reinterpret_cast<uint4*>(&tile[lr * QT_PITCH + cchunk * 8]) = v[i];
     if (a.do_row) {
       if (a.mx) {
         uint32_t m = 0;
-        m = abs_bits_bf16x2_max(v.x, m);
-        m = abs_bits_bf16x2_max(v.y, m);
-        m = abs_bits_bf16x2_max(v.z, m);
-        m = abs_bits_bf16x2_max(v.w, m);
+        m = abs_bits_bf16x2_max(v[i].x, m);
+        m = abs_bits_bf16x2_max(v[i].y, m);
+        m = abs_bits_bf16x2_max(v[i].z, m);
+        m = abs_bits_bf16x2_max(v[i].w, m);
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
         const uint32_t sb = e8m0_from_amax_bits(m);
         const float inv = e8m0_inv_scale(sb);
         if (valid_row && col_ok) {
           float f[8];
-          const bf16* h = reinterpret_cast<const bf16*>(&v);
+          const bf16* h = reinterpret_cast<const bf16*>(&v[i]);
 #pragma unroll
           for (int j = 0; j < 8; ++j) f[j] = __bfloat162float(h[j]) * inv;
           const uint2 q = e4m3x8(f);
-          uint8_t* qrow = a.q_row + (static_cast<int64_t>(b) * R + r) * C + col;
+          uint8_t* qrow = a.q_row + (static_cast<int64_t>(b) * R + dr) * C + col;
           *reinterpret_cast<uint2*>(qrow) = q;
           if ((cchunk & 3) == 0) {
             const int64_t kb = col / 32;
-            const int64_t off = a.sf_mma ? sf_mma_offset(r, kb, KBr) : r * KBr + kb;
+            const int64_t off = a.sf_mma ? sf_mma_offset(dr, kb, KBr) : dr * KBr + kb;
             a.s_row[static_cast<int64_t>(b) * R * KBr + off] = static_cast<uint8_t>(sb);
           }
         }
       } else if (valid_row && col_ok) {
-        *reinterpret_cast<uint4*>(a.o_row + (static_cast<int64_t>(b) * R + r) * C + col) = v;
+        *reinterpret_cast<uint4*>(a.o_row + (static_cast<int64_t>(b) * R + dr) * C + col) = v[i];
       }
     }
   }
   if (!a.do_col) return;
   __syncthreads();
 
-  // ---- column-wise: thread -> (column c, 32-row block rb)
+  // ---- column-wise: thread -> column c, two consecutive 32-row blocks
   const int c = tid & 127;
-  const int rb = tid >> 7;
   const int64_t gc = col0 + c;
-  const int64_t gr = row0 + rb * 32;
-  if (gc >= C || gr >= R) return;
-  float f[32];
-  uint32_t m = 0;
+  if (gc >= C) return;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const bf16 h = tile[(rb * 32 + i) * QT_PITCH + c];
-    f[i] = __bfloat162float(h);
-    m = max(m, __float_as_uint(f[i]) & 0x7FFFFFFFu);
-  }
-  if (a.mx) {
-    const uint32_t sb = e8m0_from_amax_bits(m);
-    const float inv = e8m0_inv_scale(sb);
+  for (int hb = 0; hb < 2; ++hb) {
+    const int rb = 2 * (tid >> 7) + hb;
+    const int64_t gr = row0 + rb * 32;
+    if (gr >= R) break;
+    float f[32];
+    uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) f[i] *= inv;
-    uint8_t* qc = a.q_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
-    uint4 w0, w1;
-    uint2 q0 = e4m3x8(f), q1 = e4m3x8(f + 8), q2 = e4m3x8(f + 16), q3 = e4m3x8(f + 24);
-    w0 = make_uint4(q0.x, q0.y, q1.x, q1.y);
-    w1 = make_uint4(q2.x, q2.y, q3.x, q3.y);
-    reinterpret_cast<uint4*>(qc)[0] = w0;
-    reinterpret_cast<uint4*>(qc)[1] = w1;
-    const int64_t kb = gr / 32;
-    const int64_t off = a.sf_mma ? sf_mma_offset(gc, kb, KBc) : gc * KBc + kb;
-    a.s_colT[static_cast<int64_t>(b) * C * KBc + off] = static_cast<uint8_t>(sb);
-  } else {
-    bf16* oc = a.o_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
+    for (int i = 0; i < 32; ++i) {
+      f[i] = __bfloat162float(tile[(rb * 32 + i) * QT_PITCH + c]);
+      m = max(m, __float_as_uint(f[i]) & 0x7FFFFFFFu);
+    }
+    if (a.mx) {
+      const uint32_t sb = e8m0_from_amax_bits(m);
+      const float inv = e8m0_inv_scale(sb);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint4 w;
-      bf16* hw = reinterpret_cast<bf16*>(&w);
+      for (int i = 0; i < 32; ++i) f[i] *= inv;
+      uint8_t* qc = a.q_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
+      const uint2 q0 = e4m3x8(f), q1 = e4m3x8(f + 8), q2 = e4m3x8(f + 16), q3 = e4m3x8(f + 24);
+      reinterpret_cast<uint4*>(qc)[0] = make_uint4(q0.x, q0.y, q1.x, q1.y);
+      reinterpret_cast<uint4*>(qc)[1] = make_uint4(q2.x, q2.y, q3.x, q3.y);
+      const int64_t kb = gr / 32;
+      const int64_t off = a.sf_mma ? sf_mma_offset(gc, kb, KBc) : gc * KBc + kb;
+      a.s_colT[static_cast<int64_t>(b) * C * KBc + off] = static_cast<uint8_t>(sb);
+    } else {
+      bf16* oc = a.o_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) hw[j] = tile[(rb * 32 + 8 * i + j) * QT_PITCH + c];
-      reinterpret_cast<uint4*>(oc)[i] = w;
+      for (int i = 0; i < 4; ++i) {
+        uint4 w;
+        bf16* hw = reinterpret_cast<bf16*>(&w);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hw[j] = tile[(rb * 32 + 8 * i + j) * QT_PITCH + c];
+        reinterpret_cast<uint4*>(oc)[i] = w;
+      }
     }
   }
 }

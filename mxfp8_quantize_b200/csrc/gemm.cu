@@ -1,6 +1,6 @@
 // Persistent grouped GEMM for sm_100a.
 //
-// C[m, n] = sum_k A[m, k] * B[n, k] with both operands K-major, tiles of 128 x 256 outputs,
+// C[m, n] = sum_k A[m, k] * B[n, k] with both operands K-major, tiles of 128 x BN outputs,
 // over a device-side list of (expert, m-tile, n-tile) built from the padded expert offsets:
 //  * M-grouped (forward and dgrad GEMMs): A's rows are the expert-sorted tokens, expert e
 //    owning rows [poffsets[e], poffsets[e+1]); B is expert e's weight matrix.
@@ -12,10 +12,15 @@
 // Kernels") is what the tile list provides.
 //
 // One CTA per SM, 12 warps:
-//   warp 0  TMA producer (one thread): operand tiles + scale tiles into a 4-stage smem ring
+//   warp 0  TMA producer (one thread): operand tiles + scale tiles into a STAGES-deep smem ring
 //   warp 1  MMA issuer (one thread): scale tiles smem->TMEM, 4 MMAs per stage, commits
 //   warp 2  TMEM allocator
 //   warps 4-11 epilogue: TMEM -> registers -> fused math -> global stores
+// Tiles are 128 x 256 with one TMEM accumulator (two 256-column accumulators would leave no room
+// for the per-stage scale tiles; the template keeps a double-buffered variant available).  Plain
+// bf16-store epilogues drain the accumulator into packed registers and release it before storing;
+// the fused ScaledSwiGLU / dSwiGLU epilogues release it after their last TMEM load and requantise
+// column-wise through a small padded smem transpose (one scale per column per lane).
 // Every wait is bounded: on expiry the kernel records MOE_ERR_TIMEOUT and all roles stop.
 #include <cuda_fp8.h>
 
@@ -26,26 +31,38 @@ namespace moemx {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * 128;  // 128 rows x 128 bytes of K
-constexpr int B_BYTES = BN * 128;
-constexpr int OFF_B = A_BYTES;
-constexpr int OFF_SFA = A_BYTES + B_BYTES;
-constexpr int OFF_SFB = OFF_SFA + 512;
-constexpr int STAGE_BYTES = 51200;  // 1024-aligned
 constexpr int EPI_WARPS = 8;
 constexpr int NUM_THREADS = 32 * (4 + EPI_WARPS);
-constexpr int STAGING_PER_WARP = 2048;
-constexpr int SMEM_DYN = STAGES * STAGE_BYTES + EPI_WARPS * STAGING_PER_WARP + 1024;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_TMEM_COL = 256;  // scale tiles live after the 256 accumulator columns
+constexpr int STAGE_PITCH = 17;  // floats per row of an epilogue warp's 32 x 16 transpose buffer (odd: no bank conflicts)
+
+template <int BN_, int NBUF_, int STAGES_, bool STAGING_>
+struct Shape {
+  static constexpr int BN = BN_;
+  static constexpr int NBUF = NBUF_;
+  static constexpr int STAGES = STAGES_;
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int SFB_BYTES = (BN / 128) * 512;
+  static constexpr int OFF_B = A_BYTES;
+  static constexpr int OFF_SFA = A_BYTES + B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + 512;
+  static constexpr int STAGE_BYTES = (OFF_SFB + SFB_BYTES + 1023) / 1024 * 1024;
+  static constexpr int SF_COLS = 4 + 4 * (BN / 128);
+  static constexpr uint32_t SF_TMEM_COL = NBUF * BN;
+  static constexpr int STAGING_PER_WARP = STAGING_ ? (32 * STAGE_PITCH * 4 + 15) / 16 * 16 : 0;
+  static constexpr int SMEM_DYN = STAGES * STAGE_BYTES + EPI_WARPS * STAGING_PER_WARP + 1024;
+  static_assert(NBUF * BN + STAGES * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_DYN + 4096 <= 232448, "shared memory budget");
+};
+using ShapeStore = Shape<256, 1, 4, false>;
+using ShapeFused = Shape<256, 1, 4, true>;
 
 struct SharedState {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t acc_full;
-  uint64_t acc_empty;
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -61,7 +78,7 @@ struct Tile {
 };
 
 __device__ __forceinline__ void decode_tile(int t, const SharedState& s, const GemmArgs& g, bool mx, Tile& o) {
-  int lo = 0, hi = g.E;  // find e with prefix[e] <= t < prefix[e+1]
+  int lo = 0, hi = g.E;  // largest e with prefix[e] <= t (experts without tiles are skipped)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (s.tile_prefix[mid] <= t) lo = mid; else hi = mid;
@@ -96,30 +113,33 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, in
       : "memory");
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g * sigmoid(g); sigmoid from the hardware exp2 and a fast reciprocal-multiply
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 // Pack 8 floats as bf16 (round to nearest even) into a uint4.
 __device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
-  uint4 o;
-  uint32_t* w = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-    w[i] = *reinterpret_cast<uint32_t*>(&h);
-  }
-  return o;
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                    pack_bf16x2(v[6], v[7]));
 }
 __device__ __forceinline__ void unpack_bf16x8(uint4 v, float* o) {
-  const bf16* h = reinterpret_cast<const bf16*>(&v);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) o[i] = __bfloat162float(h[i]);
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
 }
 __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
-// Row-wise MXFP8 of 32 consecutive values of this thread's row: 32 codes + 1 scale byte.
-__device__ __forceinline__ void quant_row32(const float* v, uint8_t* q, uint8_t* sbyte) {
+// MXFP8 of 32 values with the scale of their own amax: 32 codes stored at q (16-byte aligned);
+// returns the E8M0 byte.
+__device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q) {
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) m = max(m, __float_as_uint(v[i]) & 0x7FFFFFFFu);
@@ -131,76 +151,58 @@ __device__ __forceinline__ void quant_row32(const float* v, uint8_t* q, uint8_t*
     w[i] = e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv) | (e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv) << 16);
   reinterpret_cast<uint4*>(q)[0] = make_uint4(w[0], w[1], w[2], w[3]);
   reinterpret_cast<uint4*>(q)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  *sbyte = static_cast<uint8_t>(sb);
+  return sb;
 }
 
-// Column-wise MXFP8 of a 32 x 32 block held one row per lane (v = this lane's row): per column
-// the amax is taken over the 32 lanes; codes are transposed through ``stage`` so that lane l
-// stores column l's 32 codes contiguously at colT + l * ld, and its scale byte at sf[l].
-__device__ __forceinline__ void quant_col32(const float* v, uint8_t* stage, uint8_t* colT, int64_t ld,
-                                            uint8_t* sf_base, int64_t sf_row0, int64_t sf_kb, int64_t sf_KB) {
+// Column-wise outputs of a 32 x 32 block held one row per lane (v = this lane's 32 values), in two
+// passes of 16 columns through the warp's padded smem buffer: after a pass lane l holds column
+// c = l % 16 of the pass, rows 16*(l/16) .. +16.
+template <class F>
+__device__ __forceinline__ void column_passes(const float* v, float* stage, F&& emit) {
   const int lane = threadIdx.x & 31;
-  uint32_t my_sb = 0;
-  uint32_t w[8];
 #pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const uint32_t m0 = __reduce_max_sync(0xffffffffu, __float_as_uint(v[i]) & 0x7FFFFFFFu);
-    const uint32_t m1 = __reduce_max_sync(0xffffffffu, __float_as_uint(v[i + 1]) & 0x7FFFFFFFu);
-    const uint32_t s0 = e8m0_from_amax_bits(m0), s1 = e8m0_from_amax_bits(m1);
-    if (lane == i) my_sb = s0;
-    if (lane == i + 1) my_sb = s1;
-    const uint32_t c = e4m3x2(v[i] * e8m0_inv_scale(s0), v[i + 1] * e8m0_inv_scale(s1));
-    if ((i & 3) == 0) w[i >> 2] = c; else w[i >> 2] |= c << 16;
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) stage[lane * STAGE_PITCH + c] = v[16 * h + c];
+    __syncwarp();
+    float col[16];
+    const int cl = lane & 15, rh = lane >> 4;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) col[i] = stage[(16 * rh + i) * STAGE_PITCH + cl];
+    __syncwarp();
+    emit(h, cl, rh, col);
   }
-  // stage row ``lane`` (32 bytes, two 16-byte chunks swizzled by bit 2 of the row)
-  const int sw = (lane >> 2) & 1;
-  reinterpret_cast<uint4*>(stage + lane * 32)[0 ^ sw] = make_uint4(w[0], w[1], w[2], w[3]);
-  reinterpret_cast<uint4*>(stage + lane * 32)[1 ^ sw] = make_uint4(w[4], w[5], w[6], w[7]);
-  __syncwarp();
-  uint32_t o[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    uint32_t acc = 0;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int r = 4 * j + b;
-      const int ch = (lane >> 4) ^ ((r >> 2) & 1);
-      acc |= static_cast<uint32_t>(stage[r * 32 + ch * 16 + (lane & 15)]) << (8 * b);
-    }
-    o[j] = acc;
-  }
-  __syncwarp();
-  uint8_t* dst = colT + lane * ld;
-  reinterpret_cast<uint4*>(dst)[0] = make_uint4(o[0], o[1], o[2], o[3]);
-  reinterpret_cast<uint4*>(dst)[1] = make_uint4(o[4], o[5], o[6], o[7]);
-  sf_base[sf_mma_offset(sf_row0 + lane, sf_kb, sf_KB)] = static_cast<uint8_t>(my_sb);
 }
 
-// Column-wise bf16 transpose of a 32 x 32 block held one row per lane: lane l stores column l.
-__device__ __forceinline__ void transpose_col32_bf16(const float* v, uint8_t* stage, bf16* colT, int64_t ld) {
-  const int lane = threadIdx.x & 31;
-  const int sw = (lane >> 1) & 3;
+// Column-wise MXFP8 of a 32 x 32 block (rows = lanes): each column is quantised with the scale of
+// its 32 values; column c's 32 codes go to colT + c * ld, its scale to S[sf_row0 + c][sf_kb] of a
+// tile-layout scale matrix with sf_KB columns.
+__device__ __forceinline__ void colwise_mx(const float* v, float* stage, uint8_t* colT, int64_t ld, uint8_t* sf,
+                                           int64_t sf_row0, int64_t sf_kb, int64_t sf_KB) {
+  column_passes(v, stage, [&](int h, int cl, int rh, const float* col) {
+    uint32_t m = 0;
 #pragma unroll
-  for (int c = 0; c < 4; ++c)
-    reinterpret_cast<uint4*>(stage + lane * 64)[c ^ sw] = pack_bf16x8(v + 8 * c);
-  __syncwarp();
-  uint32_t o[16];
+    for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(col[i]) & 0x7FFFFFFFu);
+    m = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
+    const uint32_t sb = e8m0_from_amax_bits(m);
+    const float inv = e8m0_inv_scale(sb);
+    uint32_t w[4];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    uint32_t acc = 0;
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      const int r = 2 * j + b;
-      const int ch = (lane >> 3) ^ ((r >> 1) & 3);
-      const uint16_t hv = *reinterpret_cast<const uint16_t*>(stage + r * 64 + ch * 16 + (lane & 7) * 2);
-      acc |= static_cast<uint32_t>(hv) << (16 * b);
-    }
-    o[j] = acc;
-  }
-  __syncwarp();
-  uint4* dst = reinterpret_cast<uint4*>(colT + lane * ld);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+    for (int i = 0; i < 4; ++i)
+      w[i] = e4m3x2(col[4 * i] * inv, col[4 * i + 1] * inv) | (e4m3x2(col[4 * i + 2] * inv, col[4 * i + 3] * inv) << 16);
+    const int c = 16 * h + cl;
+    *reinterpret_cast<uint4*>(colT + c * ld + 16 * rh) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (rh == 0) sf[sf_mma_offset(sf_row0 + c, sf_kb, sf_KB)] = static_cast<uint8_t>(sb);
+  });
+}
+
+// Column-wise bf16 of a 32 x 32 block: column c (32 bf16) goes to colT + c * ld.
+__device__ __forceinline__ void colwise_bf16(const float* v, float* stage, bf16* colT, int64_t ld) {
+  column_passes(v, stage, [&](int h, int cl, int rh, const float* col) {
+    uint4* dst = reinterpret_cast<uint4*>(colT + (16 * h + cl) * ld + 16 * rh);
+    dst[0] = pack_bf16x8(col);
+    dst[1] = pack_bf16x8(col + 8);
+  });
 }
 
 __device__ __forceinline__ void load_acc32(uint32_t taddr, float* v) {
@@ -213,12 +215,13 @@ __device__ __forceinline__ void load_acc32(uint32_t taddr, float* v) {
 
 }  // namespace
 
-template <bool MX, int EPI>
+template <bool MX, int EPI, class S>
 __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs g) {
   __shared__ SharedState s;
   extern __shared__ uint8_t dyn_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* staging_base = smem + STAGES * STAGE_BYTES;
+  float* staging_base = reinterpret_cast<float*>(smem + S::STAGES * S::STAGE_BYTES);
+  constexpr int BN = S::BN;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -236,12 +239,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     s.tile_prefix[g.E] = acc;
     s.total_tiles = acc;
     s.abort_flag = 0;
-    for (int i = 0; i < STAGES; ++i) {
+    for (int i = 0; i < S::STAGES; ++i) {
       ptx::mbar_init(&s.full[i], 1);
       ptx::mbar_init(&s.empty[i], 1);
     }
-    ptx::mbar_init(&s.acc_full, 1);
-    ptx::mbar_init(&s.acc_empty, EPI_WARPS);
+    for (int i = 0; i < S::NBUF; ++i) {
+      ptx::mbar_init(&s.acc_full[i], 1);
+      ptx::mbar_init(&s.acc_empty[i], EPI_WARPS);
+    }
     ptx::mbar_init(&s.drain, 1);
     ptx::fence_mbar_init();
   }
@@ -266,54 +271,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, last_parity = 0;
-    const uint32_t tx = A_BYTES + B_BYTES + (MX ? 512 + 1024 : 0);
+    const uint32_t tx = S::A_BYTES + S::B_BYTES + (MX ? 512 + S::SFB_BYTES : 0);
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
       const int bk = MX ? 128 : 64;
       for (int kb = 0; kb < tl.nk; ++kb) {
         if (!ptx::mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, lim)) break;
-        uint8_t* st = smem + stage * STAGE_BYTES;
+        uint8_t* st = smem + stage * S::STAGE_BYTES;
         ptx::mbar_arrive_expect_tx(&s.full[stage], tx);
         const int kx = tl.k0 + kb * bk;
         ptx::tma_load_2d(st, &g.tmap_a, kx, tl.a_row, &s.full[stage]);
-        int b_r0, b_r1;
-        if (!g.kgrouped) {
-          if (g.gate_up_half) {
-            b_r0 = tl.nb * 128;
-            b_r1 = g.gate_up_half + tl.nb * 128;
-          } else {
-            b_r0 = tl.nb * BN;
-            b_r1 = b_r0 + 128;
-          }
-          tma_load_3d(st + OFF_B, &g.tmap_b, kx, b_r0, tl.e, &s.full[stage]);
-          tma_load_3d(st + OFF_B + B_BYTES / 2, &g.tmap_b, kx, b_r1, tl.e, &s.full[stage]);
+        if (!g.kgrouped && g.gate_up_half) {
+          // bf16 gate_up: BN/2 gate rows then the matching BN/2 up rows of expert e
+          tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * (BN / 2), tl.e, &s.full[stage]);
+          tma_load_3d(st + S::OFF_B + S::B_BYTES / 2, &g.tmap_b, kx, g.gate_up_half + tl.nb * (BN / 2), tl.e,
+                      &s.full[stage]);
         } else {
-          b_r0 = tl.nb * BN;
-          b_r1 = b_r0 + 128;
-          ptx::tma_load_2d(st + OFF_B, &g.tmap_b, kx, b_r0, &s.full[stage]);
-          ptx::tma_load_2d(st + OFF_B + B_BYTES / 2, &g.tmap_b, kx, b_r1, &s.full[stage]);
+#pragma unroll
+          for (int i = 0; i < BN / 128; ++i) {
+            const int brow = tl.nb * BN + i * 128;
+            if (!g.kgrouped)
+              tma_load_3d(st + S::OFF_B + i * 16384, &g.tmap_b, kx, brow, tl.e, &s.full[stage]);
+            else
+              ptx::tma_load_2d(st + S::OFF_B + i * 16384, &g.tmap_b, kx, brow, &s.full[stage]);
+          }
         }
         if (MX) {
           const int64_t kq = kx / 128;
           const uint8_t* sa = g.sfa + ((static_cast<int64_t>(tl.a_row) / 128) * g.sfa_kb4 + kq) * 512;
-          ptx::bulk_load(st + OFF_SFA, sa, 512, &s.full[stage]);
+          ptx::bulk_load(st + S::OFF_SFA, sa, 512, &s.full[stage]);
           const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * g.sfb_expert_rows;
-          const uint8_t* sb0 = g.sfb + (((eb + b_r0) / 128) * g.sfb_kb4 + kq) * 512;
-          const uint8_t* sb1 = g.sfb + (((eb + b_r1) / 128) * g.sfb_kb4 + kq) * 512;
-          ptx::bulk_load(st + OFF_SFB, sb0, 512, &s.full[stage]);
-          ptx::bulk_load(st + OFF_SFB + 512, sb1, 512, &s.full[stage]);
+#pragma unroll
+          for (int i = 0; i < BN / 128; ++i) {
+            const int64_t brow = eb + static_cast<int64_t>(tl.nb) * BN + i * 128;
+            ptx::bulk_load(st + S::OFF_SFB + i * 512, g.sfb + ((brow / 128) * g.sfb_kb4 + kq) * 512, 512,
+                           &s.full[stage]);
+          }
         }
         issued_mask |= 1u << stage;
         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == STAGES) {
+        if (++stage == S::STAGES) {
           stage = 0;
           phase ^= 1;
         }
       }
     }
     // wait for the loads still in flight (only possible after an abort)
-    for (int i = 0; i < STAGES; ++i)
+    for (int i = 0; i < S::STAGES; ++i)
       if (issued_mask & (1u << i)) {
         volatile int never = 0;
         ptx::mbar_wait(&s.full[i], (last_parity >> i) & 1u, &never, lim);
@@ -321,15 +326,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   } else if (warp == 1 && lane == 0) {
     // ================= MMA issuer
     int stage = 0;
-    uint32_t phase = 0, acc_phase = 0;
+    uint32_t phase = 0;
+    int local = 0;  // tiles with MMAs issued by this CTA
     bool issued_any = false;
-    const uint32_t d_tmem = tmem;
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
       if (tl.nk == 0) continue;
-      if (!ptx::mbar_wait(&s.acc_empty, acc_phase ^ 1, abort_flag, lim)) break;
+      const int buf = S::NBUF == 2 ? (local & 1) : 0;
+      const uint32_t acc_par = static_cast<uint32_t>((S::NBUF == 2 ? (local >> 1) : local) & 1);
+      if (!ptx::mbar_wait(&s.acc_empty[buf], acc_par ^ 1, abort_flag, lim)) break;
       ptx::tc_fence_after();
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * BN);
       bool ok = true;
       for (int kb = 0; kb < tl.nk; ++kb) {
         if (!ptx::mbar_wait(&s.full[stage], phase, abort_flag, lim)) {
@@ -337,15 +345,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t st = ptx::smem_u32(smem + stage * STAGE_BYTES);
+        const uint32_t st = ptx::smem_u32(smem + stage * S::STAGE_BYTES);
         const uint64_t adesc = ptx::smem_desc(st, 16, 1024, ptx::kSwizzle128B);
-        const uint64_t bdesc = ptx::smem_desc(st + OFF_B, 16, 1024, ptx::kSwizzle128B);
+        const uint64_t bdesc = ptx::smem_desc(st + S::OFF_B, 16, 1024, ptx::kSwizzle128B);
         if (MX) {
-          const uint32_t sfa_t = tmem + SF_TMEM_COL + 12 * stage;
+          const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * stage;
           const uint32_t sfb_t = sfa_t + 4;
-          ptx::tc_cp_32x128b_warpx4(sfa_t, ptx::smem_desc(st + OFF_SFA, 0, 128, ptx::kSwizzleNone));
-          ptx::tc_cp_32x128b_warpx4(sfb_t, ptx::smem_desc(st + OFF_SFB, 0, 128, ptx::kSwizzleNone));
-          ptx::tc_cp_32x128b_warpx4(sfb_t + 4, ptx::smem_desc(st + OFF_SFB + 512, 0, 128, ptx::kSwizzleNone));
+          ptx::tc_cp_32x128b_warpx4(sfa_t, ptx::smem_desc(st + S::OFF_SFA, 0, 128, ptx::kSwizzleNone));
+#pragma unroll
+          for (int i = 0; i < BN / 128; ++i)
+            ptx::tc_cp_32x128b_warpx4(sfb_t + 4 * i,
+                                      ptx::smem_desc(st + S::OFF_SFB + 512 * i, 0, 128, ptx::kSwizzleNone));
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             ptx::tc_mma_mxf8(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(BM, BN, k, k), sfa_t, sfb_t,
@@ -357,14 +367,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         }
         ptx::tc_commit(&s.empty[stage]);
         issued_any = true;
-        if (++stage == STAGES) {
+        if (++stage == S::STAGES) {
           stage = 0;
           phase ^= 1;
         }
       }
       if (!ok) break;
-      ptx::tc_commit(&s.acc_full);
-      acc_phase ^= 1;
+      ptx::tc_commit(&s.acc_full[buf]);
+      ++local;
     }
     if (issued_any) {  // all MMAs of this CTA complete before TMEM can be released
       ptx::tc_commit(&s.drain);
@@ -375,10 +385,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     // ================= epilogue
     const int q = warp & 3;          // TMEM lane quadrant this warp may read
     const int ch = (warp - 4) >> 2;  // column half of the tile
-    uint8_t* stage_buf = staging_base + (warp - 4) * STAGING_PER_WARP;
+    float* stage_buf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(staging_base) +
+                                                (warp - 4) * S::STAGING_PER_WARP);
     const EpiArgs& ep = g.epi;
-    uint32_t acc_phase = 0;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    int local = 0;
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
@@ -388,36 +398,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         // K-grouped expert without tokens: its weight gradient is zero
         if (EPI == EPI_STORE) {
           bf16* out = static_cast<bf16*>(const_cast<void*>(ep.out_ptrs.p[tl.e]));
-          const int64_t c0 = static_cast<int64_t>(tl.nb) * BN + 128 * ch;
+          const int64_t c0 = static_cast<int64_t>(tl.nb) * BN + (BN / 2) * ch;
           uint4* dst = reinterpret_cast<uint4*>(out + row * ep.ldo + c0);
 #pragma unroll 4
-          for (int i = 0; i < 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < BN / 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
         }
         continue;
       }
-      if (!ptx::mbar_wait(&s.acc_full, acc_phase, abort_flag, lim)) break;
-      ptx::tc_fence_after();
+      const int buf = S::NBUF == 2 ? (local & 1) : 0;
+      const uint32_t acc_par = static_cast<uint32_t>((S::NBUF == 2 ? (local >> 1) : local) & 1);
+      ++local;
 
       if (EPI == EPI_STORE) {
-        bf16* out = g.kgrouped ? static_cast<bf16*>(const_cast<void*>(ep.out_ptrs.p[tl.e])) : ep.out;
-        const int64_t c0 = static_cast<int64_t>(tl.nb) * BN + 128 * ch;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          float v[32];
-          load_acc32(t_lane + 128 * ch + 32 * cc, v);
-          uint4* dst = reinterpret_cast<uint4*>(out + row * ep.ldo + c0 + 32 * cc);
+        // drain the accumulator into packed bf16, release it, then store
+        if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
+        ptx::tc_fence_after();
+        const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
+        uint32_t pk[BN / 4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = pack_bf16x8(v + 8 * i);
+        for (int cc = 0; cc < BN / 64; ++cc) {
+          float v[32];
+          load_acc32(t_lane + (BN / 2) * ch + 32 * cc, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[16 * cc + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
         }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
+        bf16* out = g.kgrouped ? static_cast<bf16*>(const_cast<void*>(ep.out_ptrs.p[tl.e])) : ep.out;
+        uint4* dst = reinterpret_cast<uint4*>(out + row * ep.ldo + static_cast<int64_t>(tl.nb) * BN + (BN / 2) * ch);
+#pragma unroll
+        for (int i = 0; i < BN / 16; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       } else if (EPI == EPI_SWIGLU) {
+        // tile = 128 output columns; accumulator columns [0,128) gate, [128,256) up
         const float p = ep.p_perm[row];
         const int64_t f = ep.f;
+        if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
+        ptx::tc_fence_after();
+        const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
-          const int64_t j = static_cast<int64_t>(tl.nb) * 128 + 64 * ch + 32 * cc;  // output column
+          const int64_t j = static_cast<int64_t>(tl.nb) * 128 + 64 * ch + 32 * cc;  // 32 output columns
           float gv[32], uv[32];
           load_acc32(t_lane + 64 * ch + 32 * cc, gv);
           load_acc32(t_lane + 128 + 64 * ch + 32 * cc, uv);
+          if (cc == 1) {
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
+          }
           if (ep.h) {
             uint4* hg = reinterpret_cast<uint4*>(ep.h + row * 2 * f + j);
             uint4* hu = reinterpret_cast<uint4*>(ep.h + row * 2 * f + f + j);
@@ -428,49 +457,71 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
             }
           }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) gv[i] = silu_f(gv[i]) * uv[i] * p;  // a, in place
+          for (int i = 0; i < 32; ++i) gv[i] = gv[i] * sigmoid_f(gv[i]) * uv[i] * p;  // a, in place
           if (ep.dump) {
             float4* dd = reinterpret_cast<float4*>(ep.dump + row * f + j);
 #pragma unroll
             for (int i = 0; i < 8; ++i) dd[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
           }
           if (MX) {
-            uint8_t sb;
-            quant_row32(gv, ep.q_row + row * f + j, &sb);
-            ep.s_row[sf_mma_offset(row, j / 32, f / 32)] = sb;
+            const uint32_t sb = quant32_store(gv, ep.q_row + row * f + j);
+            ep.s_row[sf_mma_offset(row, j / 32, f / 32)] = static_cast<uint8_t>(sb);
             if (ep.q_colT)
-              quant_col32(gv, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
-                          ep.cap / 32);
+              colwise_mx(gv, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
+                         ep.cap / 32);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(ep.o_row + row * f + j);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = pack_bf16x8(gv + 8 * i);
-            if (ep.o_colT) transpose_col32_bf16(gv, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
+            if (ep.o_colT) colwise_bf16(gv, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
           }
         }
-      } else {  // EPI_DSWIGLU
+      } else {  // EPI_DSWIGLU: tile = 256 f-columns of da; this thread owns 128 of them
         const float p = ep.p_perm[row];
         const int64_t f = ep.f, f2 = 2 * ep.f;
+        const int64_t j0 = static_cast<int64_t>(tl.nb) * BN + 128 * ch;
+        const bf16* hrow = ep.h + row * f2;
+        uint4 hg[4], hu[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {  // saved gate/up values of the first group, before the wait
+          hg[i] = reinterpret_cast<const uint4*>(hrow + j0)[i];
+          hu[i] = reinterpret_cast<const uint4*>(hrow + f + j0)[i];
+        }
+        if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
+        ptx::tc_fence_after();
+        const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
         float dp = 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
-          const int64_t j = static_cast<int64_t>(tl.nb) * BN + 128 * ch + 32 * cc;  // f column
+          const int64_t j = j0 + 32 * cc;
           float da[32];
           load_acc32(t_lane + 128 * ch + 32 * cc, da);
+          if (cc == 3) {
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
+          }
           float dg[32], du[32];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float gg[8], uu[8];
-            unpack_bf16x8(reinterpret_cast<const uint4*>(ep.h + row * f2 + j)[i], gg);
-            unpack_bf16x8(reinterpret_cast<const uint4*>(ep.h + row * f2 + f + j)[i], uu);
+            unpack_bf16x8(hg[i], gg);
+            unpack_bf16x8(hu[i], uu);
 #pragma unroll
             for (int q8 = 0; q8 < 8; ++q8) {
               const float gx = gg[q8], ux = uu[q8], d = da[8 * i + q8];
-              const float sg = 1.0f / (1.0f + __expf(-gx));
+              const float sg = sigmoid_f(gx);
               const float sl = gx * sg;
               dg[8 * i + q8] = d * p * ux * sg * (1.0f + gx * (1.0f - sg));
               du[8 * i + q8] = d * p * sl;
               dp += d * sl * ux;
+            }
+          }
+          if (cc < 3) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // next group's saved values
+              hg[i] = reinterpret_cast<const uint4*>(hrow + j + 32)[i];
+              hu[i] = reinterpret_cast<const uint4*>(hrow + f + j + 32)[i];
             }
           }
           if (ep.dump) {
@@ -483,14 +534,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
             }
           }
           if (MX) {
-            uint8_t sb;
-            quant_row32(dg, ep.q_row + row * f2 + j, &sb);
-            ep.s_row[sf_mma_offset(row, j / 32, f2 / 32)] = sb;
-            quant_row32(du, ep.q_row + row * f2 + f + j, &sb);
-            ep.s_row[sf_mma_offset(row, (f + j) / 32, f2 / 32)] = sb;
-            quant_col32(dg, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32, ep.cap / 32);
-            quant_col32(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j, row_w / 32,
-                        ep.cap / 32);
+            uint32_t sb = quant32_store(dg, ep.q_row + row * f2 + j);
+            ep.s_row[sf_mma_offset(row, j / 32, f2 / 32)] = static_cast<uint8_t>(sb);
+            sb = quant32_store(du, ep.q_row + row * f2 + f + j);
+            ep.s_row[sf_mma_offset(row, (f + j) / 32, f2 / 32)] = static_cast<uint8_t>(sb);
+            colwise_mx(dg, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32, ep.cap / 32);
+            colwise_mx(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j, row_w / 32,
+                       ep.cap / 32);
           } else {
             uint4* d0 = reinterpret_cast<uint4*>(ep.o_row + row * f2 + j);
             uint4* d1 = reinterpret_cast<uint4*>(ep.o_row + row * f2 + f + j);
@@ -499,16 +549,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
               d0[i] = pack_bf16x8(dg + 8 * i);
               d1[i] = pack_bf16x8(du + 8 * i);
             }
-            transpose_col32_bf16(dg, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
-            transpose_col32_bf16(du, stage_buf, ep.o_colT + (f + j) * ep.cap + row_w, ep.cap);
+            colwise_bf16(dg, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
+            colwise_bf16(du, stage_buf, ep.o_colT + (f + j) * ep.cap + row_w, ep.cap);
           }
         }
         ep.dp_part[(static_cast<int64_t>(tl.nb) * 2 + ch) * ep.cap + row] = dp;
       }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&s.acc_empty);
-      acc_phase ^= 1;
     }
   }
 
@@ -521,25 +567,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
 }
 
 namespace {
-template <bool MX, int EPI>
+template <bool MX, int EPI, class S>
 cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
-  auto kern = grouped_gemm_kernel<MX, EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN);
+  auto kern = grouped_gemm_kernel<MX, EPI, S>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_DYN);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms, NUM_THREADS, SMEM_DYN, st>>>(args);
+  kern<<<num_sms, NUM_THREADS, S::SMEM_DYN, st>>>(args);
   return cudaGetLastError();
 }
 }  // namespace
 
+int gemm_tile_n(int epi) { return epi == EPI_STORE ? ShapeStore::BN : ShapeFused::BN; }
+
 cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st) {
   if (mx) {
-    if (epi == EPI_STORE) return launch_t<true, EPI_STORE>(args, num_sms, st);
-    if (epi == EPI_SWIGLU) return launch_t<true, EPI_SWIGLU>(args, num_sms, st);
-    return launch_t<true, EPI_DSWIGLU>(args, num_sms, st);
+    if (epi == EPI_STORE) return launch_t<true, EPI_STORE, ShapeStore>(args, num_sms, st);
+    if (epi == EPI_SWIGLU) return launch_t<true, EPI_SWIGLU, ShapeFused>(args, num_sms, st);
+    return launch_t<true, EPI_DSWIGLU, ShapeFused>(args, num_sms, st);
   }
-  if (epi == EPI_STORE) return launch_t<false, EPI_STORE>(args, num_sms, st);
-  if (epi == EPI_SWIGLU) return launch_t<false, EPI_SWIGLU>(args, num_sms, st);
-  return launch_t<false, EPI_DSWIGLU>(args, num_sms, st);
+  if (epi == EPI_STORE) return launch_t<false, EPI_STORE, ShapeStore>(args, num_sms, st);
+  if (epi == EPI_SWIGLU) return launch_t<false, EPI_SWIGLU, ShapeFused>(args, num_sms, st);
+  return launch_t<false, EPI_DSWIGLU, ShapeFused>(args, num_sms, st);
 }
 
 }  // namespace moemx

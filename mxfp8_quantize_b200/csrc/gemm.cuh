@@ -40,7 +40,8 @@ struct GemmArgs {
   int K;               // M-grouped reduction length
   int n_tiles;         // output tiles along N per expert
   int m_tiles;         // K-grouped: M / 128
-  int gate_up_half;    // M-grouped SWIGLU: f (B rows of the up half start at f); else 0
+  int gate_up_half;    // B tile made of two 128-row boxes: gate rows nb*128, up rows gate_up_half + nb*128
+                       // (bf16 gate_up GEMM reading the unpermuted weights); 0 = BN/128 boxes of 128 rows
   const int32_t* poffsets;
   const uint8_t* sfa;  // MXFP8 scales of A / B in the tile layout
   int64_t sfa_kb4;     // 128-wide K blocks per 128-row block of A's scales

@@ -108,11 +108,15 @@ def test_small_quantised_operands_bit_exact(small):
     w1 = ref["np"]["w_gate_up"]
     w2 = ref["np"]["w_down"]
     # weights, row-wise (forward GEMMs) ...
+    # (the row-wise copy of W1 is stored in 256-row groups of 128 gate rows + the matching 128 up rows)
     q = _view(g["ws"], 1, "w1_q", cfg, precision, True, E * 2 * f * d).cpu().numpy().reshape(E * 2 * f, d)
     s = _view(g["ws"], 1, "w1_s", cfg, precision, True, E * 2 * f * d // 32).cpu().numpy()
     rq, rs = mx.quantize_rowwise(w1.reshape(E * 2 * f, d))
-    assert np.array_equal(q, rq)
-    assert np.array_equal(unswizzle_scales(s, E * 2 * f, d // 32), rs)
+    r = np.arange(2 * f)
+    dst = np.where(r < f, (r // 128) * 256 + r % 128, ((r - f) // 128) * 256 + 128 + (r - f) % 128)
+    dst = (np.arange(E)[:, None] * 2 * f + dst[None, :]).reshape(-1)
+    assert np.array_equal(q[dst], rq)
+    assert np.array_equal(unswizzle_scales(s, E * 2 * f, d // 32)[dst], rs)
     q = _view(g["ws"], 1, "w2_q", cfg, precision, True, E * d * f).cpu().numpy().reshape(E * d, f)
     assert np.array_equal(q, mx.quantize_rowwise(w2.reshape(E * d, f))[0])
     # ... and down the columns, transposed (dgrad GEMMs)
