@@ -171,7 +171,7 @@ void carve_bwd(Carve& c, const Dims& D, BwdWs& w) {
     w.w2T = c.take<bf16>(D.E * D.f * D.d * 2);
   }
   w.dx_perm = c.take<bf16>(D.cap * D.d * 2);
-  w.dp_part = c.take<float>(2 * (D.f / 256) * D.cap * 4);
+  w.dp_part = c.take<float>(2 * (D.f / gemm_tile_n(EPI_DSWIGLU)) * D.cap * 4);
 }
 
 int64_t capacity_rows(int64_t T, int k, int E) {
@@ -364,7 +364,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
   a.s_row = s_row;
   a.q_colT = q_colT;
   a.s_colT = s_colT;
-  MOE_LAUNCH(ctx, "mxfp8_quantize", stream, launch_quant(a, static_cast<int>(batch), static_cast<cudaStream_t>(stream)));
+  MOE_LAUNCH(ctx, "mxfp8_quantize", stream, launch_quant(a, static_cast<int>(batch), ctx->num_sms, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 
@@ -405,7 +405,7 @@ moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, 
     a.mx = 0;
     a.do_row = 1;
     a.o_row = static_cast<bf16*>(x_perm);
-    MOE_LAUNCH(ctx, "permute_x", st, launch_quant(a, 1, st));
+    MOE_LAUNCH(ctx, "permute_x", st, launch_quant(a, 1, ctx->num_sms, st));
   }
   return MOE_OK;
 }
@@ -508,7 +508,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     a.q_colT = s.w1c_q;
     a.s_colT = s.w1c_s;
     a.gate_up_half = f;  // row-wise copy in 256-row groups of 128 gate + 128 up rows (one B tile each)
-    MOE_LAUNCH(ctx, "quantize_w_gate_up", st, launch_quant(a, E, st));
+    MOE_LAUNCH(ctx, "quantize_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
     a.gate_up_half = 0;
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
     a.src_ld = f;
@@ -518,7 +518,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     a.s_row = w.w2_s;
     a.q_colT = s.w2c_q;
     a.s_colT = s.w2c_s;
-    MOE_LAUNCH(ctx, "quantize_w_down", st, launch_quant(a, E, st));
+    MOE_LAUNCH(ctx, "quantize_w_down", st, launch_quant(a, E, ctx->num_sms, st));
     w1_base = w.w1_q;
     w1_stride = 2 * f * d;
     w2_base = w.w2_q;
@@ -540,7 +540,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.do_col = training;
     xa.q_colT = s.xT_q;
     xa.s_colT = s.xT_s;
-    MOE_LAUNCH(ctx, "permute_quantize_x", st, launch_quant(xa, 1, st));
+    MOE_LAUNCH(ctx, "permute_quantize_x", st, launch_quant(xa, 1, ctx->num_sms, st));
   } else {
     w1_stride = uniform_stride(w_gate_up, E, 2 * f * d * 2);
     w2_stride = uniform_stride(w_down, E, d * f * 2);
@@ -555,7 +555,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       a.rows = 2 * f;
       a.cols = d;
       a.o_row = w.w1_copy;
-      MOE_LAUNCH(ctx, "gather_w_gate_up", st, launch_quant(a, E, st));
+      MOE_LAUNCH(ctx, "gather_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
       w1_base = w.w1_copy;
       w1_stride = 2 * f * d * 2;
     }
@@ -565,7 +565,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       a.rows = d;
       a.cols = f;
       a.o_row = w.w2_copy;
-      MOE_LAUNCH(ctx, "gather_w_down", st, launch_quant(a, E, st));
+      MOE_LAUNCH(ctx, "gather_w_down", st, launch_quant(a, E, ctx->num_sms, st));
       w2_base = w.w2_copy;
       w2_stride = d * f * 2;
     }
@@ -581,7 +581,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.o_row = w.x_perm;
     xa.do_col = training;
     xa.o_colT = s.xT;
-    MOE_LAUNCH(ctx, "permute_x", st, launch_quant(xa, 1, st));
+    MOE_LAUNCH(ctx, "permute_x", st, launch_quant(xa, 1, ctx->num_sms, st));
   }
 
   // 3. gate_up GEMM + ScaledSwiGLU + requantisation of a
@@ -697,7 +697,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
       a.o_row = w.dy_perm;
       a.o_colT = w.dyT;
     }
-    MOE_LAUNCH(ctx, "gather_quantize_dy", st, launch_quant(a, 1, st));
+    MOE_LAUNCH(ctx, "gather_quantize_dy", st, launch_quant(a, 1, ctx->num_sms, st));
   }
   const void* w1c;  // B of dgrad of gate_up: [E, d, 2f]
   const void* w2c;  // B of dgrad of down:    [E, f, d]
@@ -713,13 +713,13 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     a.rows = 2 * f;
     a.cols = d;
     a.o_colT = w.w1T;
-    MOE_LAUNCH(ctx, "transpose_w_gate_up", st, launch_quant(a, E, st));
+    MOE_LAUNCH(ctx, "transpose_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
     a.src_ld = f;
     a.rows = d;
     a.cols = f;
     a.o_colT = w.w2T;
-    MOE_LAUNCH(ctx, "transpose_w_down", st, launch_quant(a, E, st));
+    MOE_LAUNCH(ctx, "transpose_w_down", st, launch_quant(a, E, ctx->num_sms, st));
     w1c = w.w1T;
     w2c = w.w2T;
   }
@@ -733,7 +733,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     g.kgrouped = 0;
     g.E = E;
     g.K = static_cast<int>(d);
-    g.n_tiles = static_cast<int>(f / 256);
+    g.n_tiles = static_cast<int>(f / gemm_tile_n(EPI_DSWIGLU));
     g.poffsets = s.poff;
     g.sfa = w.dy_s;
     g.sfa_kb4 = d / 128;
@@ -821,7 +821,8 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   }
   // 6. combine dx, reduce the probability gradient
   MOE_LAUNCH(ctx, "unpermute_dx", st, launch_unpermute(w.dx_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(dx), ctx->num_sms, st));
-  MOE_LAUNCH(ctx, "dprob_reduce", st, launch_dprob_reduce(w.dp_part, static_cast<int>(2 * (f / 256)), D.cap, s.src2s, D.Tk, d_topk_prob, st));
+  MOE_LAUNCH(ctx, "dprob_reduce", st, launch_dprob_reduce(w.dp_part, static_cast<int>(2 * (f / gemm_tile_n(EPI_DSWIGLU))), D.cap, s.src2s, D.Tk,
+                                           d_topk_prob, st));
   return MOE_OK;
 }
 

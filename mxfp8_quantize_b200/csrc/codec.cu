@@ -116,30 +116,24 @@ constexpr int QT_COLS = 128;
 constexpr int QT_PITCH = QT_COLS + 8;  // bf16 elements per smem row (padding against bank conflicts)
 constexpr int QT_LOADS = QT_ROWS * QT_COLS / 8 / 256;
 
-__device__ __forceinline__ uint32_t abs_bits_bf16x2_max(uint32_t w, uint32_t m) {
-  const uint32_t lo = (w & 0x7FFFu) << 16;
-  const uint32_t hi = (w & 0x7FFF0000u);
-  return max(m, max(lo, hi));
+// |a| and |b| of two bf16 pairs, max per half (max.bf16x2); inputs are finite.
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  a &= 0x7FFF7FFFu;
+  b &= 0x7FFF7FFFu;
+  __nv_bfloat162 r = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
 }
+// fp32 bits of the larger half of a bf16 pair of non-negative values
+__device__ __forceinline__ uint32_t fold_halves(uint32_t m2) { return max(m2 << 16, m2 & 0xFFFF0000u); }
 
-// E4M3 codes of 8 values, packed little-endian into two 32-bit words.
-__device__ __forceinline__ uint2 e4m3x8(const float* v) {
-  uint2 out;
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(make_float2(v[2 * i], v[2 * i + 1]), __NV_SATFINITE, __NV_E4M3);
-    w[i] = static_cast<uint32_t>(p);
-  }
-  out.x = w[0] | (w[1] << 16);
-  out.y = w[2] | (w[3] << 16);
-  return out;
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 }  // namespace
 
 __global__ void __launch_bounds__(256)
 quant_tile_kernel(QuantArgs a) {
-  __shared__ __align__(16) bf16 tile[QT_ROWS * QT_PITCH];
+  __shared__ __align__(16) uint32_t tile[QT_ROWS * QT_PITCH / 2];  // bf16 pairs
   const int tid = threadIdx.x;
   const int64_t row0 = static_cast<int64_t>(blockIdx.x) * QT_ROWS;
   const int64_t col0 = static_cast<int64_t>(blockIdx.y) * QT_COLS;
@@ -170,89 +164,98 @@ quant_tile_kernel(QuantArgs a) {
     }
   }
   // ---- row-wise outputs (and the smem copy for the column pass)
+  uint8_t* qbase = a.q_row + static_cast<int64_t>(b) * R * C + col;
+  uint8_t* sbase = a.s_row + static_cast<int64_t>(b) * R * KBr;
+  bf16* obase = a.o_row + static_cast<int64_t>(b) * R * C + col;
 #pragma unroll
   for (int i = 0; i < QT_LOADS; ++i) {
     const int lr = (tid >> 4) + 16 * i;
     const int64_t r = row0 + lr;
-    const bool valid_row = r < R;
+    const bool valid = r < R && col_ok;
     // destination row: identity, or the gate/up interleaving (128 rows from each half per 256-row group)
     int64_t dr = r;
     if (a.gate_up_half) {
       const int64_t hf = a.gate_up_half;
       dr = r < hf ? (r / 128) * 256 + (r % 128) : ((r - hf) / 128) * 256 + 128 + ((r - hf) % 128);
     }
-    if (a.do_col) *reinterpret_cast<uint4*>(&tile[lr * QT_PITCH + cchunk * 8]) = v[i];
-    if (a.do_row) {
-      if (a.mx) {
-        uint32_t m = 0;
-        m = abs_bits_bf16x2_max(v[i].x, m);
-        m = abs_bits_bf16x2_max(v[i].y, m);
-        m = abs_bits_bf16x2_max(v[i].z, m);
-        m = abs_bits_bf16x2_max(v[i].w, m);
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        const uint32_t sb = e8m0_from_amax_bits(m);
-        const float inv = e8m0_inv_scale(sb);
-        if (valid_row && col_ok) {
-          float f[8];
-          const bf16* h = reinterpret_cast<const bf16*>(&v[i]);
+    if (a.do_col) *reinterpret_cast<uint4*>(&tile[lr * (QT_PITCH / 2) + cchunk * 4]) = v[i];
+    if (!a.do_row) continue;
+    if (a.mx) {
+      uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w)));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      const uint32_t sb = e8m0_from_amax_bits(m);
+      const float inv = e8m0_inv_scale(sb);
+      if (valid) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        uint32_t q[4];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) f[j] = __bfloat162float(h[j]) * inv;
-          const uint2 q = e4m3x8(f);
-          uint8_t* qrow = a.q_row + (static_cast<int64_t>(b) * R + dr) * C + col;
-          *reinterpret_cast<uint2*>(qrow) = q;
-          if ((cchunk & 3) == 0) {
-            const int64_t kb = col / 32;
-            const int64_t off = a.sf_mma ? sf_mma_offset(dr, kb, KBr) : dr * KBr + kb;
-            a.s_row[static_cast<int64_t>(b) * R * KBr + off] = static_cast<uint8_t>(sb);
-          }
+        for (int j = 0; j < 4; ++j)
+          q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
+        *reinterpret_cast<uint2*>(qbase + dr * C) = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+        if ((cchunk & 3) == 0) {
+          const int64_t kb = col / 32;
+          sbase[a.sf_mma ? sf_mma_offset(dr, kb, KBr) : dr * KBr + kb] = static_cast<uint8_t>(sb);
         }
-      } else if (valid_row && col_ok) {
-        *reinterpret_cast<uint4*>(a.o_row + (static_cast<int64_t>(b) * R + dr) * C + col) = v[i];
       }
+    } else if (valid) {
+      *reinterpret_cast<uint4*>(obase + dr * C) = v[i];
     }
   }
   if (!a.do_col) return;
   __syncthreads();
 
-  // ---- column-wise: thread -> column c, two consecutive 32-row blocks
-  const int c = tid & 127;
-  const int64_t gc = col0 + c;
-  if (gc >= C) return;
+  // ---- column-wise: thread -> columns (2p, 2p+1) of the tile, 32-row block rb; each smem word
+  //      holds one row of both columns
+  const int p = tid & 63;
+  const int rb = tid >> 6;
+  const int64_t gc = col0 + 2 * p;
+  const int64_t gr = row0 + rb * 32;
+  if (gc >= C || gr >= R) return;
+  uint32_t wv[32];
+  uint32_t m2 = 0;
 #pragma unroll
-  for (int hb = 0; hb < 2; ++hb) {
-    const int rb = 2 * (tid >> 7) + hb;
-    const int64_t gr = row0 + rb * 32;
-    if (gr >= R) break;
-    float f[32];
-    uint32_t m = 0;
+  for (int i = 0; i < 32; ++i) {
+    wv[i] = tile[(rb * 32 + i) * (QT_PITCH / 2) + p];
+    m2 = absmax_bf16x2(m2, wv[i]);
+  }
+  if (a.mx) {
+    const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16), sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u);
+    const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
+    uint32_t q0[8], q1[8];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      f[i] = __bfloat162float(tile[(rb * 32 + i) * QT_PITCH + c]);
-      m = max(m, __float_as_uint(f[i]) & 0x7FFFFFFFu);
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t lo0 = e4m3x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0);
+      const uint32_t hi0 =
+          e4m3x2(__uint_as_float(wv[4 * i + 2] << 16) * inv0, __uint_as_float(wv[4 * i + 3] << 16) * inv0);
+      const uint32_t lo1 = e4m3x2(__uint_as_float(wv[4 * i] & 0xFFFF0000u) * inv1,
+                                  __uint_as_float(wv[4 * i + 1] & 0xFFFF0000u) * inv1);
+      const uint32_t hi1 = e4m3x2(__uint_as_float(wv[4 * i + 2] & 0xFFFF0000u) * inv1,
+                                  __uint_as_float(wv[4 * i + 3] & 0xFFFF0000u) * inv1);
+      q0[i] = lo0 | (hi0 << 16);
+      q1[i] = lo1 | (hi1 << 16);
     }
-    if (a.mx) {
-      const uint32_t sb = e8m0_from_amax_bits(m);
-      const float inv = e8m0_inv_scale(sb);
+    uint8_t* qc = a.q_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
+    reinterpret_cast<uint4*>(qc)[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+    reinterpret_cast<uint4*>(qc)[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+    reinterpret_cast<uint4*>(qc + R)[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+    reinterpret_cast<uint4*>(qc + R)[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+    const int64_t kb = gr / 32;
+    uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
+    sc[a.sf_mma ? sf_mma_offset(gc, kb, KBc) : gc * KBc + kb] = static_cast<uint8_t>(sb0);
+    sc[a.sf_mma ? sf_mma_offset(gc + 1, kb, KBc) : (gc + 1) * KBc + kb] = static_cast<uint8_t>(sb1);
+  } else {
+    uint32_t c0[16], c1[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) f[i] *= inv;
-      uint8_t* qc = a.q_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
-      const uint2 q0 = e4m3x8(f), q1 = e4m3x8(f + 8), q2 = e4m3x8(f + 16), q3 = e4m3x8(f + 24);
-      reinterpret_cast<uint4*>(qc)[0] = make_uint4(q0.x, q0.y, q1.x, q1.y);
-      reinterpret_cast<uint4*>(qc)[1] = make_uint4(q2.x, q2.y, q3.x, q3.y);
-      const int64_t kb = gr / 32;
-      const int64_t off = a.sf_mma ? sf_mma_offset(gc, kb, KBc) : gc * KBc + kb;
-      a.s_colT[static_cast<int64_t>(b) * C * KBc + off] = static_cast<uint8_t>(sb);
-    } else {
-      bf16* oc = a.o_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
+    for (int i = 0; i < 16; ++i) {
+      c0[i] = __byte_perm(wv[2 * i], wv[2 * i + 1], 0x5410);  // low halves: column 2p
+      c1[i] = __byte_perm(wv[2 * i], wv[2 * i + 1], 0x7632);  // high halves: column 2p+1
+    }
+    bf16* oc = a.o_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint4 w;
-        bf16* hw = reinterpret_cast<bf16*>(&w);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) hw[j] = tile[(rb * 32 + 8 * i + j) * QT_PITCH + c];
-        reinterpret_cast<uint4*>(oc)[i] = w;
-      }
+    for (int i = 0; i < 4; ++i) {
+      reinterpret_cast<uint4*>(oc)[i] = make_uint4(c0[4 * i], c0[4 * i + 1], c0[4 * i + 2], c0[4 * i + 3]);
+      reinterpret_cast<uint4*>(oc + R)[i] = make_uint4(c1[4 * i], c1[4 * i + 1], c1[4 * i + 2], c1[4 * i + 3]);
     }
   }
 }
@@ -338,7 +341,7 @@ cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant(const QuantArgs& a, int batch, cudaStream_t st) {
+cudaError_t launch_quant(const QuantArgs& a, int batch, int /*num_sms*/, cudaStream_t st) {
   if (a.rows == 0 || a.cols == 0 || batch == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(ceil_div(a.rows, QT_ROWS)), static_cast<unsigned>(ceil_div(a.cols, QT_COLS)),
             static_cast<unsigned>(batch));

@@ -31,7 +31,7 @@ struct QuantArgs {
 cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk, int E, int capacity,
                          const int32_t* split_in, int32_t* split_out, int32_t* poffsets, int32_t* sorted_to_src,
                          int32_t* src_to_sorted, float* prob_perm, int* status, cudaStream_t st);
-cudaError_t launch_quant(const QuantArgs& a, int batch, cudaStream_t st);
+cudaError_t launch_quant(const QuantArgs& a, int batch, int num_sms, cudaStream_t st);
 cudaError_t launch_unpermute(const bf16* rows, const int32_t* src_to_sorted, const float* probs, int64_t T, int k,
                              int64_t d, bf16* y, int num_sms, cudaStream_t st);
 cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_stride, const int32_t* src_to_sorted,

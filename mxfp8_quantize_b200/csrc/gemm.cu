@@ -55,8 +55,9 @@ struct Shape {
   static_assert(NBUF * BN + STAGES * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
   static_assert(SMEM_DYN + 4096 <= 232448, "shared memory budget");
 };
-using ShapeStore = Shape<256, 1, 4, false>;
-using ShapeFused = Shape<256, 1, 4, true>;
+using ShapeStore = Shape<256, 1, 4, false>;   // plain bf16-store epilogues
+using ShapeSwiglu = Shape<256, 1, 4, true>;   // gate_up + ScaledSwiGLU
+using ShapeDswiglu = Shape<128, 2, 6, true>;  // dgrad of down + dSwiGLU: epilogue overlaps the next tile
 
 struct SharedState {
   uint64_t full[8];
@@ -430,19 +431,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
 #pragma unroll
         for (int i = 0; i < BN / 16; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       } else if (EPI == EPI_SWIGLU) {
-        // tile = 128 output columns; accumulator columns [0,128) gate, [128,256) up
+        // tile = BN/2 output columns; accumulator columns [0,BN/2) gate, [BN/2,BN) up
+        constexpr int G = BN / 128;  // groups of 32 output columns per thread
         const float p = ep.p_perm[row];
         const int64_t f = ep.f;
         if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
         ptx::tc_fence_after();
         const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          const int64_t j = static_cast<int64_t>(tl.nb) * 128 + 64 * ch + 32 * cc;  // 32 output columns
+        for (int cc = 0; cc < G; ++cc) {
+          const int64_t j = static_cast<int64_t>(tl.nb) * (BN / 2) + (BN / 4) * ch + 32 * cc;  // 32 output columns
           float gv[32], uv[32];
-          load_acc32(t_lane + 64 * ch + 32 * cc, gv);
-          load_acc32(t_lane + 128 + 64 * ch + 32 * cc, uv);
-          if (cc == 1) {
+          load_acc32(t_lane + (BN / 4) * ch + 32 * cc, gv);
+          load_acc32(t_lane + BN / 2 + (BN / 4) * ch + 32 * cc, uv);
+          if (cc == G - 1) {
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
@@ -476,10 +478,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
             if (ep.o_colT) colwise_bf16(gv, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
           }
         }
-      } else {  // EPI_DSWIGLU: tile = 256 f-columns of da; this thread owns 128 of them
+      } else {  // EPI_DSWIGLU: tile = BN f-columns of da; this thread owns BN/2 of them
+        constexpr int G = BN / 64;  // groups of 32 columns per thread
         const float p = ep.p_perm[row];
         const int64_t f = ep.f, f2 = 2 * ep.f;
-        const int64_t j0 = static_cast<int64_t>(tl.nb) * BN + 128 * ch;
+        const int64_t j0 = static_cast<int64_t>(tl.nb) * BN + (BN / 2) * ch;
         const bf16* hrow = ep.h + row * f2;
         uint4 hg[4], hu[4];
 #pragma unroll
@@ -492,11 +495,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
         float dp = 0.f;
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < G; ++cc) {
           const int64_t j = j0 + 32 * cc;
           float da[32];
-          load_acc32(t_lane + 128 * ch + 32 * cc, da);
-          if (cc == 3) {
+          load_acc32(t_lane + (BN / 2) * ch + 32 * cc, da);
+          if (cc == G - 1) {
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
@@ -517,7 +520,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
               dp += d * sl * ux;
             }
           }
-          if (cc < 3) {
+          if (cc < G - 1) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {  // next group's saved values
               hg[i] = reinterpret_cast<const uint4*>(hrow + j + 32)[i];
@@ -577,17 +580,19 @@ cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
 }
 }  // namespace
 
-int gemm_tile_n(int epi) { return epi == EPI_STORE ? ShapeStore::BN : ShapeFused::BN; }
+int gemm_tile_n(int epi) {
+  return epi == EPI_STORE ? ShapeStore::BN : (epi == EPI_SWIGLU ? ShapeSwiglu::BN : ShapeDswiglu::BN);
+}
 
 cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st) {
   if (mx) {
     if (epi == EPI_STORE) return launch_t<true, EPI_STORE, ShapeStore>(args, num_sms, st);
-    if (epi == EPI_SWIGLU) return launch_t<true, EPI_SWIGLU, ShapeFused>(args, num_sms, st);
-    return launch_t<true, EPI_DSWIGLU, ShapeFused>(args, num_sms, st);
+    if (epi == EPI_SWIGLU) return launch_t<true, EPI_SWIGLU, ShapeSwiglu>(args, num_sms, st);
+    return launch_t<true, EPI_DSWIGLU, ShapeDswiglu>(args, num_sms, st);
   }
   if (epi == EPI_STORE) return launch_t<false, EPI_STORE, ShapeStore>(args, num_sms, st);
-  if (epi == EPI_SWIGLU) return launch_t<false, EPI_SWIGLU, ShapeFused>(args, num_sms, st);
-  return launch_t<false, EPI_DSWIGLU, ShapeFused>(args, num_sms, st);
+  if (epi == EPI_SWIGLU) return launch_t<false, EPI_SWIGLU, ShapeSwiglu>(args, num_sms, st);
+  return launch_t<false, EPI_DSWIGLU, ShapeDswiglu>(args, num_sms, st);
 }
 
 }  // namespace moemx

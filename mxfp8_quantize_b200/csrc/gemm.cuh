@@ -52,6 +52,9 @@ struct GemmArgs {
   EpiArgs epi;
 };
 
+// Output tile width (N) of the kernel used for an epilogue kind.
+int gemm_tile_n(int epi);
+
 // Launch one grouped GEMM.  ``mx``: MXFP8 (kind::mxf8f6f4) or BF16 (kind::f16).
 cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st);
 
