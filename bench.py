@@ -171,6 +171,21 @@ def time_oracle(cfg, m_tokens, f_slab, repeats):
     return flops, ts, desc
 
 
+# ------------------------------------------------------------------------------ replicas
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest ``value`` over all ranks (the job's step time is the slowest replica's)."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(cfg, ms_per_step: float, world: int) -> float:
+    """Whole-job algorithmic TFLOP/s: every rank runs its own replica of the layer."""
+    return world * cfg.flops_fwd_bwd() / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------------------ GPU arm
 def run_ours(args, cfg, rank, world, local_rank):
     import mxfp8_quantize_b200 as moe
@@ -309,19 +324,12 @@ def run_ours(args, cfg, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        ms_e2e = e0.elapsed_time(e1) / n2
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": round(world * cfg.flops_fwd_bwd() / (ms_e2e * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n2, world, dev)
+        e2e = {"value": round(job_tflops(cfg, ms_e2e, world), 2), "unit": "TFLOP/s",
                "ms_per_step": round(ms_e2e, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "tokens_per_s": round(world * T / (ms_e2e * 1e-3), 1)}
 
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     return dict(ms=ms, kernels=kern, roofline=roofline, clocks=clk, e2e=e2e, launches=launches)
 
 
@@ -384,7 +392,7 @@ def main():
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
-    tflops = world * cfg.flops_fwd_bwd() / (res["ms"] * 1e-3) / 1e12
+    tflops = job_tflops(cfg, res["ms"], world)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         flops, ts, desc = time_oracle(cfg, 2048, 512, 2)
