@@ -195,6 +195,32 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
                                  void* const* dw_down, float* d_topk_prob, void* workspace, size_t workspace_bytes,
                                  void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Inference forward without any device allocation (no counterpart on the pages; this is a
+ * deployment convenience).  Some callers cannot allocate device memory when they run the layer:
+ * a serving loop whose device memory is entirely owned by its own pool allocator, or a host
+ * framework whose extensions may not call cudaMalloc / cudaFree on the hot path (those calls can
+ * synchronise the device and fail once the pool has taken the memory).  This entry point computes
+ * exactly what moe_grouped_mlp_fwd computes with training = 0, but takes no context and no
+ * workspace: its scratch is one file-scope device array of MOE_NOALLOC_SCRATCH_BYTES that every
+ * GPU which loads the library holds until the process exits.
+ *  - It runs on the current CUDA device.  The first call on a device looks up that array's device
+ *    address (and checks the device); make that first call before any stream capture.
+ *  - Sizes whose forward workspace (moe_fwd_workspace_size with training = 0) exceeds
+ *    MOE_NOALLOC_SCRATCH_BYTES are rejected with MOE_ERR_WORKSPACE before anything is enqueued.
+ *  - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *  - Every call uses the same array, so calls that overlap on the GPU (different streams, or
+ *    different host threads) race and must be serialised by the caller.  Nothing in the array
+ *    needs to start at zero: each call writes every scratch byte it later reads.
+ *  - device_status: optional device int; kernels OR MOE_ERR_DEVICE-type findings into it as bit 1
+ *    (bad expert index / split_sizes mismatch) and bit 2 (a bounded wait expired).  NULL drops them.
+ * Arguments and layouts are those of moe_grouped_mlp_fwd. */
+#define MOE_NOALLOC_SCRATCH_BYTES (64u << 20)
+moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx, const float* topk_prob,
+                                         const int32_t* split_sizes, const void* const* w_gate_up,
+                                         const void* const* w_down, int64_t T, int64_t d, int64_t f, int E, int k,
+                                         moe_precision_t prec, void* y, int* device_status, void* stream);
+
 /* Inspection hook (tests): address of a named intermediate inside a saved buffer (which = 0),
  * a forward workspace (which = 1) or a backward workspace (which = 2) laid out for these
  * dimensions, given the buffer's base address ``base``; NULL for an unknown name.  Names:

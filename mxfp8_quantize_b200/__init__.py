@@ -29,7 +29,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "unsupported", 4: "cuda
 EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_get_status", "moe_ctx_set_debug_dump", "moe_status_string",
            "mxfp8_quantize", "mxfp8_dequantize", "moe_capacity_rows", "moe_permute", "moe_unpermute",
            "moe_saved_size", "moe_fwd_workspace_size", "moe_bwd_workspace_size", "moe_grouped_mlp_fwd",
-           "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook"]
+           "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook", "moe_grouped_mlp_fwd_noalloc"]
 
 LAUNCH_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_grouped_mlp_bwd": (c_int, [c_vp, c_vp, c_vp, c_size, c_vp, c_vp, c_i64, c_i64, c_i64, c_int, c_int,
                                         c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
         "moe_ctx_set_launch_hook": (c_int, [c_vp, LAUNCH_HOOK, c_vp]),
+        "moe_grouped_mlp_fwd_noalloc": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_int, c_int,
+                                                c_int, c_vp, c_vp, c_vp]),
         "moe_buffer_address": (c_vp, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int, c_int, c_vp,
                                       ctypes.c_char_p]),
     }
@@ -284,6 +286,31 @@ def moe_grouped_mlp_fwd(x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torc
         y.data_ptr(), _ptr(saved.buf) if training else None, saved.buf.numel() if training else 0,
         workspace.data_ptr(), workspace.numel(), _stream(dev)))
     return y, (saved if training else None)
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def moe_grouped_mlp_fwd_noalloc(x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor,
+                                w_gate_up: Weights, w_down: Weights, precision: str = "mxfp8",
+                                y: Optional[torch.Tensor] = None, device_status: Optional[torch.Tensor] = None,
+                                split_sizes: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Inference forward that allocates no device memory inside the call (scratch is a static
+    device array of NOALLOC_SCRATCH_BYTES; see include/moemx.h).  ``y`` may be preallocated."""
+    dev = _device_index(x)
+    T, d = x.shape
+    E = len(w_gate_up)
+    f = w_down[0].shape[1]
+    k = topk_idx.shape[1]
+    if y is None:
+        y = torch.empty((T, d), dtype=torch.bfloat16, device=x.device)
+    L = load_library()
+    with torch.cuda.device(dev):
+        _check("moe_grouped_mlp_fwd_noalloc", L.moe_grouped_mlp_fwd_noalloc(
+            x.data_ptr(), topk_idx.data_ptr(), topk_prob.data_ptr(), _ptr(split_sizes), _ptr_array(w_gate_up, E),
+            _ptr_array(w_down, E), T, d, f, E, k, PRECISIONS[precision], y.data_ptr(), _ptr(device_status),
+            _stream(dev)))
+    return y
 
 
 def moe_grouped_mlp_bwd(dy: torch.Tensor, saved: Saved, w_gate_up: Weights, w_down: Weights,

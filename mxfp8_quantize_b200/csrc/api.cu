@@ -876,4 +876,70 @@ void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_prec
   return nullptr;
 }
 
+// ---- forward without allocation: file-scope scratch, looked up once per device
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+static __device__ __align__(256) int g_noalloc_status[64];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+struct NoAllocDevice {
+  bool ready;
+  int num_sms;
+  void* scratch;  // device address of g_noalloc_scratch on this device
+  int* status;    // device address of g_noalloc_status on this device
+};
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+std::mutex g_noalloc_mu;
+
+moe_status_t noalloc_setup(int dev, NoAllocDevice& out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& nd = g_noalloc_dev[dev];
+  if (!nd.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED;
+    if (!encoder()) return MOE_ERR_CUDA;
+    void* scratch = nullptr;
+    void* status = nullptr;
+    // host code must not use the arrays' names as device addresses: ask the runtime, with ``dev`` current
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaGetSymbolAddress(&status, g_noalloc_status) != cudaSuccess) return MOE_ERR_CUDA;
+    nd.num_sms = sms;
+    nd.scratch = scratch;
+    nd.status = static_cast<int*>(status);
+    nd.ready = true;
+  }
+  out = nd;
+  return MOE_OK;
+}
+}  // namespace
+
+moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx, const float* topk_prob,
+                                         const int32_t* split_sizes, const void* const* w_gate_up,
+                                         const void* const* w_down, int64_t T, int64_t d, int64_t f, int E, int k,
+                                         moe_precision_t prec, void* y, int* device_status, void* stream) {
+  const moe_status_t dc = check_dims(T, d, f, E, k);
+  if (dc != MOE_OK) return dc;
+  if (moe_fwd_workspace_size(T, k, E, d, f, prec, 0) > MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_CUDA;
+  NoAllocDevice nd;
+  const moe_status_t st = noalloc_setup(dev, nd);
+  if (st != MOE_OK) return st;
+  // a context on the stack: no debug hooks, status into the caller's word (or the static one)
+  moe_ctx_s c;
+  c.device = dev;
+  c.num_sms = nd.num_sms;
+  c.d_status = device_status ? device_status : nd.status;
+  c.dbg_a = c.dbg_dh = nullptr;
+  c.hook = nullptr;
+  c.hook_user = nullptr;
+  // the scratch base is 256-aligned; the workspace carving aligns to 1 KiB inside the size bound
+  return moe_grouped_mlp_fwd(&c, x, topk_idx, topk_prob, split_sizes, w_gate_up, w_down, T, d, f, E, k, prec, 0, y,
+                             nullptr, 0, nd.scratch, MOE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 }  // extern "C"
