@@ -160,7 +160,8 @@ def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: in
 def backward(dy, state, w_gate_up, w_down):
     """Gradients of the forward in ``state`` for upstream gradient dy [T, d].
 
-    Returns dict(dx [T,d], dw_gate_up [E,2f,d], dw_down [E,d,f], d_topk_prob [T,k]).
+    Returns dict(dx [T,d], dw_gate_up [E,2f,d], dw_down [E,d,f], d_topk_prob [T,k]) and the
+    per-row intermediates dx_perm, dh_perm (= [dg, du]) and dp_perm of the padded expert rows.
     dW of an expert that received no tokens is exactly zero.
     """
     precision = state["precision"]
@@ -171,6 +172,7 @@ def backward(dy, state, w_gate_up, w_down):
     dy = np.asarray(dy, dtype=np.float64)
 
     dx_perm = np.zeros((Tp, d))
+    dh_perm = np.zeros((Tp, 2 * f))
     dp_perm = np.zeros(Tp)
     dW1 = np.zeros((E, 2 * f, d))
     dW2 = np.zeros((E, d, f))
@@ -214,12 +216,14 @@ def backward(dy, state, w_gate_up, w_down):
         dx_perm[lo:hi] = _round_out(gemm(dh, W1, precision), precision)
         dW1[e] = _round_out(gemm(np.asarray(dh, dtype=np.float64).T, Xe, precision), precision)
         dp_perm[lo:hi] = dp
+        dh_perm[lo:hi] = dh
 
     dx = _combine(dx_perm, r["src_to_sorted"], T, k, precision)
     d_prob = dp_perm[r["src_to_sorted"]].reshape(T, k)
     if precision != "fp64":
         d_prob = d_prob.astype(np.float32)
-    return dict(dx=dx, dw_gate_up=dW1, dw_down=dW2, d_topk_prob=d_prob, dx_perm=dx_perm, dp_perm=dp_perm)
+    return dict(dx=dx, dw_gate_up=dW1, dw_down=dW2, d_topk_prob=d_prob, dx_perm=dx_perm, dh_perm=dh_perm,
+                dp_perm=dp_perm)
 
 
 def unpermute(y_perm, src_to_sorted, T, k, probs=None):
