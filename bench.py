@@ -283,7 +283,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
-        traffic = json.load(open(tpath)).get(cfg.name, {}).get(dom)
+        import hashlib
+        rec = json.load(open(tpath))
+        src = os.path.join(ROOT, "mxfp8_quantize_b200", "csrc", "gemm.cu")
+        if hashlib.sha1(open(src, "rb").read()).hexdigest()[:12] == rec.get("gemm_cu_sha1"):
+            traffic = rec.get(cfg.name, {}).get(dom)  # counters taken on this very kernel source
     roofline = {"bound": kind, "kernel": dom, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": (f"{peak_src}: bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s"
