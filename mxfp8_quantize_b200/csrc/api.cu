@@ -346,7 +346,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
   if (cols % 32) return MOE_ERR_SHAPE;
   if (col && rows % 32) return MOE_ERR_SHAPE;
   if (mma && (rows % 128 || cols % 128)) return MOE_ERR_SHAPE;
-  if (batch > MOE_MAX_EXPERTS * 256 || rows > (int64_t(1) << 31) / 64 * 64 || cols > (int64_t(1) << 31))
+  if (batch > 65535 || ceil_div(rows, 128) > 65535 || ceil_div(cols, 128) > (int64_t(1) << 31) - 1)
     return MOE_ERR_UNSUPPORTED;
   if (!aligned16(x) || (row && !aligned16(q_row)) || (col && !aligned16(q_colT))) return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->device);

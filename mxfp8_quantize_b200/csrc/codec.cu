@@ -135,8 +135,9 @@ __global__ void __launch_bounds__(256)
 quant_tile_kernel(QuantArgs a) {
   __shared__ __align__(16) uint32_t tile[QT_ROWS * QT_PITCH / 2];  // bf16 pairs
   const int tid = threadIdx.x;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * QT_ROWS;
-  const int64_t col0 = static_cast<int64_t>(blockIdx.y) * QT_COLS;
+  // column tiles vary fastest so that CTAs running together read whole contiguous rows
+  const int64_t row0 = static_cast<int64_t>(blockIdx.y) * QT_ROWS;
+  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * QT_COLS;
   const int b = blockIdx.z;
   const int64_t R = a.rows, C = a.cols, KBr = C / 32, KBc = R / 32;
 
@@ -343,7 +344,7 @@ cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk
 
 cudaError_t launch_quant(const QuantArgs& a, int batch, int /*num_sms*/, cudaStream_t st) {
   if (a.rows == 0 || a.cols == 0 || batch == 0) return cudaSuccess;
-  dim3 grid(static_cast<unsigned>(ceil_div(a.rows, QT_ROWS)), static_cast<unsigned>(ceil_div(a.cols, QT_COLS)),
+  dim3 grid(static_cast<unsigned>(ceil_div(a.cols, QT_COLS)), static_cast<unsigned>(ceil_div(a.rows, QT_ROWS)),
             static_cast<unsigned>(batch));
   quant_tile_kernel<<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
