@@ -31,16 +31,20 @@ namespace moemx {
 namespace {
 
 constexpr int BM = 128;
-constexpr int EPI_WARPS = 8;
-constexpr int NUM_THREADS = 32 * (4 + EPI_WARPS);
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int STAGE_PITCH = 17;  // floats per row of an epilogue warp's 32 x 16 transpose buffer (odd: no bank conflicts)
 
-template <int BN_, int NBUF_, int STAGES_, bool STAGING_>
+// Tile shape and thread layout of one kernel instance.
+//   EPI_WARPS epilogue warps (a multiple of 4: each TMEM lane quadrant gets EPI_WARPS/4 warps that
+//   split the tile's columns); PASS columns per pass of the column-wise transpose buffer.
+template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_>
 struct Shape {
   static constexpr int BN = BN_;
   static constexpr int NBUF = NBUF_;
   static constexpr int STAGES = STAGES_;
+  static constexpr int EPI_WARPS = EPI_WARPS_;
+  static constexpr int NUM_THREADS = 32 * (4 + EPI_WARPS);
+  static constexpr int PASS = PASS_;
+  static constexpr int PITCH = PASS + 1;  // odd pitch: conflict-free row writes and column reads
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int SFB_BYTES = (BN / 128) * 512;
@@ -50,14 +54,15 @@ struct Shape {
   static constexpr int STAGE_BYTES = (OFF_SFB + SFB_BYTES + 1023) / 1024 * 1024;
   static constexpr int SF_COLS = 4 + 4 * (BN / 128);
   static constexpr uint32_t SF_TMEM_COL = NBUF * BN;
-  static constexpr int STAGING_PER_WARP = STAGING_ ? (32 * STAGE_PITCH * 4 + 15) / 16 * 16 : 0;
+  static constexpr int STAGING_PER_WARP = STAGING_ ? (32 * PITCH * 4 + 15) / 16 * 16 : 0;
   static constexpr int SMEM_DYN = STAGES * STAGE_BYTES + EPI_WARPS * STAGING_PER_WARP + 1024;
   static_assert(NBUF * BN + STAGES * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
   static_assert(SMEM_DYN + 4096 <= 232448, "shared memory budget");
+  static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0, "thread layout");
 };
-using ShapeStore = Shape<256, 1, 4, false>;   // plain bf16-store epilogues
-using ShapeSwiglu = Shape<256, 1, 4, true>;   // gate_up + ScaledSwiGLU
-using ShapeDswiglu = Shape<128, 2, 6, true>;  // dgrad of down + dSwiGLU: epilogue overlaps the next tile
+using ShapeStore = Shape<256, 1, 4, false, 8, 16>;    // plain bf16-store epilogues
+using ShapeSwiglu = Shape<256, 1, 4, true, 16, 8>;    // gate_up + ScaledSwiGLU: one 32-column group per thread
+using ShapeDswiglu = Shape<128, 2, 6, true, 8, 16>;   // dgrad of down + dSwiGLU: epilogue overlaps the next tile
 
 struct SharedState {
   uint64_t full[8];
@@ -155,54 +160,64 @@ __device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q) {
   return sb;
 }
 
-// Column-wise outputs of a 32 x 32 block held one row per lane (v = this lane's 32 values), in two
-// passes of 16 columns through the warp's padded smem buffer: after a pass lane l holds column
-// c = l % 16 of the pass, rows 16*(l/16) .. +16.
-template <class F>
+// Column-wise outputs of a 32 x 32 block held one row per lane (v = this lane's 32 values), in
+// 32/P passes of P columns through the warp's padded smem buffer: after a pass lane l holds column
+// c = l % P of the pass, rows P*(l/P) .. +P.
+template <int P, class F>
 __device__ __forceinline__ void column_passes(const float* v, float* stage, F&& emit) {
   const int lane = threadIdx.x & 31;
+  constexpr int PITCH = P + 1;
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < 32 / P; ++h) {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) stage[lane * STAGE_PITCH + c] = v[16 * h + c];
+    for (int c = 0; c < P; ++c) stage[lane * PITCH + c] = v[P * h + c];
     __syncwarp();
-    float col[16];
-    const int cl = lane & 15, rh = lane >> 4;
+    float col[P];
+    const int cl = lane % P, rg = lane / P;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) col[i] = stage[(16 * rh + i) * STAGE_PITCH + cl];
+    for (int i = 0; i < P; ++i) col[i] = stage[(P * rg + i) * PITCH + cl];
     __syncwarp();
-    emit(h, cl, rh, col);
+    emit(h, cl, rg, col);
   }
 }
 
 // Column-wise MXFP8 of a 32 x 32 block (rows = lanes): each column is quantised with the scale of
 // its 32 values; column c's 32 codes go to colT + c * ld, its scale to S[sf_row0 + c][sf_kb] of a
 // tile-layout scale matrix with sf_KB columns.
+template <int P>
 __device__ __forceinline__ void colwise_mx(const float* v, float* stage, uint8_t* colT, int64_t ld, uint8_t* sf,
                                            int64_t sf_row0, int64_t sf_kb, int64_t sf_KB) {
-  column_passes(v, stage, [&](int h, int cl, int rh, const float* col) {
+  column_passes<P>(v, stage, [&](int h, int cl, int rg, const float* col) {
     uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = max(m, __float_as_uint(col[i]) & 0x7FFFFFFFu);
-    m = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
+    for (int i = 0; i < P; ++i) m = max(m, __float_as_uint(col[i]) & 0x7FFFFFFFu);
+#pragma unroll
+    for (int s = P; s < 32; s <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, s));
     const uint32_t sb = e8m0_from_amax_bits(m);
     const float inv = e8m0_inv_scale(sb);
-    uint32_t w[4];
+    uint32_t w[P / 4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < P / 4; ++i)
       w[i] = e4m3x2(col[4 * i] * inv, col[4 * i + 1] * inv) | (e4m3x2(col[4 * i + 2] * inv, col[4 * i + 3] * inv) << 16);
-    const int c = 16 * h + cl;
-    *reinterpret_cast<uint4*>(colT + c * ld + 16 * rh) = make_uint4(w[0], w[1], w[2], w[3]);
-    if (rh == 0) sf[sf_mma_offset(sf_row0 + c, sf_kb, sf_KB)] = static_cast<uint8_t>(sb);
+    const int c = P * h + cl;
+    uint8_t* dst = colT + c * ld + P * rg;
+    if constexpr (P == 16) {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      static_assert(P == 8, "pass width");
+      *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    }
+    if (rg == 0) sf[sf_mma_offset(sf_row0 + c, sf_kb, sf_KB)] = static_cast<uint8_t>(sb);
   });
 }
 
 // Column-wise bf16 of a 32 x 32 block: column c (32 bf16) goes to colT + c * ld.
+template <int P>
 __device__ __forceinline__ void colwise_bf16(const float* v, float* stage, bf16* colT, int64_t ld) {
-  column_passes(v, stage, [&](int h, int cl, int rh, const float* col) {
-    uint4* dst = reinterpret_cast<uint4*>(colT + (16 * h + cl) * ld + 16 * rh);
-    dst[0] = pack_bf16x8(col);
-    dst[1] = pack_bf16x8(col + 8);
+  column_passes<P>(v, stage, [&](int h, int cl, int rg, const float* col) {
+    uint4* dst = reinterpret_cast<uint4*>(colT + (P * h + cl) * ld + P * rg);
+#pragma unroll
+    for (int i = 0; i < P / 8; ++i) dst[i] = pack_bf16x8(col + 8 * i);
   });
 }
 
@@ -217,7 +232,7 @@ __device__ __forceinline__ void load_acc32(uint32_t taddr, float* v) {
 }  // namespace
 
 template <bool MX, int EPI, class S>
-__global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs g) {
+__global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs g) {
   __shared__ SharedState s;
   extern __shared__ uint8_t dyn_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
@@ -246,7 +261,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     }
     for (int i = 0; i < S::NBUF; ++i) {
       ptx::mbar_init(&s.acc_full[i], 1);
-      ptx::mbar_init(&s.acc_empty[i], EPI_WARPS);
+      ptx::mbar_init(&s.acc_empty[i], S::EPI_WARPS);
     }
     ptx::mbar_init(&s.drain, 1);
     ptx::fence_mbar_init();
@@ -385,7 +400,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   } else if (warp >= 4) {
     // ================= epilogue
     const int q = warp & 3;          // TMEM lane quadrant this warp may read
-    const int ch = (warp - 4) >> 2;  // column half of the tile
+    const int ch = (warp - 4) >> 2;  // which of the quadrant's EPI_WARPS/4 column parts this warp owns
+    constexpr int NPART = S::EPI_WARPS / 4;
     float* stage_buf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(staging_base) +
                                                 (warp - 4) * S::STAGING_PER_WARP);
     const EpiArgs& ep = g.epi;
@@ -399,10 +415,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         // K-grouped expert without tokens: its weight gradient is zero
         if (EPI == EPI_STORE) {
           bf16* out = static_cast<bf16*>(const_cast<void*>(ep.out_ptrs.p[tl.e]));
-          const int64_t c0 = static_cast<int64_t>(tl.nb) * BN + (BN / 2) * ch;
+          const int64_t c0 = static_cast<int64_t>(tl.nb) * BN + (BN / NPART) * ch;
           uint4* dst = reinterpret_cast<uint4*>(out + row * ep.ldo + c0);
 #pragma unroll 4
-          for (int i = 0; i < BN / 16; ++i) dst[i] = make_uint4(0, 0, 0, 0);
+          for (int i = 0; i < BN / NPART / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
         }
         continue;
       }
@@ -415,11 +431,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
         ptx::tc_fence_after();
         const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
-        uint32_t pk[BN / 4];
+        constexpr int CPT = BN / NPART;  // columns per thread
+        uint32_t pk[CPT / 2];
 #pragma unroll
-        for (int cc = 0; cc < BN / 64; ++cc) {
+        for (int cc = 0; cc < CPT / 32; ++cc) {
           float v[32];
-          load_acc32(t_lane + (BN / 2) * ch + 32 * cc, v);
+          load_acc32(t_lane + CPT * ch + 32 * cc, v);
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[16 * cc + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
         }
@@ -427,12 +444,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
         bf16* out = g.kgrouped ? static_cast<bf16*>(const_cast<void*>(ep.out_ptrs.p[tl.e])) : ep.out;
-        uint4* dst = reinterpret_cast<uint4*>(out + row * ep.ldo + static_cast<int64_t>(tl.nb) * BN + (BN / 2) * ch);
+        uint4* dst = reinterpret_cast<uint4*>(out + row * ep.ldo + static_cast<int64_t>(tl.nb) * BN + CPT * ch);
 #pragma unroll
-        for (int i = 0; i < BN / 16; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int i = 0; i < CPT / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
       } else if (EPI == EPI_SWIGLU) {
         // tile = BN/2 output columns; accumulator columns [0,BN/2) gate, [BN/2,BN) up
-        constexpr int G = BN / 128;  // groups of 32 output columns per thread
+        constexpr int OPT = BN / 2 / NPART;  // output columns per thread
+        constexpr int G = OPT / 32;          // groups of 32 output columns per thread
         const float p = ep.p_perm[row];
         const int64_t f = ep.f;
         if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
@@ -440,10 +458,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
         for (int cc = 0; cc < G; ++cc) {
-          const int64_t j = static_cast<int64_t>(tl.nb) * (BN / 2) + (BN / 4) * ch + 32 * cc;  // 32 output columns
+          const int64_t j = static_cast<int64_t>(tl.nb) * (BN / 2) + OPT * ch + 32 * cc;  // 32 output columns
           float gv[32], uv[32];
-          load_acc32(t_lane + (BN / 4) * ch + 32 * cc, gv);
-          load_acc32(t_lane + BN / 2 + (BN / 4) * ch + 32 * cc, uv);
+          load_acc32(t_lane + OPT * ch + 32 * cc, gv);
+          load_acc32(t_lane + BN / 2 + OPT * ch + 32 * cc, uv);
           if (cc == G - 1) {
             ptx::tc_fence_before();
             __syncwarp();
@@ -469,20 +487,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
             const uint32_t sb = quant32_store(gv, ep.q_row + row * f + j);
             ep.s_row[sf_mma_offset(row, j / 32, f / 32)] = static_cast<uint8_t>(sb);
             if (ep.q_colT)
-              colwise_mx(gv, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
-                         ep.cap / 32);
+              colwise_mx<S::PASS>(gv, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
+                                  ep.cap / 32);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(ep.o_row + row * f + j);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = pack_bf16x8(gv + 8 * i);
-            if (ep.o_colT) colwise_bf16(gv, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
+            if (ep.o_colT) colwise_bf16<S::PASS>(gv, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
           }
         }
       } else {  // EPI_DSWIGLU: tile = BN f-columns of da; this thread owns BN/2 of them
-        constexpr int G = BN / 64;  // groups of 32 columns per thread
+        constexpr int CPT = BN / NPART;  // da columns per thread
+        constexpr int G = CPT / 32;      // groups of 32 columns per thread
         const float p = ep.p_perm[row];
         const int64_t f = ep.f, f2 = 2 * ep.f;
-        const int64_t j0 = static_cast<int64_t>(tl.nb) * BN + (BN / 2) * ch;
+        const int64_t j0 = static_cast<int64_t>(tl.nb) * BN + CPT * ch;
         const bf16* hrow = ep.h + row * f2;
         uint4 hg[4], hu[4];
 #pragma unroll
@@ -498,7 +517,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         for (int cc = 0; cc < G; ++cc) {
           const int64_t j = j0 + 32 * cc;
           float da[32];
-          load_acc32(t_lane + (BN / 2) * ch + 32 * cc, da);
+          load_acc32(t_lane + CPT * ch + 32 * cc, da);
           if (cc == G - 1) {
             ptx::tc_fence_before();
             __syncwarp();
@@ -541,9 +560,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
             ep.s_row[sf_mma_offset(row, j / 32, f2 / 32)] = static_cast<uint8_t>(sb);
             sb = quant32_store(du, ep.q_row + row * f2 + f + j);
             ep.s_row[sf_mma_offset(row, (f + j) / 32, f2 / 32)] = static_cast<uint8_t>(sb);
-            colwise_mx(dg, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32, ep.cap / 32);
-            colwise_mx(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j, row_w / 32,
-                       ep.cap / 32);
+            colwise_mx<S::PASS>(dg, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
+                                ep.cap / 32);
+            colwise_mx<S::PASS>(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j,
+                                row_w / 32, ep.cap / 32);
           } else {
             uint4* d0 = reinterpret_cast<uint4*>(ep.o_row + row * f2 + j);
             uint4* d1 = reinterpret_cast<uint4*>(ep.o_row + row * f2 + f + j);
@@ -552,8 +572,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
               d0[i] = pack_bf16x8(dg + 8 * i);
               d1[i] = pack_bf16x8(du + 8 * i);
             }
-            colwise_bf16(dg, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
-            colwise_bf16(du, stage_buf, ep.o_colT + (f + j) * ep.cap + row_w, ep.cap);
+            colwise_bf16<S::PASS>(dg, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
+            colwise_bf16<S::PASS>(du, stage_buf, ep.o_colT + (f + j) * ep.cap + row_w, ep.cap);
           }
         }
         ep.dp_part[(static_cast<int64_t>(tl.nb) * 2 + ch) * ep.cap + row] = dp;
@@ -575,7 +595,7 @@ cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
   auto kern = grouped_gemm_kernel<MX, EPI, S>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_DYN);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms, NUM_THREADS, S::SMEM_DYN, st>>>(args);
+  kern<<<num_sms, S::NUM_THREADS, S::SMEM_DYN, st>>>(args);
   return cudaGetLastError();
 }
 }  // namespace
