@@ -728,7 +728,8 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   {
     GemmArgs g = gemm_args(ctx);
     const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dy_q) : w.dy_perm, D.mx, d, D.cap, d * es) &&
-                    map_3d(&g.tmap_b, w2c, D.mx, d, f, E, d * es, f * d * es);
+                    map_3d(&g.tmap_b, w2c, D.mx, d, f, E, d * es, f * d * es) &&
+                    map_2d(&g.tmap_h, s.h, false, 2 * f, D.cap, 2 * f * 2);  // bf16 boxes of 128 rows x 64 columns
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;

@@ -131,88 +131,12 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 }
 }  // namespace
 
-__global__ void __launch_bounds__(256)
-quant_tile_kernel(QuantArgs a) {
-  __shared__ __align__(16) uint32_t tile[QT_ROWS * QT_PITCH / 2];  // bf16 pairs
-  const int tid = threadIdx.x;
-  // column tiles vary fastest so that CTAs running together read whole contiguous rows
-  const int64_t row0 = static_cast<int64_t>(blockIdx.y) * QT_ROWS;
-  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * QT_COLS;
-  const int b = blockIdx.z;
-  const int64_t R = a.rows, C = a.cols, KBr = C / 32, KBc = R / 32;
-
-  const bf16* src = a.src_ptrs.p[0] ? static_cast<const bf16*>(a.src_ptrs.p[b])
-                                    : static_cast<const bf16*>(a.src) + static_cast<int64_t>(b) * a.src_batch_stride;
-
-  // ---- load 128 x 128: 8 chunks of 8 bf16 per thread, all issued before any use
-  const int cchunk = tid & 15;
-  const int64_t col = col0 + cchunk * 8;
-  const bool col_ok = col < C;
-  uint4 v[QT_LOADS];
-#pragma unroll
-  for (int i = 0; i < QT_LOADS; ++i) {
-    const int64_t r = row0 + (tid >> 4) + 16 * i;
-    v[i] = make_uint4(0, 0, 0, 0);
-    if (r < R && col_ok) {
-      int64_t sr = r;
-      bool zero = false;
-      if (a.sorted_to_src) {
-        const int32_t s = a.sorted_to_src[r];
-        zero = s < 0;
-        sr = zero ? 0 : static_cast<int64_t>(s / a.k);
-      }
-      if (!zero) v[i] = __ldg(reinterpret_cast<const uint4*>(src + sr * a.src_ld + col));
-    }
-  }
-  // ---- row-wise outputs (and the smem copy for the column pass)
-  uint8_t* qbase = a.q_row + static_cast<int64_t>(b) * R * C + col;
-  uint8_t* sbase = a.s_row + static_cast<int64_t>(b) * R * KBr;
-  bf16* obase = a.o_row + static_cast<int64_t>(b) * R * C + col;
-#pragma unroll
-  for (int i = 0; i < QT_LOADS; ++i) {
-    const int lr = (tid >> 4) + 16 * i;
-    const int64_t r = row0 + lr;
-    const bool valid = r < R && col_ok;
-    // destination row: identity, or the gate/up interleaving (128 rows from each half per 256-row group)
-    int64_t dr = r;
-    if (a.gate_up_half) {
-      const int64_t hf = a.gate_up_half;
-      dr = r < hf ? (r / 128) * 256 + (r % 128) : ((r - hf) / 128) * 256 + 128 + ((r - hf) % 128);
-    }
-    if (a.do_col) *reinterpret_cast<uint4*>(&tile[lr * (QT_PITCH / 2) + cchunk * 4]) = v[i];
-    if (!a.do_row) continue;
-    if (a.mx) {
-      uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w)));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      const uint32_t sb = e8m0_from_amax_bits(m);
-      const float inv = e8m0_inv_scale(sb);
-      if (valid) {
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-        uint32_t q[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
-        *reinterpret_cast<uint2*>(qbase + dr * C) = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
-        if ((cchunk & 3) == 0) {
-          const int64_t kb = col / 32;
-          sbase[a.sf_mma ? sf_mma_offset(dr, kb, KBr) : dr * KBr + kb] = static_cast<uint8_t>(sb);
-        }
-      }
-    } else if (valid) {
-      *reinterpret_cast<uint4*>(obase + dr * C) = v[i];
-    }
-  }
-  if (!a.do_col) return;
-  __syncthreads();
-
-  // ---- column-wise: thread -> columns (2p, 2p+1) of the tile, 32-row block rb; each smem word
-  //      holds one row of both columns
-  const int p = tid & 63;
-  const int rb = tid >> 6;
-  const int64_t gc = col0 + 2 * p;
-  const int64_t gr = row0 + rb * 32;
-  if (gc >= C || gr >= R) return;
+// Column-wise outputs of one thread: columns (2p, 2p+1) of the tile and 32-row block rb (each smem
+// word holds one row of both columns).  Scales go to the block's 512-byte scale tile in smem when
+// the tensor-core layout is requested, else straight to the row-major scale matrix.
+__device__ __forceinline__ void column_pass(const QuantArgs& a, const uint32_t* tile, int p, int rb, int64_t gc,
+                                            int64_t gr, int b, uint8_t* satom_col) {
+  const int64_t R = a.rows, C = a.cols, KBc = R / 32;
   uint32_t wv[32];
   uint32_t m2 = 0;
 #pragma unroll
@@ -241,10 +165,15 @@ quant_tile_kernel(QuantArgs a) {
     reinterpret_cast<uint4*>(qc)[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
     reinterpret_cast<uint4*>(qc + R)[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
     reinterpret_cast<uint4*>(qc + R)[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
-    const int64_t kb = gr / 32;
-    uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
-    sc[a.sf_mma ? sf_mma_offset(gc, kb, KBc) : gc * KBc + kb] = static_cast<uint8_t>(sb0);
-    sc[a.sf_mma ? sf_mma_offset(gc + 1, kb, KBc) : (gc + 1) * KBc + kb] = static_cast<uint8_t>(sb1);
+    if (a.sf_mma) {
+      satom_col[sf_mma_offset(2 * p, rb, 4)] = static_cast<uint8_t>(sb0);
+      satom_col[sf_mma_offset(2 * p + 1, rb, 4)] = static_cast<uint8_t>(sb1);
+    } else {
+      const int64_t kb = gr / 32;
+      uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
+      sc[gc * KBc + kb] = static_cast<uint8_t>(sb0);
+      sc[(gc + 1) * KBc + kb] = static_cast<uint8_t>(sb1);
+    }
   } else {
     uint32_t c0[16], c1[16];
 #pragma unroll
@@ -257,6 +186,115 @@ quant_tile_kernel(QuantArgs a) {
     for (int i = 0; i < 4; ++i) {
       reinterpret_cast<uint4*>(oc)[i] = make_uint4(c0[4 * i], c0[4 * i + 1], c0[4 * i + 2], c0[4 * i + 3]);
       reinterpret_cast<uint4*>(oc + R)[i] = make_uint4(c1[4 * i], c1[4 * i + 1], c1[4 * i + 2], c1[4 * i + 3]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+quant_tile_kernel(QuantArgs a) {
+  __shared__ __align__(16) uint32_t tile[QT_ROWS * QT_PITCH / 2];  // bf16 pairs
+  // In the tensor-core scale layout a 128 x 128 tile's row-wise scales and its column-wise scales
+  // are each exactly one 512-byte scale tile: they are assembled here and stored with one write
+  // each (single-byte scale stores scattered over the scale matrix cost more than the codes).
+  __shared__ __align__(16) uint8_t satom_row[512], satom_col[512];
+  const int tid = threadIdx.x;
+  // column tiles vary fastest so that CTAs running together read whole contiguous rows
+  const int64_t row0 = static_cast<int64_t>(blockIdx.y) * QT_ROWS;
+  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * QT_COLS;
+  const int b = blockIdx.z;
+  const int64_t R = a.rows, C = a.cols, KBr = C / 32, KBc = R / 32;
+  const bool sf_atoms = a.mx && a.sf_mma;
+
+  const bf16* src = a.src_ptrs.p[0] ? static_cast<const bf16*>(a.src_ptrs.p[b])
+                                    : static_cast<const bf16*>(a.src) + static_cast<int64_t>(b) * a.src_batch_stride;
+
+  // ---- load 128 x 128: 8 chunks of 8 bf16 per thread, all issued before any use
+  const int cchunk = tid & 15;
+  const int64_t col = col0 + cchunk * 8;
+  const bool col_ok = col < C;
+  uint4 v[QT_LOADS];
+#pragma unroll
+  for (int i = 0; i < QT_LOADS; ++i) {
+    const int64_t r = row0 + (tid >> 4) + 16 * i;
+    v[i] = make_uint4(0, 0, 0, 0);
+    if (r < R && col_ok) {
+      int64_t sr = r;
+      bool zero = false;
+      if (a.sorted_to_src) {
+        const int32_t s = a.sorted_to_src[r];
+        zero = s < 0;
+        sr = zero ? 0 : static_cast<int64_t>(s / a.k);
+      }
+      if (!zero) v[i] = __ldg(reinterpret_cast<const uint4*>(src + sr * a.src_ld + col));
+    }
+  }
+  // destination rows: identity, or the gate/up interleaving (128 rows from each half per 256-row group)
+  auto dst_row = [&](int64_t r) -> int64_t {
+    if (!a.gate_up_half) return r;
+    const int64_t hf = a.gate_up_half;
+    return r < hf ? (r / 128) * 256 + (r % 128) : ((r - hf) / 128) * 256 + 128 + ((r - hf) % 128);
+  };
+  // ---- row-wise outputs (and the smem copy for the column pass)
+  uint8_t* qbase = a.q_row + static_cast<int64_t>(b) * R * C + col;
+  uint8_t* sbase = a.s_row + static_cast<int64_t>(b) * R * KBr;
+  bf16* obase = a.o_row + static_cast<int64_t>(b) * R * C + col;
+#pragma unroll
+  for (int i = 0; i < QT_LOADS; ++i) {
+    const int lr = (tid >> 4) + 16 * i;
+    const int64_t r = row0 + lr;
+    const bool valid = r < R && col_ok;
+    const int64_t dr = dst_row(r);
+    if (a.do_col) *reinterpret_cast<uint4*>(&tile[lr * (QT_PITCH / 2) + cchunk * 4]) = v[i];
+    if (!a.do_row) continue;
+    if (a.mx) {
+      uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w)));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      const uint32_t sb = e8m0_from_amax_bits(m);
+      const float inv = e8m0_inv_scale(sb);
+      if (valid) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        uint32_t q[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
+        *reinterpret_cast<uint2*>(qbase + dr * C) = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+        if ((cchunk & 3) == 0) {
+          const int64_t kb = col / 32;
+          if (sf_atoms)
+            satom_row[sf_mma_offset(lr, kb & 3, 4)] = static_cast<uint8_t>(sb);
+          else
+            sbase[dr * KBr + kb] = static_cast<uint8_t>(sb);
+        }
+      }
+    } else if (valid) {
+      *reinterpret_cast<uint4*>(obase + dr * C) = v[i];
+    }
+  }
+
+  // ---- column-wise: thread -> columns (2p, 2p+1) of the tile, 32-row block rb
+  if (a.do_col) {
+    __syncthreads();
+    const int p = tid & 63;
+    const int rb = tid >> 6;
+    const int64_t gc = col0 + 2 * p;
+    const int64_t gr = row0 + rb * 32;
+    if (gc < C && gr < R) column_pass(a, tile, p, rb, gc, gr, b, satom_col);
+  }
+
+  // ---- one 512-byte store per scale tile (this layout needs rows and columns in multiples of 128)
+  if (sf_atoms) {
+    __syncthreads();
+    if (tid < 32) {
+      if (a.do_row)
+        reinterpret_cast<uint4*>(sbase + ((dst_row(row0) / 128) * (KBr / 4) + col0 / 128) * 512)[tid] =
+            reinterpret_cast<const uint4*>(satom_row)[tid];
+    } else if (tid < 64) {
+      if (a.do_col) {
+        uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
+        reinterpret_cast<uint4*>(sc + ((col0 / 128) * (KBc / 4) + row0 / 128) * 512)[tid - 32] =
+            reinterpret_cast<const uint4*>(satom_col)[tid - 32];
+      }
     }
   }
 }

@@ -36,7 +36,7 @@ constexpr uint32_t TMEM_COLS = 512;
 // Tile shape and thread layout of one kernel instance.
 //   EPI_WARPS epilogue warps (a multiple of 4: each TMEM lane quadrant gets EPI_WARPS/4 warps that
 //   split the tile's columns); PASS columns per pass of the column-wise transpose buffer.
-template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_>
+template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_, bool HTILE_ = false>
 struct Shape {
   static constexpr int BN = BN_;
   static constexpr int NBUF = NBUF_;
@@ -55,14 +55,18 @@ struct Shape {
   static constexpr int SF_COLS = 4 + 4 * (BN / 128);
   static constexpr uint32_t SF_TMEM_COL = NBUF * BN;
   static constexpr int STAGING_PER_WARP = STAGING_ ? (32 * PITCH * 4 + 15) / 16 * 16 : 0;
-  static constexpr int SMEM_DYN = STAGES * STAGE_BYTES + EPI_WARPS * STAGING_PER_WARP + 1024;
+  static constexpr bool HTILE = HTILE_;  // dSwiGLU: the tile's saved gate/up values staged in smem by TMA
+  static constexpr int H_BYTES = HTILE ? BM * 2 * BN * 2 : 0;
+  static constexpr int OFF_H = STAGES * STAGE_BYTES;
+  static constexpr int OFF_STAGING = OFF_H + H_BYTES;
+  static constexpr int SMEM_DYN = OFF_STAGING + EPI_WARPS * STAGING_PER_WARP + 1024;
   static_assert(NBUF * BN + STAGES * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
   static_assert(SMEM_DYN + 4096 <= 232448, "shared memory budget");
   static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0, "thread layout");
 };
 using ShapeStore = Shape<256, 1, 4, false, 8, 16>;    // plain bf16-store epilogues
 using ShapeSwiglu = Shape<256, 1, 4, true, 16, 8>;    // gate_up + ScaledSwiGLU: one 32-column group per thread
-using ShapeDswiglu = Shape<128, 2, 6, true, 8, 16>;   // dgrad of down + dSwiGLU: epilogue overlaps the next tile
+using ShapeDswiglu = Shape<128, 2, 4, true, 8, 16, true>;  // dgrad of down + dSwiGLU: epilogue overlaps the next tile
 
 struct SharedState {
   uint64_t full[8];
@@ -70,6 +74,8 @@ struct SharedState {
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
+  uint64_t h_full;
+  uint64_t h_empty;
   uint32_t tmem_base;
   int abort_flag;
   int total_tiles;
@@ -236,7 +242,8 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
   __shared__ SharedState s;
   extern __shared__ uint8_t dyn_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
-  float* staging_base = reinterpret_cast<float*>(smem + S::STAGES * S::STAGE_BYTES);
+  float* staging_base = reinterpret_cast<float*>(smem + S::OFF_STAGING);
+  uint8_t* hbuf = smem + S::OFF_H;
   constexpr int BN = S::BN;
 
   const int warp = threadIdx.x >> 5;
@@ -264,11 +271,14 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       ptx::mbar_init(&s.acc_empty[i], S::EPI_WARPS);
     }
     ptx::mbar_init(&s.drain, 1);
+    ptx::mbar_init(&s.h_full, 1);
+    ptx::mbar_init(&s.h_empty, S::EPI_WARPS);
     ptx::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&g.tmap_a);
     ptx::prefetch_tmap(&g.tmap_b);
+    if (S::HTILE) ptx::prefetch_tmap(&g.tmap_h);
   }
   if (warp == 2) {
     ptx::tmem_alloc(&s.tmem_base, TMEM_COLS);
@@ -287,6 +297,8 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, last_parity = 0;
+    uint32_t h_count = 0;
+    bool h_issued = false;
     const uint32_t tx = S::A_BYTES + S::B_BYTES + (MX ? 512 + S::SFB_BYTES : 0);
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
       Tile tl;
@@ -332,6 +344,25 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           phase ^= 1;
         }
       }
+      if (S::HTILE && !*abort_flag) {
+        // the tile's saved gate/up columns, once the epilogue has finished with the previous tile's
+        if (!ptx::mbar_wait(&s.h_empty, (h_count & 1) ^ 1, abort_flag, lim)) break;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        ptx::mbar_arrive_expect_tx(&s.h_full, S::H_BYTES);
+        const int32_t hr = tl.a_row, gc = tl.nb * BN;
+#pragma unroll
+        for (int i = 0; i < BN / 64; ++i) {
+          ptx::tma_load_2d(hbuf + i * 16384, &g.tmap_h, gc + 64 * i, hr, &s.h_full);
+          ptx::tma_load_2d(hbuf + (BN / 64 + i) * 16384, &g.tmap_h, static_cast<int32_t>(g.epi.f) + gc + 64 * i, hr,
+                           &s.h_full);
+        }
+        h_issued = true;
+        ++h_count;
+      }
+    }
+    if (S::HTILE && h_issued) {  // the last h tile must have landed before the CTA exits
+      volatile int never = 0;
+      ptx::mbar_wait(&s.h_full, (h_count - 1) & 1, &never, lim);
     }
     // wait for the loads still in flight (only possible after an abort)
     for (int i = 0; i < S::STAGES; ++i)
@@ -503,13 +534,35 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         const int64_t f = ep.f, f2 = 2 * ep.f;
         const int64_t j0 = static_cast<int64_t>(tl.nb) * BN + CPT * ch;
         const bf16* hrow = ep.h + row * f2;
+        // saved gate/up values: 16-byte chunk c (of this thread's 32-column group cc) of the gate part
+        // and of the up part, from the TMA-staged tile in smem (128B-swizzled rows) or from global
+        const int rl = 32 * q + lane;  // row within the tile
+        auto h_chunk = [&](int up, int cc, int c) -> uint4 {
+          if (S::HTILE) {
+            const int col = CPT * ch + 32 * cc + 8 * c;  // column within the tile's gate (or up) part
+            const uint8_t* box = hbuf + (up * (BN / 64) + col / 64) * 16384;
+            const int chunk = ((col % 64) / 8) ^ (rl & 7);
+            return *reinterpret_cast<const uint4*>(box + rl * 128 + chunk * 16);
+          }
+          return reinterpret_cast<const uint4*>(hrow + (up ? f : 0) + j0 + 32 * cc)[c];
+        };
         uint4 hg[4], hu[4];
+        if (!S::HTILE) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // saved gate/up values of the first group, before the wait
-          hg[i] = reinterpret_cast<const uint4*>(hrow + j0)[i];
-          hu[i] = reinterpret_cast<const uint4*>(hrow + f + j0)[i];
+          for (int i = 0; i < 4; ++i) {  // saved gate/up values of the first group, before the wait
+            hg[i] = h_chunk(0, 0, i);
+            hu[i] = h_chunk(1, 0, i);
+          }
         }
         if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
+        if (S::HTILE) {
+          if (!ptx::mbar_wait(&s.h_full, static_cast<uint32_t>((local - 1) & 1), abort_flag, lim)) break;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            hg[i] = h_chunk(0, 0, i);
+            hu[i] = h_chunk(1, 0, i);
+          }
+        }
         ptx::tc_fence_after();
         const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
         float dp = 0.f;
@@ -542,9 +595,12 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           if (cc < G - 1) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {  // next group's saved values
-              hg[i] = reinterpret_cast<const uint4*>(hrow + j + 32)[i];
-              hu[i] = reinterpret_cast<const uint4*>(hrow + f + j + 32)[i];
+              hg[i] = h_chunk(0, cc + 1, i);
+              hu[i] = h_chunk(1, cc + 1, i);
             }
+          } else if (S::HTILE) {  // done with the staged h tile: the producer may refill it
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&s.h_empty);
           }
           if (ep.dump) {
             float4* d0 = reinterpret_cast<float4*>(ep.dump + row * f2 + j);

@@ -35,6 +35,7 @@ struct EpiArgs {
 struct GemmArgs {
   CUtensorMap tmap_a;  // A: 2-D [rows, K] K-contiguous, box 128 rows x 128 bytes, 128B swizzle
   CUtensorMap tmap_b;  // B: 3-D [E, rows, K] (M-grouped) or 2-D [rows, K] (K-grouped)
+  CUtensorMap tmap_h;  // dSwiGLU: saved h [cap, 2f] bf16, box 128 rows x 64 columns, 128B swizzle
   int kgrouped;        // 0: M grouped by expert (rows of A = expert segments); 1: K grouped (wgrad)
   int E;
   int K;               // M-grouped reduction length
