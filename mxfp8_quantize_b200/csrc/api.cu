@@ -65,6 +65,34 @@ bool map_3d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// MXFP8 with the tensor-core scale layout: code tiles are written by TMA tensor stores (uint8 maps
+// over [batch*rows, cols] and [batch*cols, rows], 128 x 128 boxes, 128-byte swizzle).
+bool quant_store_maps(QuantArgs& a, int batch) {
+  a.tma_store = 0;
+  if (!a.mx || !a.sf_mma) return true;
+  const uint64_t R = a.rows, C = a.cols, B = batch;
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t es[2] = {1, 1};
+  if (a.do_row) {
+    cuuint64_t dims[2] = {C, B * R};
+    cuuint64_t strides[1] = {C};
+    if (g_encode(&a.tmap_qrow, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q_row, dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  if (a.do_col) {
+    cuuint64_t dims[2] = {R, B * C};
+    cuuint64_t strides[1] = {R};
+    if (g_encode(&a.tmap_qcol, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, a.q_colT, dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  a.tma_store = 1;
+  return true;
+}
+
 // Bump allocator over a caller buffer (1 KiB granules); with base == nullptr it only measures.
 struct Carve {
   uint8_t* base;
@@ -364,6 +392,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
   a.s_row = s_row;
   a.q_colT = q_colT;
   a.s_colT = s_colT;
+  if (!quant_store_maps(a, static_cast<int>(batch))) return MOE_ERR_CUDA;
   MOE_LAUNCH(ctx, "mxfp8_quantize", stream, launch_quant(a, static_cast<int>(batch), ctx->num_sms, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
@@ -405,6 +434,7 @@ moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, 
     a.mx = 0;
     a.do_row = 1;
     a.o_row = static_cast<bf16*>(x_perm);
+    if (!quant_store_maps(a, static_cast<int>(1))) return MOE_ERR_CUDA;
     MOE_LAUNCH(ctx, "permute_x", st, launch_quant(a, 1, ctx->num_sms, st));
   }
   return MOE_OK;
@@ -508,6 +538,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     a.q_colT = s.w1c_q;
     a.s_colT = s.w1c_s;
     a.gate_up_half = f;  // row-wise copy in 256-row groups of 128 gate + 128 up rows (one B tile each)
+    if (!quant_store_maps(a, static_cast<int>(E))) return MOE_ERR_CUDA;
     MOE_LAUNCH(ctx, "quantize_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
     a.gate_up_half = 0;
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
@@ -518,6 +549,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     a.s_row = w.w2_s;
     a.q_colT = s.w2c_q;
     a.s_colT = s.w2c_s;
+    if (!quant_store_maps(a, static_cast<int>(E))) return MOE_ERR_CUDA;
     MOE_LAUNCH(ctx, "quantize_w_down", st, launch_quant(a, E, ctx->num_sms, st));
     w1_base = w.w1_q;
     w1_stride = 2 * f * d;
@@ -540,6 +572,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.do_col = training;
     xa.q_colT = s.xT_q;
     xa.s_colT = s.xT_s;
+    if (!quant_store_maps(xa, static_cast<int>(1))) return MOE_ERR_CUDA;
     MOE_LAUNCH(ctx, "permute_quantize_x", st, launch_quant(xa, 1, ctx->num_sms, st));
   } else {
     w1_stride = uniform_stride(w_gate_up, E, 2 * f * d * 2);
@@ -555,7 +588,8 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       a.rows = 2 * f;
       a.cols = d;
       a.o_row = w.w1_copy;
-      MOE_LAUNCH(ctx, "gather_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
+      if (!quant_store_maps(a, static_cast<int>(E))) return MOE_ERR_CUDA;
+    MOE_LAUNCH(ctx, "gather_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
       w1_base = w.w1_copy;
       w1_stride = 2 * f * d * 2;
     }
@@ -565,7 +599,8 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       a.rows = d;
       a.cols = f;
       a.o_row = w.w2_copy;
-      MOE_LAUNCH(ctx, "gather_w_down", st, launch_quant(a, E, ctx->num_sms, st));
+      if (!quant_store_maps(a, static_cast<int>(E))) return MOE_ERR_CUDA;
+    MOE_LAUNCH(ctx, "gather_w_down", st, launch_quant(a, E, ctx->num_sms, st));
       w2_base = w.w2_copy;
       w2_stride = d * f * 2;
     }
@@ -581,6 +616,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.o_row = w.x_perm;
     xa.do_col = training;
     xa.o_colT = s.xT;
+    if (!quant_store_maps(xa, static_cast<int>(1))) return MOE_ERR_CUDA;
     MOE_LAUNCH(ctx, "permute_x", st, launch_quant(xa, 1, ctx->num_sms, st));
   }
 
@@ -697,6 +733,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
       a.o_row = w.dy_perm;
       a.o_colT = w.dyT;
     }
+    if (!quant_store_maps(a, static_cast<int>(1))) return MOE_ERR_CUDA;
     MOE_LAUNCH(ctx, "gather_quantize_dy", st, launch_quant(a, 1, ctx->num_sms, st));
   }
   const void* w1c;  // B of dgrad of gate_up: [E, d, 2f]
@@ -713,12 +750,14 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     a.rows = 2 * f;
     a.cols = d;
     a.o_colT = w.w1T;
+    if (!quant_store_maps(a, static_cast<int>(E))) return MOE_ERR_CUDA;
     MOE_LAUNCH(ctx, "transpose_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_down[e];
     a.src_ld = f;
     a.rows = d;
     a.cols = f;
     a.o_colT = w.w2T;
+    if (!quant_store_maps(a, static_cast<int>(E))) return MOE_ERR_CUDA;
     MOE_LAUNCH(ctx, "transpose_w_down", st, launch_quant(a, E, ctx->num_sms, st));
     w1c = w.w1T;
     w2c = w.w2T;

@@ -135,7 +135,7 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 // word holds one row of both columns).  Scales go to the block's 512-byte scale tile in smem when
 // the tensor-core layout is requested, else straight to the row-major scale matrix.
 __device__ __forceinline__ void column_pass(const QuantArgs& a, const uint32_t* tile, int p, int rb, int64_t gc,
-                                            int64_t gr, int b, uint8_t* satom_col) {
+                                            int64_t gr, int b, uint8_t* satom_col, uint8_t* qcol_tile) {
   const int64_t R = a.rows, C = a.cols, KBc = R / 32;
   uint32_t wv[32];
   uint32_t m2 = 0;
@@ -160,11 +160,22 @@ __device__ __forceinline__ void column_pass(const QuantArgs& a, const uint32_t* 
       q0[i] = lo0 | (hi0 << 16);
       q1[i] = lo1 | (hi1 << 16);
     }
-    uint8_t* qc = a.q_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
-    reinterpret_cast<uint4*>(qc)[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
-    reinterpret_cast<uint4*>(qc)[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
-    reinterpret_cast<uint4*>(qc + R)[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
-    reinterpret_cast<uint4*>(qc + R)[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+    if (a.tma_store) {  // transposed code tile: 128-byte row per column, 32-byte run per row block
+      uint8_t* ct = qcol_tile;
+      const int r0 = 2 * p, r1 = 2 * p + 1;
+      uint8_t* row0p = ct + r0 * 128;
+      uint8_t* row1p = ct + r1 * 128;
+      *reinterpret_cast<uint4*>(row0p + (((2 * rb) ^ (r0 & 7)) << 4)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+      *reinterpret_cast<uint4*>(row0p + (((2 * rb + 1) ^ (r0 & 7)) << 4)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+      *reinterpret_cast<uint4*>(row1p + (((2 * rb) ^ (r1 & 7)) << 4)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+      *reinterpret_cast<uint4*>(row1p + (((2 * rb + 1) ^ (r1 & 7)) << 4)) = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+    } else {
+      uint8_t* qc = a.q_colT + (static_cast<int64_t>(b) * C + gc) * R + gr;
+      reinterpret_cast<uint4*>(qc)[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+      reinterpret_cast<uint4*>(qc)[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+      reinterpret_cast<uint4*>(qc + R)[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+      reinterpret_cast<uint4*>(qc + R)[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+    }
     if (a.sf_mma) {
       satom_col[sf_mma_offset(2 * p, rb, 4)] = static_cast<uint8_t>(sb0);
       satom_col[sf_mma_offset(2 * p + 1, rb, 4)] = static_cast<uint8_t>(sb1);
@@ -191,8 +202,11 @@ __device__ __forceinline__ void column_pass(const QuantArgs& a, const uint32_t* 
 }
 
 __global__ void __launch_bounds__(256)
-quant_tile_kernel(QuantArgs a) {
+quant_tile_kernel(const __grid_constant__ QuantArgs a) {
   __shared__ __align__(16) uint32_t tile[QT_ROWS * QT_PITCH / 2];  // bf16 pairs
+  // code tiles for the TMA stores (128B-swizzled rows of 128 bytes)
+  extern __shared__ uint8_t qdyn_raw[];
+  uint8_t* qdyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qdyn_raw) + 1023) & ~uintptr_t(1023));
   // In the tensor-core scale layout a 128 x 128 tile's row-wise scales and its column-wise scales
   // are each exactly one 512-byte scale tile: they are assembled here and stored with one write
   // each (single-byte scale stores scattered over the scale matrix cost more than the codes).
@@ -258,7 +272,13 @@ quant_tile_kernel(QuantArgs a) {
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
-        *reinterpret_cast<uint2*>(qbase + dr * C) = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+        const uint2 qq = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+        if (a.tma_store) {  // row lr, bytes 8*cchunk.. of the swizzled 128-byte row
+          uint8_t* rowp = qdyn + lr * 128;
+          *reinterpret_cast<uint2*>(rowp + (((cchunk >> 1) ^ (lr & 7)) << 4) + ((cchunk & 1) << 3)) = qq;
+        } else {
+          *reinterpret_cast<uint2*>(qbase + dr * C) = qq;
+        }
         if ((cchunk & 3) == 0) {
           const int64_t kb = col / 32;
           if (sf_atoms)
@@ -279,12 +299,32 @@ quant_tile_kernel(QuantArgs a) {
     const int rb = tid >> 6;
     const int64_t gc = col0 + 2 * p;
     const int64_t gr = row0 + rb * 32;
-    if (gc < C && gr < R) column_pass(a, tile, p, rb, gc, gr, b, satom_col);
+    if (gc < C && gr < R) column_pass(a, tile, p, rb, gc, gr, b, satom_col, qdyn + 16384);
   }
 
-  // ---- one 512-byte store per scale tile (this layout needs rows and columns in multiples of 128)
-  if (sf_atoms) {
+  // ---- code tiles through TMA tensor stores; scales as one 512-byte store per scale tile (this
+  //      layout needs rows and columns in multiples of 128)
+  if (a.tma_store) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // smem writes -> visible to the copy engine
     __syncthreads();
+    if (tid == 0) {
+      if (a.do_row)
+        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                         reinterpret_cast<uint64_t>(&a.tmap_qrow)),
+                     "r"(static_cast<int32_t>(col0)), "r"(static_cast<int32_t>(b * R + dst_row(row0))),
+                     "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qdyn)))
+                     : "memory");
+      if (a.do_col)
+        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                         reinterpret_cast<uint64_t>(&a.tmap_qcol)),
+                     "r"(static_cast<int32_t>(row0)), "r"(static_cast<int32_t>(b * C + col0)),
+                     "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qdyn + 16384)))
+                     : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+  }
+  if (sf_atoms) {
+    if (!a.tma_store) __syncthreads();
     if (tid < 32) {
       if (a.do_row)
         reinterpret_cast<uint4*>(sbase + ((dst_row(row0) / 128) * (KBr / 4) + col0 / 128) * 512)[tid] =
@@ -297,6 +337,7 @@ quant_tile_kernel(QuantArgs a) {
       }
     }
   }
+  if (a.tma_store && tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // ------------------------------------------------------------------------------------------
@@ -384,7 +425,12 @@ cudaError_t launch_quant(const QuantArgs& a, int batch, int /*num_sms*/, cudaStr
   if (a.rows == 0 || a.cols == 0 || batch == 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(ceil_div(a.cols, QT_COLS)), static_cast<unsigned>(ceil_div(a.rows, QT_ROWS)),
             static_cast<unsigned>(batch));
-  quant_tile_kernel<<<grid, 256, 0, st>>>(a);
+  const int dyn = a.tma_store ? 32768 + 1024 : 0;
+  if (dyn) {
+    cudaError_t e = cudaFuncSetAttribute(quant_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    if (e != cudaSuccess) return e;
+  }
+  quant_tile_kernel<<<grid, 256, dyn, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,7 @@
 // Declarations of the HBM-bound kernels' launchers (codec.cu).
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace moemx {
@@ -26,6 +28,11 @@ struct QuantArgs {
   uint8_t* s_colT;
   bf16* o_row;
   bf16* o_colT;
+  // MXFP8 with the tensor-core scale layout: code tiles leave through TMA tensor stores
+  // (uint8 maps over [batch*rows, cols] and [batch*cols, rows], 128 x 128 boxes, 128B swizzle)
+  int tma_store;
+  CUtensorMap tmap_qrow;
+  CUtensorMap tmap_qcol;
 };
 
 cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk, int E, int capacity,
