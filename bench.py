@@ -23,6 +23,7 @@ import json
 import os
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -85,8 +86,8 @@ REASON_FIELDS = ["clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_th
 
 
 class ClockSampler:
-    def __init__(self, gpu_index: int):
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+    def __init__(self, gpu_index: int, out_dir: str):
+        self.path = os.path.join(out_dir, f"clocks_gpu{gpu_index}.csv")
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
         q = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," + ",".join(REASON_FIELDS)
         try:
@@ -232,7 +233,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         ev.record(stream)
         records.append((name, after, ev))
 
-    clocks = ClockSampler(local_rank if world > 1 else (torch.cuda.current_device()))
+    clocks = ClockSampler(local_rank if world > 1 else (torch.cuda.current_device()), args.clocks_dir)
     barrier()
     torch.cuda.synchronize(dev)
     moe.set_launch_hook(local_rank, hook)
@@ -356,6 +357,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling cases)")
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling cases)")
+    ap.add_argument("--clocks-dir", default=tempfile.gettempdir(), help="where the nvidia-smi clock samples go")
     args = ap.parse_args()
     cfg = workloads.CONFIGS[args.config]
     if args.tokens or args.experts:
