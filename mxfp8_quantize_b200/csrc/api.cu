@@ -65,6 +65,24 @@ bool map_3d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A scale buffer in the tensor-core tile layout (512-byte tiles, [rows/128][kb4]) as a 3-D u32
+// array [rows/128][kb4][128]; a box is ``box_tiles`` tiles of consecutive 128-row blocks at one kb4.
+bool map_sf(CUtensorMap* m, const void* base, uint64_t rows, int64_t kb4, uint32_t box_tiles) {
+  cuuint64_t dims[3] = {128, static_cast<uint64_t>(kb4), rows / 128};
+  cuuint64_t strides[2] = {512, static_cast<uint64_t>(kb4) * 512};
+  cuuint32_t box[3] = {128, 1, box_tiles};
+  cuuint32_t es[3] = {1, 1, 1};
+  return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// Scale maps of a GEMM's A (``a_rows`` rows) and B (``b_rows`` rows over all experts) operands, for
+// the kernel whose tiles are ``bn`` wide.
+bool sf_maps(GemmArgs& g, uint64_t a_rows, uint64_t b_rows, int bn) {
+  return map_sf(&g.tmap_sfa, g.sfa, a_rows, g.sfa_kb4, 1) &&
+         map_sf(&g.tmap_sfb, g.sfb, b_rows, g.sfb_kb4, static_cast<uint32_t>(bn / 128));
+}
+
 // MXFP8 with the tensor-core scale layout: code tiles are written by TMA tensor stores (uint8 maps
 // over [batch*rows, cols] and [batch*cols, rows], 128 x 128 boxes, 128-byte swizzle).
 bool quant_store_maps(QuantArgs& a, int batch) {
@@ -640,6 +658,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     g.sfb = w.w1_s;
     g.sfb_kb4 = d / 128;
     g.sfb_expert_rows = 2 * f;
+    if (D.mx && !sf_maps(g, D.cap, E * 2 * f, gemm_tile_n(EPI_SWIGLU))) return MOE_ERR_CUDA;
     EpiArgs& ep = g.epi;
     ep.f = f;
     ep.cap = D.cap;
@@ -674,6 +693,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     g.sfb = w.w2_s;
     g.sfb_kb4 = f / 128;
     g.sfb_expert_rows = d;
+    if (D.mx && !sf_maps(g, D.cap, E * d, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
     g.epi.out = w.y_perm;
     g.epi.ldo = d;
     MOE_LAUNCH(ctx, "gemm_down", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
@@ -780,6 +800,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     g.sfb = s.w2c_s;
     g.sfb_kb4 = d / 128;
     g.sfb_expert_rows = f;
+    if (D.mx && !sf_maps(g, D.cap, E * f, gemm_tile_n(EPI_DSWIGLU))) return MOE_ERR_CUDA;
     EpiArgs& ep = g.epi;
     ep.f = f;
     ep.cap = D.cap;
@@ -814,6 +835,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     g.sfa_kb4 = D.cap / 128;
     g.sfb = s.aT_s;
     g.sfb_kb4 = D.cap / 128;
+    if (D.mx && !sf_maps(g, d, f, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
     g.epi.ldo = f;
     for (int e = 0; e < E; ++e) g.epi.out_ptrs.p[e] = dw_down[e];
     MOE_LAUNCH(ctx, "gemm_wgrad_down", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
@@ -835,6 +857,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     g.sfb = s.w1c_s;
     g.sfb_kb4 = 2 * f / 128;
     g.sfb_expert_rows = d;
+    if (D.mx && !sf_maps(g, D.cap, E * d, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
     g.epi.out = w.dx_perm;
     g.epi.ldo = d;
     MOE_LAUNCH(ctx, "gemm_dgrad_gate_up", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
@@ -855,6 +878,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     g.sfa_kb4 = D.cap / 128;
     g.sfb = s.xT_s;
     g.sfb_kb4 = D.cap / 128;
+    if (D.mx && !sf_maps(g, 2 * f, d, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
     g.epi.ldo = d;
     for (int e = 0; e < E; ++e) g.epi.out_ptrs.p[e] = dw_gate_up[e];
     MOE_LAUNCH(ctx, "gemm_wgrad_gate_up", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));

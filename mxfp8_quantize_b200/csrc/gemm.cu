@@ -278,6 +278,10 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&g.tmap_a);
     ptx::prefetch_tmap(&g.tmap_b);
+    if (MX) {
+      ptx::prefetch_tmap(&g.tmap_sfa);
+      ptx::prefetch_tmap(&g.tmap_sfb);
+    }
     if (S::HTILE) ptx::prefetch_tmap(&g.tmap_h);
   }
   if (warp == 2) {
@@ -325,17 +329,12 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
               ptx::tma_load_2d(st + S::OFF_B + i * 16384, &g.tmap_b, kx, brow, &s.full[stage]);
           }
         }
-        if (MX) {
-          const int64_t kq = kx / 128;
-          const uint8_t* sa = g.sfa + ((static_cast<int64_t>(tl.a_row) / 128) * g.sfa_kb4 + kq) * 512;
-          ptx::bulk_load(st + S::OFF_SFA, sa, 512, &s.full[stage]);
+        if (MX) {  // this step's scale tiles: one of A, BN/128 consecutive ones of B
+          const int32_t kq = kx / 128;
           const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * g.sfb_expert_rows;
-#pragma unroll
-          for (int i = 0; i < BN / 128; ++i) {
-            const int64_t brow = eb + static_cast<int64_t>(tl.nb) * BN + i * 128;
-            ptx::bulk_load(st + S::OFF_SFB + i * 512, g.sfb + ((brow / 128) * g.sfb_kb4 + kq) * 512, 512,
-                           &s.full[stage]);
-          }
+          tma_load_3d(st + S::OFF_SFA, &g.tmap_sfa, 0, kq, tl.a_row / 128, &s.full[stage]);
+          tma_load_3d(st + S::OFF_SFB, &g.tmap_sfb, 0, kq,
+                      static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128), &s.full[stage]);
         }
         issued_mask |= 1u << stage;
         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
