@@ -39,12 +39,13 @@ bool encoder() {
   return g_encode != nullptr;
 }
 
-// 2-D map over [rows, inner] (inner contiguous), box 128 rows x 128 bytes, 128-byte swizzle.
-bool map_2d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t rows, uint64_t row_bytes) {
+// 2-D map over [rows, inner] (inner contiguous), box ``box_rows`` rows x 128 bytes, 128-byte swizzle.
+bool map_2d(CUtensorMap* m, const void* base, bool fp8, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+            uint32_t box_rows = 128) {
   const CUtensorMapDataType dt = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {fp8 ? 128u : 64u, 128u};
+  cuuint32_t box[2] = {fp8 ? 128u : 64u, box_rows};
   cuuint32_t es[2] = {1, 1};
   return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -645,7 +646,8 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     // unpermuted weights as a 128-row gate box plus the matching 128-row up box.
     const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.x_q) : w.x_perm, D.mx, d, D.cap,
                            d * (D.mx ? 1 : 2)) &&
-                    map_3d(&g.tmap_b, w1_base, D.mx, d, 2 * f, E, d * (D.mx ? 1 : 2), w1_stride);
+                    map_3d(&g.tmap_b, w1_base, D.mx, d, 2 * f, E, d * (D.mx ? 1 : 2), w1_stride,
+                           D.mx ? gemm_tile_n(EPI_SWIGLU) : gemm_tile_n(EPI_SWIGLU) / 2);
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
@@ -681,7 +683,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     GemmArgs g = gemm_args(ctx);
     const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.a_q) : w.a, D.mx, f, D.cap,
                            f * (D.mx ? 1 : 2)) &&
-                    map_3d(&g.tmap_b, w2_base, D.mx, f, d, E, f * (D.mx ? 1 : 2), w2_stride);
+                    map_3d(&g.tmap_b, w2_base, D.mx, f, d, E, f * (D.mx ? 1 : 2), w2_stride, gemm_tile_n(EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
@@ -787,7 +789,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   {
     GemmArgs g = gemm_args(ctx);
     const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dy_q) : w.dy_perm, D.mx, d, D.cap, d * es) &&
-                    map_3d(&g.tmap_b, w2c, D.mx, d, f, E, d * es, f * d * es) &&
+                    map_3d(&g.tmap_b, w2c, D.mx, d, f, E, d * es, f * d * es, gemm_tile_n(EPI_DSWIGLU)) &&
                     map_2d(&g.tmap_h, s.h, false, 2 * f, D.cap, 2 * f * 2);  // bf16 boxes of 128 rows x 64 columns
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
@@ -824,7 +826,8 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     GemmArgs g = gemm_args(ctx);
     const bool ok =
         map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dyT_q) : w.dyT, D.mx, D.cap, d, D.cap * es) &&
-        map_2d(&g.tmap_b, D.mx ? static_cast<const void*>(s.aT_q) : s.aT, D.mx, D.cap, f, D.cap * es);
+        map_2d(&g.tmap_b, D.mx ? static_cast<const void*>(s.aT_q) : s.aT, D.mx, D.cap, f, D.cap * es,
+               gemm_tile_n(EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 1;
     g.E = E;
@@ -845,7 +848,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     GemmArgs g = gemm_args(ctx);
     const bool ok =
         map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dh_q) : w.dh, D.mx, 2 * f, D.cap, 2 * f * es) &&
-        map_3d(&g.tmap_b, w1c, D.mx, 2 * f, d, E, 2 * f * es, 2 * f * d * es);
+        map_3d(&g.tmap_b, w1c, D.mx, 2 * f, d, E, 2 * f * es, 2 * f * d * es, gemm_tile_n(EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
@@ -867,7 +870,8 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     GemmArgs g = gemm_args(ctx);
     const bool ok =
         map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dhT_q) : w.dhT, D.mx, D.cap, 2 * f, D.cap * es) &&
-        map_2d(&g.tmap_b, D.mx ? static_cast<const void*>(s.xT_q) : s.xT, D.mx, D.cap, d, D.cap * es);
+        map_2d(&g.tmap_b, D.mx ? static_cast<const void*>(s.xT_q) : s.xT, D.mx, D.cap, d, D.cap * es,
+               gemm_tile_n(EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 1;
     g.E = E;

@@ -319,15 +319,10 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * (BN / 2), tl.e, &s.full[stage]);
           tma_load_3d(st + S::OFF_B + S::B_BYTES / 2, &g.tmap_b, kx, g.gate_up_half + tl.nb * (BN / 2), tl.e,
                       &s.full[stage]);
+        } else if (!g.kgrouped) {  // one box of BN rows
+          tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * BN, tl.e, &s.full[stage]);
         } else {
-#pragma unroll
-          for (int i = 0; i < BN / 128; ++i) {
-            const int brow = tl.nb * BN + i * 128;
-            if (!g.kgrouped)
-              tma_load_3d(st + S::OFF_B + i * 16384, &g.tmap_b, kx, brow, tl.e, &s.full[stage]);
-            else
-              ptx::tma_load_2d(st + S::OFF_B + i * 16384, &g.tmap_b, kx, brow, &s.full[stage]);
-          }
+          ptx::tma_load_2d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * BN, &s.full[stage]);
         }
         if (MX) {  // this step's scale tiles: one of A, BN/128 consecutive ones of B
           const int32_t kq = kx / 128;

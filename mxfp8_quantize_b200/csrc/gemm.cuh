@@ -34,7 +34,8 @@ struct EpiArgs {
 
 struct GemmArgs {
   CUtensorMap tmap_a;  // A: 2-D [rows, K] K-contiguous, box 128 rows x 128 bytes, 128B swizzle
-  CUtensorMap tmap_b;  // B: 3-D [E, rows, K] (M-grouped) or 2-D [rows, K] (K-grouped)
+  CUtensorMap tmap_b;  // B: 3-D [E, rows, K] (M-grouped) or 2-D [rows, K] (K-grouped); box BN rows (bf16
+                       // gate_up: BN/2, one box of gate rows and one of up rows)
   CUtensorMap tmap_h;  // dSwiGLU: saved h [cap, 2f] bf16, box 128 rows x 64 columns, 128B swizzle
   // MXFP8 scales of A and B in the tile layout, as 3-D u32 arrays [row tiles][kb4][128]: one box is
   // the 512-byte tile of one 128-K step for one (A) or BN/128 (B) consecutive 128-row blocks
