@@ -206,7 +206,8 @@ quant_tile_kernel(const __grid_constant__ QuantArgs a) {
   __shared__ __align__(16) uint32_t tile[QT_ROWS * QT_PITCH / 2];  // bf16 pairs
   // code tiles for the TMA stores (128B-swizzled rows of 128 bytes)
   extern __shared__ uint8_t qdyn_raw[];
-  uint8_t* qdyn = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qdyn_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, derived from the shared array (keeps the accesses in the shared state space)
+  uint8_t* qdyn = qdyn_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(qdyn_raw)) & 1023u)) & 1023u);
   // In the tensor-core scale layout a 128 x 128 tile's row-wise scales and its column-wise scales
   // are each exactly one 512-byte scale tile: they are assembled here and stored with one write
   // each (single-byte scale stores scattered over the scale matrix cost more than the codes).

@@ -241,7 +241,9 @@ template <bool MX, int EPI, class S>
 __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs g) {
   __shared__ SharedState s;
   extern __shared__ uint8_t dyn_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned start, derived from the shared array itself (not through an integer) so
+  // that the compiler keeps every access below in the shared state space
+  uint8_t* smem = dyn_raw + ((1024u - (ptx::smem_u32(dyn_raw) & 1023u)) & 1023u);
   float* staging_base = reinterpret_cast<float*>(smem + S::OFF_STAGING);
   uint8_t* hbuf = smem + S::OFF_H;
   constexpr int BN = S::BN;
