@@ -86,8 +86,31 @@ bool sf_maps(GemmArgs& g, uint64_t a_rows, uint64_t b_rows, int bn) {
 
 // MXFP8 with the tensor-core scale layout: code tiles are written by TMA tensor stores (uint8 maps
 // over [batch*rows, cols] and [batch*cols, rows], 128 x 128 boxes, 128-byte swizzle).
+int64_t uniform_stride(const void* const* p, int E, int64_t min_bytes);
+
+// TMA source map of a quantisation pass when the persistent kernel can take it: one uniformly
+// strided [batch, rows, cols] bf16 source with 16-byte aligned rows, rows and cols multiples of 128.
+void quant_load_map(QuantArgs& a, int batch) {
+  a.tma_load = 0;
+  if (a.sorted_to_src || a.rows % 128 || a.cols % 128 || !a.do_row || !a.do_col) return;
+  const void* base = a.src_ptrs.p[0] ? a.src_ptrs.p[0] : a.src;
+  const int64_t row_bytes = a.src_ld * 2, tile_bytes = a.rows * row_bytes;
+  int64_t stride = a.src_ptrs.p[0] ? uniform_stride(a.src_ptrs.p, batch, tile_bytes) : a.src_batch_stride * 2;
+  if (batch == 1) stride = tile_bytes;
+  if (!base || !aligned16(base) || (row_bytes & 15) || stride <= 0 || (stride & 15) || stride < tile_bytes) return;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(a.cols), static_cast<cuuint64_t>(a.rows), static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(stride)};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  if (g_encode(&a.tmap_src, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+    a.tma_load = 1;
+}
+
 bool quant_store_maps(QuantArgs& a, int batch) {
   a.tma_store = 0;
+  a.tma_load = 0;
   if (!a.mx || !a.sf_mma) return true;
   const uint64_t R = a.rows, C = a.cols, B = batch;
   cuuint32_t box[2] = {128, 128};
@@ -109,6 +132,7 @@ bool quant_store_maps(QuantArgs& a, int batch) {
       return false;
   }
   a.tma_store = 1;
+  quant_load_map(a, batch);
   return true;
 }
 
@@ -283,9 +307,10 @@ int64_t uniform_stride(const void* const* p, int E, int64_t min_bytes) {
   return s;
 }
 
-QuantArgs quant_args() {
+QuantArgs quant_args(moe_ctx_t ctx) {
   QuantArgs a;
   std::memset(&a, 0, sizeof(a));
+  a.status = ctx->d_status;
   return a;
 }
 
@@ -397,7 +422,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
     return MOE_ERR_UNSUPPORTED;
   if (!aligned16(x) || (row && !aligned16(q_row)) || (col && !aligned16(q_colT))) return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->device);
-  QuantArgs a = quant_args();
+  QuantArgs a = quant_args(ctx);
   a.src = static_cast<const bf16*>(x);
   a.src_batch_stride = rows * cols;
   a.src_ld = cols;
@@ -443,7 +468,7 @@ moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, 
   MOE_LAUNCH(ctx, "route", st, launch_route(topk_idx, topk_prob, static_cast<int>(T * k), E, static_cast<int>(cap), split_sizes_in,
                         split_sizes, poffsets, sorted_to_src, src_to_sorted, prob_perm, ctx->d_status, st));
   if (x) {
-    QuantArgs a = quant_args();
+    QuantArgs a = quant_args(ctx);
     a.src = static_cast<const bf16*>(x);
     a.src_ld = d;
     a.sorted_to_src = sorted_to_src;
@@ -543,7 +568,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
   if (D.mx) {
     // 16-bit masters -> MXFP8 every step: row-wise (K = d / f of the forward GEMMs) and, for the
     // backward, down the columns (K = 2f / d of the dgrad GEMMs), from one read of each weight.
-    QuantArgs a = quant_args();
+    QuantArgs a = quant_args(ctx);
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_gate_up[e];
     a.src_ld = d;
     a.rows = 2 * f;
@@ -576,7 +601,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     w2_stride = d * f;
 
     // x: gather by expert + row-wise MXFP8 (K = d) and, for wgrad, token-axis MXFP8 transposed
-    QuantArgs xa = quant_args();
+    QuantArgs xa = quant_args(ctx);
     xa.src = static_cast<const bf16*>(x);
     xa.src_ld = d;
     xa.sorted_to_src = s.s2src;
@@ -598,7 +623,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     w2_stride = uniform_stride(w_down, E, d * f * 2);
     w1_base = w_gate_up[0];
     w2_base = w_down[0];
-    QuantArgs a = quant_args();
+    QuantArgs a = quant_args(ctx);
     a.mx = 0;
     a.do_row = 1;
     if (!w1_stride) {  // experts not evenly spaced: gather into one [E, 2f, d] tensor
@@ -623,7 +648,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       w2_base = w.w2_copy;
       w2_stride = d * f * 2;
     }
-    QuantArgs xa = quant_args();
+    QuantArgs xa = quant_args(ctx);
     xa.src = static_cast<const bf16*>(x);
     xa.src_ld = d;
     xa.sorted_to_src = s.s2src;
@@ -735,7 +760,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
 
   // 1. dy gathered by expert: row-wise (K = d, dgrad of down) and token-axis transposed (wgrad of down)
   {
-    QuantArgs a = quant_args();
+    QuantArgs a = quant_args(ctx);
     a.src = static_cast<const bf16*>(dy);
     a.src_ld = d;
     a.sorted_to_src = s.s2src;
@@ -764,7 +789,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     w1c = s.w1c_q;
     w2c = s.w2c_q;
   } else {
-    QuantArgs a = quant_args();
+    QuantArgs a = quant_args(ctx);
     a.mx = 0;
     a.do_col = 1;
     for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_gate_up[e];

@@ -4,6 +4,7 @@
 #include <cuda_fp8.h>
 
 #include "codec.cuh"
+#include "ptx_sm100.cuh"
 
 namespace moemx {
 
@@ -342,6 +343,195 @@ quant_tile_kernel(const __grid_constant__ QuantArgs a) {
 }
 
 // ------------------------------------------------------------------------------------------
+// The same MXFP8 quantisation (tensor-core scale layout, row-wise and column-wise) for a uniformly
+// strided [batch, rows, cols] source whose rows and cols are multiples of 128, as a persistent
+// kernel: QW_CTAS_PER_SM CTAs per SM walk the 128 x 128 tiles (column tiles fastest); each source
+// tile arrives by a TMA tensor load into a QW_NIN-deep ring issued QW_NIN tiles ahead, and the
+// code tiles leave through TMA tensor stores, so the reads, math and writes of consecutive tiles
+// (and of the SM's other CTA) overlap.  Same arithmetic, bit for bit, as quant_tile_kernel.
+// ------------------------------------------------------------------------------------------
+namespace {
+constexpr int QW_NIN = 2;                           // source tiles in flight per CTA
+constexpr int QW_NOUT = 1;                          // code-tile buffers per CTA
+constexpr int QW_CTAS_PER_SM = 2;
+constexpr int QW_IN_BYTES = QT_ROWS * QT_COLS * 2;  // one bf16 source tile, rows of 256 bytes
+constexpr int QW_OUT_BYTES = 2 * QT_ROWS * QT_COLS;  // row-wise + column-wise code tiles
+constexpr int QW_SMEM = QW_NIN * QW_IN_BYTES + QW_NOUT * (QW_OUT_BYTES + 1024) + 1024;
+}  // namespace
+
+__global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const __grid_constant__ QuantArgs a, int tiles) {
+  extern __shared__ uint8_t qw_raw[];
+  uint8_t* sm = qw_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(qw_raw)) & 1023u)) & 1023u);
+  uint8_t* in_base = sm;                                   // QW_NIN source tiles
+  uint8_t* out_base = sm + QW_NIN * QW_IN_BYTES;           // QW_NOUT x [row codes 16 KB | column codes 16 KB]
+  uint8_t* atom_base = out_base + QW_NOUT * QW_OUT_BYTES;  // QW_NOUT x [row scale tile | column scale tile]
+  __shared__ uint64_t full[QW_NIN];
+  __shared__ int stop;
+  const int tid = threadIdx.x;
+  const int64_t R = a.rows, C = a.cols, KBr = C / 32, KBc = R / 32;
+  const int CT = static_cast<int>(C / QT_COLS), RT = static_cast<int>(R / QT_ROWS);
+  auto coords = [&](int t, int& b, int& rt, int& ct) {
+    b = t / (RT * CT);
+    const int rem = t - b * RT * CT;
+    rt = rem / CT;
+    ct = rem - rt * CT;
+  };
+  auto dst_row = [&](int64_t r) -> int64_t {
+    if (!a.gate_up_half) return r;
+    const int64_t hf = a.gate_up_half;
+    return r < hf ? (r / 128) * 256 + (r % 128) : ((r - hf) / 128) * 256 + 128 + ((r - hf) % 128);
+  };
+  auto issue = [&](int t, int slot) {
+    int b, rt, ct;
+    coords(t, b, rt, ct);
+    ptx::mbar_arrive_expect_tx(&full[slot], QW_IN_BYTES);
+    ptx::tma_load_3d(in_base + slot * QW_IN_BYTES, &a.tmap_src, ct * QT_COLS, rt * QT_ROWS, b, &full[slot]);
+  };
+  if (tid == 0) {
+    for (int i = 0; i < QW_NIN; ++i) ptx::mbar_init(&full[i], 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&a.tmap_src);
+    stop = 0;
+  }
+  __syncthreads();
+  int issued_last = 0;  // last tile whose load was issued (waited for at exit only after an abort)
+  if (tid == 0)
+    for (int j = 0; j < QW_NIN; ++j) {
+      const int t = blockIdx.x + j * gridDim.x;
+      if (t < tiles) {
+        issue(t, j);
+        issued_last = t;
+      }
+    }
+  int it = 0;
+  for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+    const int slot = it % QW_NIN;
+    const int ob = it % QW_NOUT;
+    if (tid == 0) {
+      // this tile's source has landed; the stores that last read output buffer ``ob`` are done
+      volatile int* never = &stop;
+      if (!ptx::mbar_wait(&full[slot], static_cast<uint32_t>((it / QW_NIN) & 1), never, kWaitLimitCycles)) {
+        stop = 1;
+        if (a.status) atomicOr(a.status, kStatusTimeout);
+      }
+      asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(QW_NOUT - 1) : "memory");
+    }
+    __syncthreads();
+    if (stop) break;
+    int b, rt, ct;
+    coords(t, b, rt, ct);
+    const int64_t row0 = static_cast<int64_t>(rt) * QT_ROWS, col0 = static_cast<int64_t>(ct) * QT_COLS;
+    const uint8_t* in = in_base + slot * QW_IN_BYTES;
+    uint8_t* qrow = out_base + ob * QW_OUT_BYTES;
+    uint8_t* qcol = qrow + QT_ROWS * QT_COLS;
+    uint8_t* satom_row = atom_base + ob * 1024;
+    uint8_t* satom_col = satom_row + 512;
+
+    // ---- row-wise: thread -> 8-column chunk ``cchunk`` of rows tid/16 + 16 i
+    const int cchunk = tid & 15;
+#pragma unroll
+    for (int i = 0; i < QT_LOADS; ++i) {
+      const int lr = (tid >> 4) + 16 * i;
+      const uint4 v = *reinterpret_cast<const uint4*>(in + lr * 256 + cchunk * 16);
+      uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      const uint32_t sb = e8m0_from_amax_bits(m);
+      const float inv = e8m0_inv_scale(sb);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
+      *reinterpret_cast<uint2*>(qrow + lr * 128 + (((cchunk >> 1) ^ (lr & 7)) << 4) + ((cchunk & 1) << 3)) =
+          make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+      if ((cchunk & 3) == 0) satom_row[sf_mma_offset(lr, (cchunk >> 2) & 3, 4)] = static_cast<uint8_t>(sb);
+    }
+
+    // ---- column-wise: thread -> columns (2p, 2p+1), 32-row block rb
+    {
+      const int p = tid & 63, rb = tid >> 6;
+      const uint32_t* words = reinterpret_cast<const uint32_t*>(in);  // 64 bf16 pairs per row
+      uint32_t wv[32];
+      uint32_t m2 = 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        wv[i] = words[(rb * 32 + i) * 64 + p];
+        m2 = absmax_bf16x2(m2, wv[i]);
+      }
+      const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16), sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u);
+      const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
+      uint32_t q0[8], q1[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t lo0 =
+            e4m3x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0);
+        const uint32_t hi0 =
+            e4m3x2(__uint_as_float(wv[4 * i + 2] << 16) * inv0, __uint_as_float(wv[4 * i + 3] << 16) * inv0);
+        const uint32_t lo1 = e4m3x2(__uint_as_float(wv[4 * i] & 0xFFFF0000u) * inv1,
+                                    __uint_as_float(wv[4 * i + 1] & 0xFFFF0000u) * inv1);
+        const uint32_t hi1 = e4m3x2(__uint_as_float(wv[4 * i + 2] & 0xFFFF0000u) * inv1,
+                                    __uint_as_float(wv[4 * i + 3] & 0xFFFF0000u) * inv1);
+        q0[i] = lo0 | (hi0 << 16);
+        q1[i] = lo1 | (hi1 << 16);
+      }
+      const int r0 = 2 * p, r1 = 2 * p + 1;  // rows of the transposed code tile
+      uint8_t* row0p = qcol + r0 * 128;
+      uint8_t* row1p = qcol + r1 * 128;
+      *reinterpret_cast<uint4*>(row0p + (((2 * rb) ^ (r0 & 7)) << 4)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+      *reinterpret_cast<uint4*>(row0p + (((2 * rb + 1) ^ (r0 & 7)) << 4)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+      *reinterpret_cast<uint4*>(row1p + (((2 * rb) ^ (r1 & 7)) << 4)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+      *reinterpret_cast<uint4*>(row1p + (((2 * rb + 1) ^ (r1 & 7)) << 4)) = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+      satom_col[sf_mma_offset(2 * p, rb, 4)] = static_cast<uint8_t>(sb0);
+      satom_col[sf_mma_offset(2 * p + 1, rb, 4)] = static_cast<uint8_t>(sb1);
+    }
+
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // code tiles -> visible to the copy engine
+    __syncthreads();  // the source tile is consumed, the code tiles and scale tiles are complete
+    if (tid == 0) {
+      asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                       reinterpret_cast<uint64_t>(&a.tmap_qrow)),
+                   "r"(static_cast<int32_t>(col0)), "r"(static_cast<int32_t>(b * R + dst_row(row0))),
+                   "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qrow)))
+                   : "memory");
+      asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                       reinterpret_cast<uint64_t>(&a.tmap_qcol)),
+                   "r"(static_cast<int32_t>(row0)), "r"(static_cast<int32_t>(b * C + col0)),
+                   "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qcol)))
+                   : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      const int tn = t + QW_NIN * gridDim.x;  // refill the slot just consumed
+      if (tn < tiles) {
+        issue(tn, slot);
+        issued_last = tn;
+      }
+    } else if (tid >= 32 && tid < 64) {  // warp 1: the two 512-byte scale tiles, 16 bytes per lane
+      const int l = tid - 32;
+      {
+        uint8_t* sr = a.s_row + static_cast<int64_t>(b) * R * KBr;
+        reinterpret_cast<uint4*>(sr + ((dst_row(row0) / 128) * (KBr / 4) + col0 / 128) * 512)[l] =
+            reinterpret_cast<const uint4*>(satom_row)[l];
+        uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
+        reinterpret_cast<uint4*>(sc + ((col0 / 128) * (KBc / 4) + row0 / 128) * 512)[l] =
+            reinterpret_cast<const uint4*>(satom_col)[l];
+      }
+    }
+  }
+  if (tid == 0) {
+    if (stop) {  // after an abort: the source tiles still in flight land before the CTA exits
+      volatile int never = 0;
+      for (int j = 0; j < QW_NIN; ++j) {
+        const int t = issued_last - j * static_cast<int>(gridDim.x);
+        if (t < static_cast<int>(blockIdx.x)) break;
+        const int k = (t - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x);
+        ptx::mbar_wait(&full[k % QW_NIN], static_cast<uint32_t>((k / QW_NIN) & 1), &never, kWaitLimitCycles);
+      }
+    }
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+  }
+}
+
+// ------------------------------------------------------------------------------------------
 // Combine: y[t] = bf16(sum_j w_j * fp32(rows[row(t, j)])), j ascending, fp32 products and sums.
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
@@ -422,8 +612,16 @@ cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant(const QuantArgs& a, int batch, int /*num_sms*/, cudaStream_t st) {
+cudaError_t launch_quant(const QuantArgs& a, int batch, int num_sms, cudaStream_t st) {
   if (a.rows == 0 || a.cols == 0 || batch == 0) return cudaSuccess;
+  if (a.tma_load && a.tma_store && a.do_row && a.do_col) {
+    const int64_t tiles = (a.rows / QT_ROWS) * (a.cols / QT_COLS) * batch;
+    cudaError_t e = cudaFuncSetAttribute(quant_w_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QW_SMEM);
+    if (e != cudaSuccess) return e;
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, static_cast<int64_t>(num_sms) * QW_CTAS_PER_SM));
+    quant_w_tma_kernel<<<grid, 256, QW_SMEM, st>>>(a, static_cast<int>(tiles));
+    return cudaGetLastError();
+  }
   dim3 grid(static_cast<unsigned>(ceil_div(a.cols, QT_COLS)), static_cast<unsigned>(ceil_div(a.rows, QT_ROWS)),
             static_cast<unsigned>(batch));
   const int dyn = a.tma_store ? 32768 + 1024 : 0;

@@ -33,6 +33,12 @@ struct QuantArgs {
   int tma_store;
   CUtensorMap tmap_qrow;
   CUtensorMap tmap_qcol;
+  // ... and, when the source is one uniformly strided [batch, rows, cols] tensor with rows and
+  // cols multiples of 128, it arrives through TMA tensor loads (bf16 map over [batch, rows, cols],
+  // 128 x 128 boxes) into a persistent kernel's ring of tiles
+  int tma_load;
+  CUtensorMap tmap_src;
+  int* status;                 // device status word (a bounded wait that expired)
 };
 
 cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk, int E, int capacity,

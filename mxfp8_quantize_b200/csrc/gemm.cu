@@ -116,14 +116,6 @@ __device__ __forceinline__ void decode_tile(int t, const SharedState& s, const G
   }
 }
 
-__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, int32_t x, int32_t y, int32_t z,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(ptx::smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(ptx::smem_u32(bar))
-      : "memory");
-}
 
 // silu(g) = g * sigmoid(g); sigmoid from the hardware exp2 and a fast reciprocal-multiply
 __device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
@@ -318,19 +310,19 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         ptx::tma_load_2d(st, &g.tmap_a, kx, tl.a_row, &s.full[stage]);
         if (!g.kgrouped && g.gate_up_half) {
           // bf16 gate_up: BN/2 gate rows then the matching BN/2 up rows of expert e
-          tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * (BN / 2), tl.e, &s.full[stage]);
-          tma_load_3d(st + S::OFF_B + S::B_BYTES / 2, &g.tmap_b, kx, g.gate_up_half + tl.nb * (BN / 2), tl.e,
+          ptx::tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * (BN / 2), tl.e, &s.full[stage]);
+          ptx::tma_load_3d(st + S::OFF_B + S::B_BYTES / 2, &g.tmap_b, kx, g.gate_up_half + tl.nb * (BN / 2), tl.e,
                       &s.full[stage]);
         } else if (!g.kgrouped) {  // one box of BN rows
-          tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * BN, tl.e, &s.full[stage]);
+          ptx::tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * BN, tl.e, &s.full[stage]);
         } else {
           ptx::tma_load_2d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * BN, &s.full[stage]);
         }
         if (MX) {  // this step's scale tiles: one of A, BN/128 consecutive ones of B
           const int32_t kq = kx / 128;
           const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * g.sfb_expert_rows;
-          tma_load_3d(st + S::OFF_SFA, &g.tmap_sfa, 0, kq, tl.a_row / 128, &s.full[stage]);
-          tma_load_3d(st + S::OFF_SFB, &g.tmap_sfb, 0, kq,
+          ptx::tma_load_3d(st + S::OFF_SFA, &g.tmap_sfa, 0, kq, tl.a_row / 128, &s.full[stage]);
+          ptx::tma_load_3d(st + S::OFF_SFB, &g.tmap_sfb, 0, kq,
                       static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128), &s.full[stage]);
         }
         issued_mask |= 1u << stage;
