@@ -141,7 +141,7 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
-// MXFP8 of 32 values with the scale of their own amax: 32 codes stored at q (16-byte aligned);
+// MXFP8 of 32 values with the scale of their own amax: 32 codes stored at q (32-byte aligned);
 // returns the E8M0 byte.
 __device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q) {
   uint32_t m = 0;
@@ -153,8 +153,7 @@ __device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q) {
 #pragma unroll
   for (int i = 0; i < 8; ++i)
     w[i] = e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv) | (e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv) << 16);
-  reinterpret_cast<uint4*>(q)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  reinterpret_cast<uint4*>(q)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  ptx::st_global_v8(q, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
   return sb;
 }
 
@@ -463,9 +462,17 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
         bf16* out = g.kgrouped ? static_cast<bf16*>(const_cast<void*>(ep.out_ptrs.p[tl.e])) : ep.out;
-        uint4* dst = reinterpret_cast<uint4*>(out + row * ep.ldo + static_cast<int64_t>(tl.nb) * BN + CPT * ch);
+        bf16* orow = out + row * ep.ldo + static_cast<int64_t>(tl.nb) * BN + CPT * ch;
+        if ((reinterpret_cast<uintptr_t>(out) & 31u) == 0 && (ep.ldo & 15) == 0) {  // whole 32-byte sectors
 #pragma unroll
-        for (int i = 0; i < CPT / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          for (int i = 0; i < CPT / 16; ++i)
+            ptx::st_global_v8(orow + 16 * i, make_uint4(pk[8 * i], pk[8 * i + 1], pk[8 * i + 2], pk[8 * i + 3]),
+                              make_uint4(pk[8 * i + 4], pk[8 * i + 5], pk[8 * i + 6], pk[8 * i + 7]));
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+          for (int i = 0; i < CPT / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
       } else if (EPI == EPI_SWIGLU) {
         // tile = BN/2 output columns; accumulator columns [0,BN/2) gate, [BN/2,BN) up
         constexpr int OPT = BN / 2 / NPART;  // output columns per thread
@@ -486,14 +493,13 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
           }
-          if (ep.h) {
-            uint4* hg = reinterpret_cast<uint4*>(ep.h + row * 2 * f + j);
-            uint4* hu = reinterpret_cast<uint4*>(ep.h + row * 2 * f + f + j);
+          if (ep.h) {  // saved gate/up pre-activations: 64 bytes of each per row, in 32-byte stores
+            bf16* hg = ep.h + row * 2 * f + j;
+            bf16* hu = hg + f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              hg[i] = pack_bf16x8(gv + 8 * i);
-              hu[i] = pack_bf16x8(uv + 8 * i);
-            }
+            for (int i = 0; i < 2; ++i) ptx::st_global_v8(hg + 16 * i, pack_bf16x8(gv + 16 * i), pack_bf16x8(gv + 16 * i + 8));
+#pragma unroll
+            for (int i = 0; i < 2; ++i) ptx::st_global_v8(hu + 16 * i, pack_bf16x8(uv + 16 * i), pack_bf16x8(uv + 16 * i + 8));
           }
 #pragma unroll
           for (int i = 0; i < 32; ++i) gv[i] = gv[i] * sigmoid_f(gv[i]) * uv[i] * p;  // a, in place
@@ -509,9 +515,9 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
               colwise_mx<S::PASS>(gv, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
                                   ep.cap / 32);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(ep.o_row + row * f + j);
+            bf16* dst = ep.o_row + row * f + j;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = pack_bf16x8(gv + 8 * i);
+            for (int i = 0; i < 2; ++i) ptx::st_global_v8(dst + 16 * i, pack_bf16x8(gv + 16 * i), pack_bf16x8(gv + 16 * i + 8));
             if (ep.o_colT) colwise_bf16<S::PASS>(gv, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
           }
         }
@@ -609,12 +615,12 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             colwise_mx<S::PASS>(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j,
                                 row_w / 32, ep.cap / 32);
           } else {
-            uint4* d0 = reinterpret_cast<uint4*>(ep.o_row + row * f2 + j);
-            uint4* d1 = reinterpret_cast<uint4*>(ep.o_row + row * f2 + f + j);
+            bf16* d0 = ep.o_row + row * f2 + j;
+            bf16* d1 = d0 + f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              d0[i] = pack_bf16x8(dg + 8 * i);
-              d1[i] = pack_bf16x8(du + 8 * i);
+            for (int i = 0; i < 2; ++i) {
+              ptx::st_global_v8(d0 + 16 * i, pack_bf16x8(dg + 16 * i), pack_bf16x8(dg + 16 * i + 8));
+              ptx::st_global_v8(d1 + 16 * i, pack_bf16x8(du + 16 * i), pack_bf16x8(du + 16 * i + 8));
             }
             colwise_bf16<S::PASS>(dg, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
             colwise_bf16<S::PASS>(du, stage_buf, ep.o_colT + (f + j) * ep.cap + row_w, ep.cap);
