@@ -286,8 +286,10 @@ def run_ours(args, cfg, rank, world, local_rank):
     if os.path.exists(tpath):
         import hashlib
         rec = json.load(open(tpath))
-        src = os.path.join(ROOT, "mxfp8_quantize_b200", "csrc", "gemm.cu")
-        if hashlib.sha1(open(src, "rb").read()).hexdigest()[:12] == rec.get("gemm_cu_sha1"):
+        h = hashlib.sha1()
+        for fn in rec.get("sources", []):
+            h.update(open(os.path.join(ROOT, fn), "rb").read())
+        if rec.get("sources") and h.hexdigest()[:12] == rec.get("sources_sha1"):
             traffic = rec.get(cfg.name, {}).get(dom)  # counters taken on this very kernel source
     roofline = {"bound": kind, "kernel": dom, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
                 "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -349,7 +351,7 @@ def config_desc(cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="mixtral_mxfp8", choices=sorted(workloads.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
