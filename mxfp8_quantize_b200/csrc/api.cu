@@ -242,7 +242,7 @@ void carve_bwd(Carve& c, const Dims& D, BwdWs& w) {
     w.w2T = c.take<bf16>(D.E * D.f * D.d * 2);
   }
   w.dx_perm = c.take<bf16>(D.cap * D.d * 2);
-  w.dp_part = c.take<float>(2 * (D.f / gemm_tile_n(EPI_DSWIGLU)) * D.cap * 4);
+  w.dp_part = c.take<float>(gemm_dswiglu_parts() * (D.f / gemm_tile_n(EPI_DSWIGLU)) * D.cap * 4);
 }
 
 int64_t capacity_rows(int64_t T, int k, int E) {
@@ -914,7 +914,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   }
   // 6. combine dx, reduce the probability gradient
   MOE_LAUNCH(ctx, "unpermute_dx", st, launch_unpermute(w.dx_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(dx), ctx->num_sms, st));
-  MOE_LAUNCH(ctx, "dprob_reduce", st, launch_dprob_reduce(w.dp_part, static_cast<int>(2 * (f / gemm_tile_n(EPI_DSWIGLU))), D.cap, s.src2s, D.Tk,
+  MOE_LAUNCH(ctx, "dprob_reduce", st, launch_dprob_reduce(w.dp_part, static_cast<int>(gemm_dswiglu_parts() * (f / gemm_tile_n(EPI_DSWIGLU))), D.cap, s.src2s, D.Tk,
                                            d_topk_prob, st));
   return MOE_OK;
 }

@@ -626,7 +626,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             colwise_bf16<S::PASS>(du, stage_buf, ep.o_colT + (f + j) * ep.cap + row_w, ep.cap);
           }
         }
-        ep.dp_part[(static_cast<int64_t>(tl.nb) * 2 + ch) * ep.cap + row] = dp;
+        ep.dp_part[(static_cast<int64_t>(tl.nb) * NPART + ch) * ep.cap + row] = dp;
       }
     }
   }
@@ -653,6 +653,8 @@ cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
 int gemm_tile_n(int epi) {
   return epi == EPI_STORE ? ShapeStore::BN : (epi == EPI_SWIGLU ? ShapeSwiglu::BN : ShapeDswiglu::BN);
 }
+
+int gemm_dswiglu_parts() { return ShapeDswiglu::EPI_WARPS / 4; }
 
 cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st) {
   if (mx) {

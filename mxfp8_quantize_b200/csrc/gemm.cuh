@@ -29,7 +29,7 @@ struct EpiArgs {
   bf16* o_row;        // BF16 path equivalents
   bf16* o_colT;
   float* dump;        // debug: fp32 values before quantisation
-  float* dp_part;     // DSWIGLU: [2 * n_tiles, cap] partial sums of the probability gradient
+  float* dp_part;     // DSWIGLU: [parts * n_tiles, cap] partial sums of the probability gradient
 };
 
 struct GemmArgs {
@@ -60,6 +60,8 @@ struct GemmArgs {
 
 // Output tile width (N) of the kernel used for an epilogue kind.
 int gemm_tile_n(int epi);
+// Partial sums of the probability gradient the dSwiGLU epilogue writes per output tile and row.
+int gemm_dswiglu_parts();
 
 // Launch one grouped GEMM.  ``mx``: MXFP8 (kind::mxf8f6f4) or BF16 (kind::f16).
 cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st);
