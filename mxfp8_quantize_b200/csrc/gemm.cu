@@ -363,6 +363,13 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     uint32_t phase = 0;
     int local = 0;  // tiles with MMAs issued by this CTA
     bool issued_any = false;
+    // descriptors of stage 0; stage s adds s * STAGE_BYTES / 16 to the 14-bit start-address field
+    // (shared addresses stay below 2^18, so the sum never carries out of it)
+    const uint32_t smem0 = ptx::smem_u32(smem);
+    const uint64_t adesc0 = ptx::smem_desc(smem0, 16, 1024, ptx::kSwizzle128B);
+    const uint64_t bdesc0 = ptx::smem_desc(smem0 + S::OFF_B, 16, 1024, ptx::kSwizzle128B);
+    const uint64_t sfadesc0 = ptx::smem_desc(smem0 + S::OFF_SFA, 0, 128, ptx::kSwizzleNone);
+    const uint64_t sfbdesc0 = ptx::smem_desc(smem0 + S::OFF_SFB, 0, 128, ptx::kSwizzleNone);
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
@@ -379,17 +386,15 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t st = ptx::smem_u32(smem + stage * S::STAGE_BYTES);
-        const uint64_t adesc = ptx::smem_desc(st, 16, 1024, ptx::kSwizzle128B);
-        const uint64_t bdesc = ptx::smem_desc(st + S::OFF_B, 16, 1024, ptx::kSwizzle128B);
+        const uint64_t soff = static_cast<uint64_t>(stage * (S::STAGE_BYTES >> 4));
+        const uint64_t adesc = adesc0 + soff;
+        const uint64_t bdesc = bdesc0 + soff;
         if (MX) {
           const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * stage;
           const uint32_t sfb_t = sfa_t + 4;
-          ptx::tc_cp_32x128b_warpx4(sfa_t, ptx::smem_desc(st + S::OFF_SFA, 0, 128, ptx::kSwizzleNone));
+          ptx::tc_cp_32x128b_warpx4(sfa_t, sfadesc0 + soff);
 #pragma unroll
-          for (int i = 0; i < BN / 128; ++i)
-            ptx::tc_cp_32x128b_warpx4(sfb_t + 4 * i,
-                                      ptx::smem_desc(st + S::OFF_SFB + 512 * i, 0, 128, ptx::kSwizzleNone));
+          for (int i = 0; i < BN / 128; ++i) ptx::tc_cp_32x128b_warpx4(sfb_t + 4 * i, sfbdesc0 + soff + 32 * i);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             ptx::tc_mma_mxf8(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(BM, BN, k, k), sfa_t, sfb_t,
