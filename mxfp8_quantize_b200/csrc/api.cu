@@ -92,7 +92,8 @@ int64_t uniform_stride(const void* const* p, int E, int64_t min_bytes);
 // strided [batch, rows, cols] bf16 source with 16-byte aligned rows, rows and cols multiples of 128.
 void quant_load_map(QuantArgs& a, int batch) {
   a.tma_load = 0;
-  if (a.sorted_to_src || a.rows % 128 || a.cols % 128 || !a.do_row || !a.do_col) return;
+  const bool outputs_ok = a.mx ? (a.do_row && a.do_col) : (a.do_col && !a.do_row);  // the kernel's two modes
+  if (a.sorted_to_src || a.rows % 128 || a.cols % 128 || !outputs_ok) return;
   const void* base = a.src_ptrs.p[0] ? a.src_ptrs.p[0] : a.src;
   const int64_t row_bytes = a.src_ld * 2, tile_bytes = a.rows * row_bytes;
   int64_t stride = a.src_ptrs.p[0] ? uniform_stride(a.src_ptrs.p, batch, tile_bytes) : a.src_batch_stride * 2;
@@ -111,7 +112,26 @@ void quant_load_map(QuantArgs& a, int batch) {
 bool quant_store_maps(QuantArgs& a, int batch) {
   a.tma_store = 0;
   a.tma_load = 0;
-  if (!a.mx || !a.sf_mma) return true;
+  if (!a.mx) {
+    // bf16 transpose of a strided source: the TMA-fed kernel writes the transposed tiles through
+    // a bf16 map over [batch*cols, rows] (boxes of 64 columns x 128 rows); otherwise the tile kernel
+    quant_load_map(a, batch);
+    if (!a.tma_load) return true;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.rows), static_cast<cuuint64_t>(batch) * a.cols};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.rows) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t es[2] = {1, 1};
+    if (!aligned16(a.o_colT) ||
+        g_encode(&a.tmap_qcol, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.o_colT, dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      a.tma_load = 0;
+      return true;
+    }
+    a.tma_store = 1;
+    return true;
+  }
+  if (!a.sf_mma) return true;
   const uint64_t R = a.rows, C = a.cols, B = batch;
   cuuint32_t box[2] = {128, 128};
   cuuint32_t es[2] = {1, 1};

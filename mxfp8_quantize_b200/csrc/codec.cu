@@ -357,6 +357,7 @@ constexpr int QW_CTAS_PER_SM = 2;
 constexpr int QW_IN_BYTES = QT_ROWS * QT_COLS * 2;  // one bf16 source tile, rows of 256 bytes
 constexpr int QW_OUT_BYTES = 2 * QT_ROWS * QT_COLS;  // row-wise + column-wise code tiles
 constexpr int QW_SMEM = QW_NIN * QW_IN_BYTES + QW_NOUT * (QW_OUT_BYTES + 1024) + 1024;
+static_assert(QW_OUT_BYTES >= QT_ROWS * QT_COLS * 2, "an output buffer also holds one transposed bf16 tile");
 }  // namespace
 
 __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const __grid_constant__ QuantArgs a, int tiles) {
@@ -427,85 +428,120 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
     uint8_t* satom_row = atom_base + ob * 1024;
     uint8_t* satom_col = satom_row + 512;
 
-    // ---- row-wise: thread -> 8-column chunk ``cchunk`` of rows tid/16 + 16 i
-    const int cchunk = tid & 15;
-#pragma unroll
-    for (int i = 0; i < QT_LOADS; ++i) {
-      const int lr = (tid >> 4) + 16 * i;
-      const uint4 v = *reinterpret_cast<const uint4*>(in + lr * 256 + cchunk * 16);
-      uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      const uint32_t sb = e8m0_from_amax_bits(m);
-      const float inv = e8m0_inv_scale(sb);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint32_t q[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
-      *reinterpret_cast<uint2*>(qrow + lr * 128 + (((cchunk >> 1) ^ (lr & 7)) << 4) + ((cchunk & 1) << 3)) =
-          make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
-      if ((cchunk & 3) == 0) satom_row[sf_mma_offset(lr, (cchunk >> 2) & 3, 4)] = static_cast<uint8_t>(sb);
-    }
-
-    // ---- column-wise: thread -> columns (2p, 2p+1), 32-row block rb
-    {
+    if (!a.mx) {
+      // bf16 transpose only: thread -> columns (2p, 2p+1) = rows of the transposed tile, source rows
+      // 32 rb .. +31; the transposed tile (32 KB: the whole output buffer, there are no row-wise
+      // codes) is two 64-column halves of 128-byte rows, 128B-swizzled
       const int p = tid & 63, rb = tid >> 6;
       const uint32_t* words = reinterpret_cast<const uint32_t*>(in);  // 64 bf16 pairs per row
-      uint32_t wv[32];
-      uint32_t m2 = 0;
+      uint32_t c0[16], c1[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        wv[i] = words[(rb * 32 + i) * 64 + p];
-        m2 = absmax_bf16x2(m2, wv[i]);
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t w0 = words[(rb * 32 + 2 * i) * 64 + p], w1 = words[(rb * 32 + 2 * i + 1) * 64 + p];
+        c0[i] = __byte_perm(w0, w1, 0x5410);  // low halves: column 2p
+        c1[i] = __byte_perm(w0, w1, 0x7632);  // high halves: column 2p+1
       }
-      const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16), sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u);
-      const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
-      uint32_t q0[8], q1[8];
+      uint8_t* half = qrow + (rb >> 1) * (QT_ROWS * 128);
+      const int r0 = 2 * p, r1 = 2 * p + 1;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t lo0 =
-            e4m3x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0);
-        const uint32_t hi0 =
-            e4m3x2(__uint_as_float(wv[4 * i + 2] << 16) * inv0, __uint_as_float(wv[4 * i + 3] << 16) * inv0);
-        const uint32_t lo1 = e4m3x2(__uint_as_float(wv[4 * i] & 0xFFFF0000u) * inv1,
-                                    __uint_as_float(wv[4 * i + 1] & 0xFFFF0000u) * inv1);
-        const uint32_t hi1 = e4m3x2(__uint_as_float(wv[4 * i + 2] & 0xFFFF0000u) * inv1,
-                                    __uint_as_float(wv[4 * i + 3] & 0xFFFF0000u) * inv1);
-        q0[i] = lo0 | (hi0 << 16);
-        q1[i] = lo1 | (hi1 << 16);
+      for (int j = 0; j < 4; ++j) {
+        const int chunk = (rb & 1) * 4 + j;
+        *reinterpret_cast<uint4*>(half + r0 * 128 + ((chunk ^ (r0 & 7)) << 4)) =
+            make_uint4(c0[4 * j], c0[4 * j + 1], c0[4 * j + 2], c0[4 * j + 3]);
+        *reinterpret_cast<uint4*>(half + r1 * 128 + ((chunk ^ (r1 & 7)) << 4)) =
+            make_uint4(c1[4 * j], c1[4 * j + 1], c1[4 * j + 2], c1[4 * j + 3]);
       }
-      const int r0 = 2 * p, r1 = 2 * p + 1;  // rows of the transposed code tile
-      uint8_t* row0p = qcol + r0 * 128;
-      uint8_t* row1p = qcol + r1 * 128;
-      *reinterpret_cast<uint4*>(row0p + (((2 * rb) ^ (r0 & 7)) << 4)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
-      *reinterpret_cast<uint4*>(row0p + (((2 * rb + 1) ^ (r0 & 7)) << 4)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
-      *reinterpret_cast<uint4*>(row1p + (((2 * rb) ^ (r1 & 7)) << 4)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
-      *reinterpret_cast<uint4*>(row1p + (((2 * rb + 1) ^ (r1 & 7)) << 4)) = make_uint4(q1[4], q1[5], q1[6], q1[7]);
-      satom_col[sf_mma_offset(2 * p, rb, 4)] = static_cast<uint8_t>(sb0);
-      satom_col[sf_mma_offset(2 * p + 1, rb, 4)] = static_cast<uint8_t>(sb1);
+    } else {
+      // ---- row-wise: thread -> 8-column chunk ``cchunk`` of rows tid/16 + 16 i
+      const int cchunk = tid & 15;
+  #pragma unroll
+      for (int i = 0; i < QT_LOADS; ++i) {
+        const int lr = (tid >> 4) + 16 * i;
+        const uint4 v = *reinterpret_cast<const uint4*>(in + lr * 256 + cchunk * 16);
+        uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        const uint32_t sb = e8m0_from_amax_bits(m);
+        const float inv = e8m0_inv_scale(sb);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t q[4];
+  #pragma unroll
+        for (int j = 0; j < 4; ++j)
+          q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
+        *reinterpret_cast<uint2*>(qrow + lr * 128 + (((cchunk >> 1) ^ (lr & 7)) << 4) + ((cchunk & 1) << 3)) =
+            make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+        if ((cchunk & 3) == 0) satom_row[sf_mma_offset(lr, (cchunk >> 2) & 3, 4)] = static_cast<uint8_t>(sb);
+      }
+
+      // ---- column-wise: thread -> columns (2p, 2p+1), 32-row block rb
+      {
+        const int p = tid & 63, rb = tid >> 6;
+        const uint32_t* words = reinterpret_cast<const uint32_t*>(in);  // 64 bf16 pairs per row
+        uint32_t wv[32];
+        uint32_t m2 = 0;
+  #pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          wv[i] = words[(rb * 32 + i) * 64 + p];
+          m2 = absmax_bf16x2(m2, wv[i]);
+        }
+        const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16), sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u);
+        const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
+        uint32_t q0[8], q1[8];
+  #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t lo0 =
+              e4m3x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0);
+          const uint32_t hi0 =
+              e4m3x2(__uint_as_float(wv[4 * i + 2] << 16) * inv0, __uint_as_float(wv[4 * i + 3] << 16) * inv0);
+          const uint32_t lo1 = e4m3x2(__uint_as_float(wv[4 * i] & 0xFFFF0000u) * inv1,
+                                      __uint_as_float(wv[4 * i + 1] & 0xFFFF0000u) * inv1);
+          const uint32_t hi1 = e4m3x2(__uint_as_float(wv[4 * i + 2] & 0xFFFF0000u) * inv1,
+                                      __uint_as_float(wv[4 * i + 3] & 0xFFFF0000u) * inv1);
+          q0[i] = lo0 | (hi0 << 16);
+          q1[i] = lo1 | (hi1 << 16);
+        }
+        const int r0 = 2 * p, r1 = 2 * p + 1;  // rows of the transposed code tile
+        uint8_t* row0p = qcol + r0 * 128;
+        uint8_t* row1p = qcol + r1 * 128;
+        *reinterpret_cast<uint4*>(row0p + (((2 * rb) ^ (r0 & 7)) << 4)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+        *reinterpret_cast<uint4*>(row0p + (((2 * rb + 1) ^ (r0 & 7)) << 4)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+        *reinterpret_cast<uint4*>(row1p + (((2 * rb) ^ (r1 & 7)) << 4)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+        *reinterpret_cast<uint4*>(row1p + (((2 * rb + 1) ^ (r1 & 7)) << 4)) = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+        satom_col[sf_mma_offset(2 * p, rb, 4)] = static_cast<uint8_t>(sb0);
+        satom_col[sf_mma_offset(2 * p + 1, rb, 4)] = static_cast<uint8_t>(sb1);
+      }
     }
 
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // code tiles -> visible to the copy engine
     __syncthreads();  // the source tile is consumed, the code tiles and scale tiles are complete
     if (tid == 0) {
-      asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                       reinterpret_cast<uint64_t>(&a.tmap_qrow)),
-                   "r"(static_cast<int32_t>(col0)), "r"(static_cast<int32_t>(b * R + dst_row(row0))),
-                   "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qrow)))
-                   : "memory");
-      asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                       reinterpret_cast<uint64_t>(&a.tmap_qcol)),
-                   "r"(static_cast<int32_t>(row0)), "r"(static_cast<int32_t>(b * C + col0)),
-                   "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qcol)))
-                   : "memory");
+      if (a.mx) {
+        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                         reinterpret_cast<uint64_t>(&a.tmap_qrow)),
+                     "r"(static_cast<int32_t>(col0)), "r"(static_cast<int32_t>(b * R + dst_row(row0))),
+                     "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qrow)))
+                     : "memory");
+        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                         reinterpret_cast<uint64_t>(&a.tmap_qcol)),
+                     "r"(static_cast<int32_t>(row0)), "r"(static_cast<int32_t>(b * C + col0)),
+                     "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qcol)))
+                     : "memory");
+      } else {  // the transposed bf16 tile: two boxes of 64 columns x 128 rows
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                           reinterpret_cast<uint64_t>(&a.tmap_qcol)),
+                       "r"(static_cast<int32_t>(row0 + 64 * h)), "r"(static_cast<int32_t>(b * C + col0)),
+                       "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qrow + h * QT_ROWS * 128)))
+                       : "memory");
+      }
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       const int tn = t + QW_NIN * gridDim.x;  // refill the slot just consumed
       if (tn < tiles) {
         issue(tn, slot);
         issued_last = tn;
       }
-    } else if (tid >= 32 && tid < 64) {  // warp 1: the two 512-byte scale tiles, 16 bytes per lane
+    } else if (a.mx && tid >= 32 && tid < 64) {  // warp 1: the two 512-byte scale tiles, 16 bytes per lane
       const int l = tid - 32;
       {
         uint8_t* sr = a.s_row + static_cast<int64_t>(b) * R * KBr;
@@ -614,7 +650,7 @@ cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk
 
 cudaError_t launch_quant(const QuantArgs& a, int batch, int num_sms, cudaStream_t st) {
   if (a.rows == 0 || a.cols == 0 || batch == 0) return cudaSuccess;
-  if (a.tma_load && a.tma_store && a.do_row && a.do_col) {
+  if (a.tma_load && a.tma_store && (a.mx ? (a.do_row && a.do_col) : (a.do_col && !a.do_row))) {
     const int64_t tiles = (a.rows / QT_ROWS) * (a.cols / QT_COLS) * batch;
     cudaError_t e = cudaFuncSetAttribute(quant_w_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QW_SMEM);
     if (e != cudaSuccess) return e;

@@ -179,3 +179,38 @@ def test_small_outputs_within_tolerance(small, name):
         assert np.all(got[7] == 0)   # expert 7 receives no tokens
     if name == "dw2":
         assert np.all(got[7] == 0)
+
+
+def _scattered(w: torch.Tensor):
+    """The experts of a stacked [E, r, c] weight copied to irregularly spaced places of one buffer
+    (gaps of 0, 256, 512, ... elements), so that no uniform stride covers them."""
+    E, r, c = w.shape
+    gaps = [256 * e for e in range(E)]
+    buf = torch.zeros(E * r * c + sum(gaps), dtype=w.dtype, device=w.device)
+    out, off = [], 0
+    for e in range(E):
+        off += gaps[e]
+        v = buf[off:off + r * c].view(r, c)
+        v.copy_(w[e])
+        out.append(v)
+        off += r * c
+    return out
+
+
+@pytest.mark.parametrize("precision", ["mxfp8", "bf16"])
+def test_scattered_expert_weights_match_stacked(precision):
+    """Experts given as separately placed tensors take the general paths (the tile quantiser, the
+    bf16 weight gather) instead of the strided ones (TMA-fed quantiser, 3-D weight maps): every
+    output must be identical."""
+    cfg = workloads.scaled_config(workloads.CONFIGS["small_mxfp8"], precision=precision, T=1024)
+    inp = workloads.make_inputs(cfg, with_dy=True)
+    dev = {n: t.cuda() for n, t in inp.items()}
+    res = []
+    for w1, w2 in [(dev["w_gate_up"], dev["w_down"]), (_scattered(dev["w_gate_up"]), _scattered(dev["w_down"]))]:
+        y, saved = moe.moe_grouped_mlp_fwd(dev["x"], dev["topk_idx"], dev["topk_prob"], w1, w2,
+                                           precision=precision, training=True)
+        dx, dw1, dw2, dp = moe.moe_grouped_mlp_bwd(dev["dy"], saved, w1, w2)
+        moe.get_status(0)
+        res.append([t.float().cpu() if t.dtype == torch.bfloat16 else t.cpu() for t in (y, dx, dw1, dw2, dp)])
+    for name, a, b in zip(("y", "dx", "dw_gate_up", "dw_down", "d_topk_prob"), *res):
+        assert torch.equal(a, b), name
