@@ -92,8 +92,27 @@ int64_t uniform_stride(const void* const* p, int E, int64_t min_bytes);
 // strided [batch, rows, cols] bf16 source with 16-byte aligned rows, rows and cols multiples of 128.
 void quant_load_map(QuantArgs& a, int batch) {
   a.tma_load = 0;
+  a.tma_gather = 0;
   const bool outputs_ok = a.mx ? (a.do_row && a.do_col) : (a.do_col && !a.do_row);  // the kernel's two modes
-  if (a.sorted_to_src || a.rows % 128 || a.cols % 128 || !outputs_ok) return;
+  if (a.rows % 128 || a.cols % 128 || !outputs_ok) return;
+  if (a.sorted_to_src) {
+    // MXFP8 gather of one [src_rows, cols] source: rows fetched four at a time by tile::gather4
+    // through a map whose box is one row of 128 columns
+    if (!a.mx || batch != 1 || a.src_ptrs.p[0] || !a.src || !aligned16(a.src) || ((a.src_ld * 2) & 15) ||
+        a.src_rows <= 0 || a.src_rows >= (int64_t(1) << 31))
+      return;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.cols), static_cast<cuuint64_t>(a.src_rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.src_ld) * 2};
+    cuuint32_t box[2] = {128, 1};
+    cuuint32_t es[2] = {1, 1};
+    if (g_encode(&a.tmap_src, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<bf16*>(a.src), dims, strides, box, es,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS) {
+      a.tma_load = 1;
+      a.tma_gather = 1;
+    }
+    return;
+  }
   const void* base = a.src_ptrs.p[0] ? a.src_ptrs.p[0] : a.src;
   const int64_t row_bytes = a.src_ld * 2, tile_bytes = a.rows * row_bytes;
   int64_t stride = a.src_ptrs.p[0] ? uniform_stride(a.src_ptrs.p, batch, tile_bytes) : a.src_batch_stride * 2;
@@ -625,6 +644,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.src = static_cast<const bf16*>(x);
     xa.src_ld = d;
     xa.sorted_to_src = s.s2src;
+    xa.src_rows = T;
     xa.k = k;
     xa.rows = D.cap;
     xa.cols = d;
@@ -672,6 +692,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.src = static_cast<const bf16*>(x);
     xa.src_ld = d;
     xa.sorted_to_src = s.s2src;
+    xa.src_rows = T;
     xa.k = k;
     xa.rows = D.cap;
     xa.cols = d;
@@ -784,6 +805,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     a.src = static_cast<const bf16*>(dy);
     a.src_ld = d;
     a.sorted_to_src = s.s2src;
+    a.src_rows = T;
     a.k = k;
     a.rows = D.cap;
     a.cols = d;

@@ -382,12 +382,29 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
     const int64_t hf = a.gate_up_half;
     return r < hf ? (r / 128) * 256 + (r % 128) : ((r - hf) / 128) * 256 + 128 + ((r - hf) % 128);
   };
+  // source tile t into ring slot ``slot``: one 3-D box (thread 0), or, for a gather, 32 gather4
+  // loads of four rows each (one per lane of warp 0)
   auto issue = [&](int t, int slot) {
     int b, rt, ct;
     coords(t, b, rt, ct);
-    ptx::mbar_arrive_expect_tx(&full[slot], QW_IN_BYTES);
-    ptx::tma_load_3d(in_base + slot * QW_IN_BYTES, &a.tmap_src, ct * QT_COLS, rt * QT_ROWS, b, &full[slot]);
+    if (!a.tma_gather) {
+      ptx::mbar_arrive_expect_tx(&full[slot], QW_IN_BYTES);
+      ptx::tma_load_3d(in_base + slot * QW_IN_BYTES, &a.tmap_src, ct * QT_COLS, rt * QT_ROWS, b, &full[slot]);
+      return;
+    }
+    const int lane = tid & 31;
+    const int64_t r0 = static_cast<int64_t>(rt) * QT_ROWS + 4 * lane;
+    int32_t y[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int32_t s = a.sorted_to_src[r0 + j];
+      y[j] = s < 0 ? static_cast<int32_t>(a.src_rows) : s / a.k;  // padding: past the last row -> zeros
+    }
+    if (lane == 0) ptx::mbar_arrive_expect_tx(&full[slot], QW_IN_BYTES);
+    ptx::tma_gather4(in_base + slot * QW_IN_BYTES + lane * 4 * 256, &a.tmap_src, ct * QT_COLS, y[0], y[1], y[2], y[3],
+                     &full[slot]);
   };
+  const bool issuer = a.tma_gather ? tid < 32 : tid == 0;
   if (tid == 0) {
     for (int i = 0; i < QW_NIN; ++i) ptx::mbar_init(&full[i], 1);
     ptx::fence_mbar_init();
@@ -396,7 +413,7 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
   }
   __syncthreads();
   int issued_last = 0;  // last tile whose load was issued (waited for at exit only after an abort)
-  if (tid == 0)
+  if (issuer)
     for (int j = 0; j < QW_NIN; ++j) {
       const int t = blockIdx.x + j * gridDim.x;
       if (t < tiles) {
@@ -536,6 +553,8 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
                        : "memory");
       }
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    if (issuer) {
       const int tn = t + QW_NIN * gridDim.x;  // refill the slot just consumed
       if (tn < tiles) {
         issue(tn, slot);

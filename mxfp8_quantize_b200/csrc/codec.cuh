@@ -38,6 +38,11 @@ struct QuantArgs {
   // 128 x 128 boxes) into a persistent kernel's ring of tiles
   int tma_load;
   CUtensorMap tmap_src;
+  // ... or, for a gather (``sorted_to_src``), a 2-D bf16 map over the [src_rows, cols] source
+  // whose boxes are single rows, four of them per tile::gather4 load (padding rows read past
+  // src_rows, which the copy fills with zeros)
+  int tma_gather;
+  int64_t src_rows;
   int* status;                 // device status word (a bounded wait that expired)
 };
 
