@@ -11,16 +11,19 @@
 // loop while handling uneven counts in one launch (andresseo.expert, "Fragmented Expert
 // Kernels") is what the tile list provides.
 //
-// One CTA per SM, 12 warps:
+// One CTA per SM, 4 + EPI_WARPS warps:
 //   warp 0  TMA producer (one thread): operand tiles + scale tiles into a STAGES-deep smem ring
+//           (scale tiles as 3-D tensor-map boxes over the tile-layout scale buffers)
 //   warp 1  MMA issuer (one thread): scale tiles smem->TMEM, 4 MMAs per stage, commits
 //   warp 2  TMEM allocator
-//   warps 4-11 epilogue: TMEM -> registers -> fused math -> global stores
-// Tiles are 128 x 256 with one TMEM accumulator (two 256-column accumulators would leave no room
-// for the per-stage scale tiles; the template keeps a double-buffered variant available).  Plain
+//   warps 4.. epilogue: TMEM -> registers -> fused math -> global stores
+// The bf16-store and gate_up kernels use 128 x 256 tiles with one TMEM accumulator (two
+// 256-column accumulators would leave no room for the per-stage scale tiles); the dSwiGLU kernel
+// uses 128 x 128 tiles with two, so that its heavy epilogue overlaps the next tile's MMAs.  Plain
 // bf16-store epilogues drain the accumulator into packed registers and release it before storing;
 // the fused ScaledSwiGLU / dSwiGLU epilogues release it after their last TMEM load and requantise
-// column-wise through a small padded smem transpose (one scale per column per lane).
+// column-wise through a small padded smem transpose (one scale per column per lane).  Row-strided
+// outputs leave in 256-bit stores (a whole 32-byte sector per lane).
 // Every wait is bounded: on expiry the kernel records MOE_ERR_TIMEOUT and all roles stop.
 #include <cuda_fp8.h>
 
