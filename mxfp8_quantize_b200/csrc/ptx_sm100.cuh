@@ -1,6 +1,7 @@
-// Thin inline-PTX wrappers for the sm_100a features the grouped GEMMs use: mbarriers with
-// bounded waits, TMA tensor loads, bulk copies, and the tcgen05 tensor-core family
-// (TMEM allocation, smem->TMEM copies, block-scaled and bf16 MMAs, TMEM loads).
+// Thin inline-PTX wrappers for the sm_100a features the grouped GEMMs and the quantisers use:
+// mbarriers with bounded waits, TMA tensor loads (tiled and gather4), 256-bit global stores, and
+// the tcgen05 tensor-core family (TMEM allocation, smem->TMEM copies, block-scaled and bf16 MMAs,
+// TMEM loads).
 // Syntax follows the PTX ISA 8.6+ definitions of these instructions.
 #pragma once
 #include <cstdint>
@@ -100,13 +101,6 @@ __device__ __forceinline__ void tma_gather4(void* smem_dst, const void* tmap, in
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
       : "memory");
 }
-// Plain bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(smem_dst)),
-               "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
 
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
@@ -205,18 +199,6 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t M, uint32_t N, uint32
          | (1u << 23)          // scale type E8M0
          | ((M >> 4) << 24)    // M / 16
          | ((sfa_id & 3u) << 29);
-}
-
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
-
-__device__ __forceinline__ bool elect_one() {
-  uint32_t pred = 0;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "elect.sync _|p, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(pred));
-  return pred != 0;
 }
 
 }  // namespace ptx
