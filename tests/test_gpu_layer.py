@@ -214,3 +214,22 @@ def test_scattered_expert_weights_match_stacked(precision):
         res.append([t.float().cpu() if t.dtype == torch.bfloat16 else t.cpu() for t in (y, dx, dw1, dw2, dp)])
     for name, a, b in zip(("y", "dx", "dw_gate_up", "dw_down", "d_topk_prob"), *res):
         assert torch.equal(a, b), name
+
+
+@pytest.mark.parametrize("T", [1, 3])
+@pytest.mark.parametrize("precision", ["mxfp8", "bf16"])
+def test_few_tokens_forward_backward(T, precision):
+    """A handful of tokens: every expert tile is almost all padding rows (gathered as zeros), and
+    most experts receive nothing (zero weight gradients)."""
+    cfg = workloads.scaled_config(workloads.CONFIGS["tiny_bf16"], precision=precision, T=T, backward=True)
+    g = _run(cfg, precision)
+    ref = _oracle(g["inp"], precision)
+    assert rel_err(bf16_np(g["y"]), ref["y"]) <= TOL[precision]
+    assert rel_err(bf16_np(g["dx"]), ref["dx"]) <= TOL[precision]
+    assert rel_err(bf16_np(g["dw1"]), ref["dw_gate_up"]) <= TOL[precision]
+    assert rel_err(bf16_np(g["dw2"]), ref["dw_down"]) <= TOL[precision]
+    assert rel_err(g["dp"].cpu().numpy(), ref["d_topk_prob"]) <= TOL[precision]
+    used = set(np.asarray(g["inp"]["topk_idx"]).reshape(-1).tolist())
+    for e in range(cfg.E):
+        if e not in used:
+            assert not bf16_np(g["dw1"][e]).any() and not bf16_np(g["dw2"][e]).any()
