@@ -1,0 +1,31 @@
+"""The benchmark's accounting (host logic, no GPU): the algorithmic work it divides by.
+
+The six GEMMs' FLOPs must add up to the step's FLOPs the headline metric uses (18 Tk d f), and
+the weight quantisers' bytes are one bf16 read plus row-wise and column-wise codes with their
+scale bytes.
+"""
+import bench
+from mxfp8_quantize_b200 import workloads
+
+GEMMS = ["gemm_gate_up_swiglu", "gemm_down", "gemm_dgrad_down_dswiglu", "gemm_wgrad_down", "gemm_dgrad_gate_up",
+         "gemm_wgrad_gate_up"]
+
+
+def test_gemm_flops_add_up_to_the_step():
+    for name in ("mixtral_mxfp8", "mixtral_bf16", "longseq_mxfp8", "small_mxfp8"):
+        cfg = workloads.CONFIGS[name]
+        kinds = [bench.kernel_work(cfg, g) for g in GEMMS]
+        assert all(kind == "tensor" for kind, _ in kinds)
+        total = sum(w for _, w in kinds)
+        assert total == 18.0 * cfg.Tk * cfg.d * cfg.f
+        assert abs(total - cfg.flops_fwd_bwd()) <= 1e-9 * total
+
+
+def test_weight_quantiser_bytes():
+    cfg = workloads.CONFIGS["mixtral_mxfp8"]
+    kind, b = bench.kernel_work(cfg, "quantize_w_gate_up")
+    n = cfg.E * 2 * cfg.f * cfg.d
+    assert kind == "hbm" and b == n * 2 + 2 * (n + n / 32)   # bf16 in; two code copies + scales out
+    assert abs(b - 3.82e9) < 0.01e9
+    kind, b = bench.kernel_work(workloads.CONFIGS["mixtral_bf16"], "transpose_w_down")
+    assert kind == "hbm" and b == cfg.E * cfg.d * cfg.f * 4  # bf16 in, bf16 transposed out
