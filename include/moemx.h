@@ -80,6 +80,17 @@ moe_status_t moe_get_status(moe_ctx_t ctx, void* stream);
  * NULL to switch off.  The buffers must outlive every call that runs while set. */
 moe_status_t moe_ctx_set_debug_dump(moe_ctx_t ctx, float* a_f32, float* dh_f32);
 
+/* Test hook for the bounded in-kernel waits (tests only).  With ``stall`` non-zero, every CTA of
+ * the persistent kernels (the grouped GEMMs and the TMA-fed quantiser) makes one extra wait on a
+ * word of the context's status block that nothing ever sets, bounded by ``limit_cycles`` SM clock
+ * cycles (1 .. about 2e9): the GEMM producer after it has issued the first stages of its first tile
+ * (operand loads and MMAs in flight), the quantiser with its first source tiles in flight.  The
+ * wait expires as any wait would: the CTA raises its abort flag, every role stops, the copies and
+ * MMAs already issued are waited for (full-length bounded waits), TMEM is freed, and the call's
+ * moe_get_status returns MOE_ERR_TIMEOUT.  Outputs of calls made while it is set are undefined.
+ * stall = 0 switches it off; the context stays usable. */
+moe_status_t moe_ctx_set_test_stall(moe_ctx_t ctx, int stall, int64_t limit_cycles);
+
 const char* moe_status_string(moe_status_t s);
 
 /* Launch hook (profiling).  When set, the fused-layer and codec entry points call
@@ -151,6 +162,8 @@ moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, 
 /* Combine rows back to tokens: y[t] = bf16( sum_{j<k} w_j * fp32(y_perm[src_to_sorted[t*k+j]]) )
  * summed in fp32 in order j = 0..k-1, with w_j = probs[t][j] (fp32 products) or 1 if probs is
  * NULL (the fused layer applies the probability inside ScaledSwiGLU, so it combines with NULL).
+ * An entry of src_to_sorted equal to -1 (a slot moe_permute rejected for its expert index) is
+ * skipped; every other entry must be a row of y_perm.
  * y_perm bf16 [capacity, d]; y bf16 [T, d]; d % 8 == 0. */
 moe_status_t moe_unpermute(moe_ctx_t ctx, const void* y_perm, const int32_t* src_to_sorted, const float* probs,
                            int64_t T, int k, int64_t d, void* y, void* stream);
@@ -212,14 +225,30 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
  *  - Every call uses the same array, so calls that overlap on the GPU (different streams, or
  *    different host threads) race and must be serialised by the caller.  Nothing in the array
  *    needs to start at zero: each call writes every scratch byte it later reads.
- *  - device_status: optional device int; kernels OR MOE_ERR_DEVICE-type findings into it as bit 1
- *    (bad expert index / split_sizes mismatch) and bit 2 (a bounded wait expired).  NULL drops them.
+ *  - device_status: optional device int the kernels OR their findings into: the value 1 (bit 0)
+ *    for a bad expert index or a split_sizes mismatch, the value 2 (bit 1) for a bounded wait that
+ *    expired.  The caller zeroes it and reads it after synchronising.  NULL drops the findings.
  * Arguments and layouts are those of moe_grouped_mlp_fwd. */
 #define MOE_NOALLOC_SCRATCH_BYTES (64u << 20)
 moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx, const float* topk_prob,
                                          const int32_t* split_sizes, const void* const* w_gate_up,
                                          const void* const* w_down, int64_t T, int64_t d, int64_t f, int E, int k,
                                          moe_precision_t prec, void* y, int* device_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Tensor-core peak loop (measurement; the denominator of the GEMMs' roofline fractions).  The
+ * MXFP8 GEMMs run on Blackwell's block-scaled tensor-core instructions (ai4snews, paragraph 2);
+ * this measures what those instructions deliver on this GPU with nothing else in the way.
+ * Enqueues one kernel: one CTA per SM, each issuing ``iters`` groups of four tcgen05 MMAs of
+ * M = 128, N = 256 (K = 32 E4M3 with E8M0 scales per MMA for MXFP8, kind::mxf8f6f4; K = 16 bf16
+ * for BF16, kind::f16) on operands resident in shared memory, into one TMEM accumulator.  It
+ * reads and writes no global memory except the context's status word.  ``scale_refresh``
+ * (MXFP8 only) also copies the scale tiles shared memory -> TMEM before every group, as the
+ * grouped GEMM mainloop does per 128-wide K step.  The caller times it (CUDA events on
+ * ``stream``); moe_tensor_peak_flops gives the FLOPs of one launch (0 on bad arguments). */
+moe_status_t moe_tensor_peak_loop(moe_ctx_t ctx, moe_precision_t prec, int64_t iters, int scale_refresh,
+                                  void* stream);
+double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters);
 
 /* Inspection hook (tests): address of a named intermediate inside a saved buffer (which = 0),
  * a forward workspace (which = 1) or a backward workspace (which = 2) laid out for these

@@ -29,7 +29,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "unsupported", 4: "cuda
 EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_get_status", "moe_ctx_set_debug_dump", "moe_status_string",
            "mxfp8_quantize", "mxfp8_dequantize", "moe_capacity_rows", "moe_permute", "moe_unpermute",
            "moe_saved_size", "moe_fwd_workspace_size", "moe_bwd_workspace_size", "moe_grouped_mlp_fwd",
-           "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook", "moe_grouped_mlp_fwd_noalloc"]
+           "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook", "moe_grouped_mlp_fwd_noalloc",
+           "moe_ctx_set_test_stall", "moe_tensor_peak_loop", "moe_tensor_peak_flops"]
 
 LAUNCH_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
@@ -59,6 +60,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ctx_destroy": (c_int, [c_vp]),
         "moe_get_status": (c_int, [c_vp, c_vp]),
         "moe_ctx_set_debug_dump": (c_int, [c_vp, c_vp, c_vp]),
+        "moe_ctx_set_test_stall": (c_int, [c_vp, c_int, c_i64]),
+        "moe_tensor_peak_loop": (c_int, [c_vp, c_int, c_i64, c_int, c_vp]),
+        "moe_tensor_peak_flops": (ctypes.c_double, [c_vp, c_int, c_i64]),
         "moe_status_string": (ctypes.c_char_p, [c_int]),
         "mxfp8_quantize": (c_int, [c_vp, c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp, c_vp, c_vp, c_vp]),
         "mxfp8_dequantize": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_int, c_vp, c_vp]),
@@ -125,6 +129,12 @@ def get_status(device: int = 0):
 def set_debug_dump(device: int, a_f32: Optional[torch.Tensor], dh_f32: Optional[torch.Tensor]):
     L = load_library()
     _check("moe_ctx_set_debug_dump", L.moe_ctx_set_debug_dump(context(device), _ptr(a_f32), _ptr(dh_f32)))
+
+
+def set_test_stall(device: int, stall: bool, limit_cycles: int = 0):
+    """Test hook for the bounded in-kernel waits (see moe_ctx_set_test_stall in moemx.h)."""
+    L = load_library()
+    _check("moe_ctx_set_test_stall", L.moe_ctx_set_test_stall(context(device), int(stall), int(limit_cycles)))
 
 
 _hooks = {}
@@ -215,6 +225,15 @@ def moe_unpermute(y_perm: torch.Tensor, src_to_sorted: torch.Tensor, T: int, k: 
     _check("moe_unpermute", L.moe_unpermute(context(dev), y_perm.data_ptr(), src_to_sorted.data_ptr(), _ptr(probs),
                                             T, k, d, y.data_ptr(), _stream(dev)))
     return y
+
+
+def tensor_peak_loop(device: int, precision: str, iters: int, scale_refresh: bool = False) -> float:
+    """Enqueue the tensor-core peak loop on the current stream of ``device``; returns its FLOPs."""
+    L = load_library()
+    ctx = context(device)
+    _check("moe_tensor_peak_loop", L.moe_tensor_peak_loop(ctx, PRECISIONS[precision], int(iters), int(scale_refresh),
+                                                          _stream(device)))
+    return float(L.moe_tensor_peak_flops(ctx, PRECISIONS[precision], int(iters)))
 
 
 Weights = Union[torch.Tensor, Sequence[torch.Tensor]]

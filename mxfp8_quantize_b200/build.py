@@ -9,7 +9,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoemx.so")
-SOURCES = ["api.cu", "codec.cu", "gemm.cu"]
+SOURCES = ["api.cu", "codec.cu", "gemm.cu", "peak.cu"]
 
 
 def nvcc_path() -> str:

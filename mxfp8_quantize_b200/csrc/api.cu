@@ -21,6 +21,8 @@ struct moe_ctx_s {
   float* dbg_dh;
   moe_launch_hook_t hook;
   void* hook_user;
+  int stall;                // test hook for the bounded waits (moe_ctx_set_test_stall)
+  long long stall_limit;
 };
 
 namespace {
@@ -346,10 +348,18 @@ int64_t uniform_stride(const void* const* p, int E, int64_t min_bytes) {
   return s;
 }
 
+// Word of the context's status block that nothing ever writes (zeroed at creation): the flag the
+// test hook's waits can only give up on.
+constexpr int kNeverSetWord = 32;
+
 QuantArgs quant_args(moe_ctx_t ctx) {
   QuantArgs a;
   std::memset(&a, 0, sizeof(a));
   a.status = ctx->d_status;
+  if (ctx->stall) {
+    a.stall_flag = ctx->d_status + kNeverSetWord;
+    a.stall_limit = ctx->stall_limit;
+  }
   return a;
 }
 
@@ -357,6 +367,10 @@ GemmArgs gemm_args(moe_ctx_t ctx) {
   GemmArgs g;
   std::memset(&g, 0, sizeof(g));
   g.status = ctx->d_status;
+  if (ctx->stall) {
+    g.stall_flag = ctx->d_status + kNeverSetWord;
+    g.stall_limit = ctx->stall_limit;
+  }
   return g;
 }
 
@@ -394,6 +408,8 @@ moe_status_t moe_ctx_create(moe_ctx_t* out, int device) {
   c->dbg_a = c->dbg_dh = nullptr;
   c->hook = nullptr;
   c->hook_user = nullptr;
+  c->stall = 0;
+  c->stall_limit = 0;
   if (cudaMalloc(&c->d_status, 256) != cudaSuccess) {
     delete c;
     return MOE_ERR_CUDA;
@@ -426,6 +442,13 @@ moe_status_t moe_ctx_set_launch_hook(moe_ctx_t ctx, moe_launch_hook_t hook, void
   if (!ctx) return MOE_ERR_INVALID_ARG;
   ctx->hook = hook;
   ctx->hook_user = user;
+  return MOE_OK;
+}
+
+moe_status_t moe_ctx_set_test_stall(moe_ctx_t ctx, int stall, int64_t limit_cycles) {
+  if (!ctx || (stall && (limit_cycles <= 0 || limit_cycles > kWaitLimitCycles))) return MOE_ERR_INVALID_ARG;
+  ctx->stall = stall ? 1 : 0;
+  ctx->stall_limit = stall ? limit_cycles : 0;
   return MOE_OK;
 }
 
@@ -961,6 +984,21 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   return MOE_OK;
 }
 
+moe_status_t moe_tensor_peak_loop(moe_ctx_t ctx, moe_precision_t prec, int64_t iters, int scale_refresh,
+                                  void* stream) {
+  if (!ctx || iters <= 0 || (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8)) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->device);
+  MOE_LAUNCH(ctx, "tensor_peak_loop", stream,
+             launch_tensor_peak(prec == MOE_PREC_MXFP8, iters, scale_refresh ? 1 : 0, ctx->num_sms, ctx->d_status,
+                                static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters) {
+  if (!ctx || iters <= 0) return 0.0;
+  return tensor_peak_flops(prec == MOE_PREC_MXFP8, ctx->num_sms, iters);
+}
+
 void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
                          int which, void* base, const char* name) {
   if (!base || !name || check_dims(T, d, f, E, k) != MOE_OK) return nullptr;
@@ -1072,6 +1110,8 @@ moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx,
   c.dbg_a = c.dbg_dh = nullptr;
   c.hook = nullptr;
   c.hook_user = nullptr;
+  c.stall = 0;
+  c.stall_limit = 0;
   // the scratch base is 256-aligned; the workspace carving aligns to 1 KiB inside the size bound
   return moe_grouped_mlp_fwd(&c, x, topk_idx, topk_prob, split_sizes, w_gate_up, w_down, T, d, f, E, k, prec, 0, y,
                              nullptr, 0, nd.scratch, MOE_NOALLOC_SCRATCH_BYTES, stream);

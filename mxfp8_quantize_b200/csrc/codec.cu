@@ -427,8 +427,13 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
     const int ob = it % QW_NOUT;
     if (tid == 0) {
       // this tile's source has landed; the stores that last read output buffer ``ob`` are done
-      volatile int* never = &stop;
-      if (!ptx::mbar_wait(&full[slot], static_cast<uint32_t>((it / QW_NIN) & 1), never, kWaitLimitCycles)) {
+      volatile int* flag = &stop;  // raised by an expired wait
+      bool ok = true;
+      if (a.stall_flag && it == 0)  // test hook: a wait that can only expire, first source tiles in flight
+        ok = ptx::wait_flag(a.stall_flag, flag, a.stall_limit);
+      if (ok && !ptx::mbar_wait(&full[slot], static_cast<uint32_t>((it / QW_NIN) & 1), flag, kWaitLimitCycles))
+        ok = false;
+      if (!ok) {
         stop = 1;
         if (a.status) atomicOr(a.status, kStatusTimeout);
       }
@@ -587,7 +592,8 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
 }
 
 // ------------------------------------------------------------------------------------------
-// Combine: y[t] = bf16(sum_j w_j * fp32(rows[row(t, j)])), j ascending, fp32 products and sums.
+// Combine: y[t] = bf16(sum_j w_j * fp32(rows[row(t, j)])), j ascending, fp32 products and sums;
+// slots whose row is -1 are skipped.
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 unpermute_kernel(const bf16* __restrict__ rows, const int32_t* __restrict__ src_to_sorted,
@@ -603,6 +609,7 @@ unpermute_kernel(const bf16* __restrict__ rows, const int32_t* __restrict__ src_
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
     for (int j = 0; j < k; ++j) {
       const int64_t r = src_to_sorted[t * k + j];
+      if (r < 0) continue;  // a slot the routing rejected (expert index out of range): contributes nothing
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(rows + r * d + c));
       const bf16* h = reinterpret_cast<const bf16*>(&v);
       if (probs) {
@@ -631,7 +638,8 @@ __global__ void dprob_reduce_kernel(const float* __restrict__ part, int n_parts,
        s += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = src_to_sorted[s];
     float acc = 0.f;
-    for (int n = 0; n < n_parts; ++n) acc = __fadd_rn(acc, part[n * part_stride + r]);
+    if (r >= 0)  // a rejected slot has no row and gets a zero gradient
+      for (int n = 0; n < n_parts; ++n) acc = __fadd_rn(acc, part[n * part_stride + r]);
     d_prob[s] = acc;
   }
 }

@@ -44,6 +44,8 @@ struct QuantArgs {
   int tma_gather;
   int64_t src_rows;
   int* status;                 // device status word (a bounded wait that expired)
+  const int* stall_flag;       // test hook: waited on once per CTA (TMA-fed kernel) for stall_limit cycles
+  long long stall_limit;
 };
 
 cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk, int E, int capacity,

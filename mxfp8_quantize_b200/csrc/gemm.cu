@@ -24,7 +24,8 @@
 // the fused ScaledSwiGLU / dSwiGLU epilogues release it after their last TMEM load and requantise
 // column-wise through a small padded smem transpose (one scale per column per lane).  Row-strided
 // outputs leave in 256-bit stores (a whole 32-byte sector per lane).
-// Every wait is bounded: on expiry the kernel records MOE_ERR_TIMEOUT and all roles stop.
+// Every wait is bounded: on expiry the kernel records MOE_ERR_TIMEOUT and all roles stop; copies
+// and MMAs already issued are waited for before TMEM is freed.
 #include <cuda_fp8.h>
 
 #include "gemm.cuh"
@@ -299,12 +300,17 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     uint32_t issued_mask = 0, last_parity = 0;
     uint32_t h_count = 0;
     bool h_issued = false;
+    bool stalled = false;
     const uint32_t tx = S::A_BYTES + S::B_BYTES + (MX ? 512 + S::SFB_BYTES : 0);
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
       const int bk = MX ? 128 : 64;
       for (int kb = 0; kb < tl.nk; ++kb) {
+        if (g.stall_flag && !stalled && kb == min(2, tl.nk - 1)) {  // test hook: a wait that can only expire
+          stalled = true;
+          if (!ptx::wait_flag(g.stall_flag, abort_flag, g.stall_limit)) break;
+        }
         if (!ptx::mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, lim)) break;
         uint8_t* st = smem + stage * S::STAGE_BYTES;
         ptx::mbar_arrive_expect_tx(&s.full[stage], tx);

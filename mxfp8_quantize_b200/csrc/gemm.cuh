@@ -55,6 +55,10 @@ struct GemmArgs {
   int64_t sfb_kb4;
   int64_t sfb_expert_rows;  // rows of B per expert (M-grouped), for the scale tile index
   int* status;
+  // test hook: a device flag nothing sets; when non-null the producer of each CTA waits on it once,
+  // for at most stall_limit cycles, after issuing the first stages of its first tile
+  const int* stall_flag;
+  long long stall_limit;
   EpiArgs epi;
 };
 
@@ -65,5 +69,11 @@ int gemm_dswiglu_parts();
 
 // Launch one grouped GEMM.  ``mx``: MXFP8 (kind::mxf8f6f4) or BF16 (kind::f16).
 cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st);
+
+// Tensor-core peak loop (peak.cu): one CTA per SM issuing iters x 4 MMAs of 128 x 256 on operands
+// resident in shared memory; its FLOPs per launch.
+cudaError_t launch_tensor_peak(bool mx, long long iters, int scale_refresh, int num_sms, int* status,
+                               cudaStream_t st);
+double tensor_peak_flops(bool mx, int num_sms, long long iters);
 
 }  // namespace moemx

@@ -61,6 +61,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait for a global flag to become non-zero (used by the test hook that exercises the
+// abort paths with a flag nothing sets).  Returns false on abort or after ``limit_cycles`` SM
+// clocks; on expiry it raises the abort flag itself, like mbar_wait.
+__device__ __forceinline__ bool wait_flag(const int* flag, volatile int* abort_flag, long long limit_cycles) {
+  const long long t0 = clock64();
+  while (true) {
+    if (*reinterpret_cast<const volatile int*>(flag) != 0) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit_cycles) {
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
 // ---------------------------------------------------------------- wide global stores
 // 32 bytes (lo then hi) to a 32-byte aligned global address with one 256-bit store: a warp of
 // these writes whole 32-byte sectors even when every lane targets a different row.

@@ -1,4 +1,7 @@
 """Helpers for the GPU parity tests (test-side code; shares nothing with the CUDA library)."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -32,3 +35,24 @@ def rel_err(got, ref) -> float:
 
 def bf16_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy()
+
+
+def p99_rel_err(got, ref) -> float:
+    """99th percentile of the element-wise relative error |got - ref| / max(|ref|, 1e-3 max|ref|)
+    (the floor keeps elements near zero from dominating)."""
+    got = np.asarray(got, dtype=np.float64).reshape(-1)
+    ref = np.asarray(ref, dtype=np.float64).reshape(-1)
+    den = np.maximum(np.abs(ref), 1e-3 * max(float(np.max(np.abs(ref))), 1e-300))
+    return float(np.percentile(np.abs(got - ref) / den, 99))
+
+
+def parity(name: str, got, ref, tol: float) -> float:
+    """Assert max|got - ref| / max|ref| <= tol and return it; the figure and the element-wise p99
+    relative error are appended as a JSON line to the file named by MOE_PARITY_REPORT, if set."""
+    err = rel_err(got, ref)
+    path = os.environ.get("MOE_PARITY_REPORT")
+    if path:
+        with open(path, "a") as fh:
+            fh.write(json.dumps({"case": name, "max_rel": err, "p99_rel": p99_rel_err(got, ref), "tol": tol}) + "\n")
+    assert err <= tol, f"{name}: {err:.3g} > {tol}"
+    return err

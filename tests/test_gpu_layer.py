@@ -12,7 +12,7 @@ import torch
 
 from oracle import moe as omoe
 from oracle import mx, routing
-from tests.gpu_util import bf16_np, has_b200, rel_err, unswizzle_scales
+from tests.gpu_util import bf16_np, has_b200, parity, rel_err, unswizzle_scales
 from mxfp8_quantize_b200 import workloads
 
 pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not has_b200(), reason="needs a B200")]
@@ -163,8 +163,8 @@ def test_small_intermediates_within_tolerance(small):
     E, f, cap = cfg.E, cfg.f, g["cap"]
     Tp = int(ref["st"]["route"]["poffsets"][E])
     h = _view(g["saved"].buf, 0, "h", cfg, precision, True, cap * 2 * f, torch.bfloat16).float().cpu().numpy()
-    assert rel_err(h.reshape(cap, 2 * f)[:Tp], ref["st"]["h"]) <= TOL[precision]
-    assert rel_err(g["dump_a"].cpu().numpy()[:Tp], ref["st"]["a"]) <= TOL[precision]
+    parity(f"small_{precision}.h", h.reshape(cap, 2 * f)[:Tp], ref["st"]["h"], TOL[precision])
+    parity(f"small_{precision}.a", g["dump_a"].cpu().numpy()[:Tp], ref["st"]["a"], TOL[precision])
 
 
 @pytest.mark.parametrize("name", ["y", "dx", "dw1", "dw2", "dp"])
@@ -173,8 +173,7 @@ def test_small_outputs_within_tolerance(small, name):
     refname = {"y": "y", "dx": "dx", "dw1": "dw_gate_up", "dw2": "dw_down", "dp": "d_topk_prob"}[name]
     got = g[name]
     got = got.float().cpu().numpy() if got.dtype == torch.bfloat16 else got.cpu().numpy()
-    err = rel_err(got, ref[refname])
-    assert err <= TOL[precision], f"{name}: {err}"
+    parity(f"small_{precision}.{name}", got, ref[refname], TOL[precision])
     if name == "dw1":
         assert np.all(got[7] == 0)   # expert 7 receives no tokens
     if name == "dw2":
