@@ -189,7 +189,7 @@ def tensor_peak(moe, device: int, precision: str, target_ms: float = 100.0, scal
     moe.tensor_peak_loop(device, precision, iters, scale_refresh)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    iters = max(100, int(iters * 10.0 / max(e0.elapsed_time(e1), 1e-3)))
+    iters = min(1000000, max(100, int(iters * 10.0 / max(e0.elapsed_time(e1), 1e-3))))
     n = max(1, int(round(target_ms / 10.0)))
     flops = 0.0
     e0.record(stream)

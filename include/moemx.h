@@ -245,7 +245,8 @@ moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx,
  * reads and writes no global memory except the context's status word.  ``scale_refresh``
  * (MXFP8 only) also copies the scale tiles shared memory -> TMEM before every group, as the
  * grouped GEMM mainloop does per 128-wide K step.  The caller times it (CUDA events on
- * ``stream``); moe_tensor_peak_flops gives the FLOPs of one launch (0 on bad arguments). */
+ * ``stream``); moe_tensor_peak_flops gives the FLOPs of one launch (0 on bad arguments).
+ * 1 <= iters <= 1000000 (MOE_ERR_INVALID_ARG otherwise). */
 moe_status_t moe_tensor_peak_loop(moe_ctx_t ctx, moe_precision_t prec, int64_t iters, int scale_refresh,
                                   void* stream);
 double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters);

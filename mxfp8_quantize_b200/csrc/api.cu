@@ -986,7 +986,8 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
 
 moe_status_t moe_tensor_peak_loop(moe_ctx_t ctx, moe_precision_t prec, int64_t iters, int scale_refresh,
                                   void* stream) {
-  if (!ctx || iters <= 0 || (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8)) return MOE_ERR_INVALID_ARG;
+  if (!ctx || iters <= 0 || iters > 1000000 || (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8))
+    return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->device);
   MOE_LAUNCH(ctx, "tensor_peak_loop", stream,
              launch_tensor_peak(prec == MOE_PREC_MXFP8, iters, scale_refresh ? 1 : 0, ctx->num_sms, ctx->d_status,

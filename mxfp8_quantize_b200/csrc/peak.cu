@@ -17,7 +17,11 @@ namespace {
 constexpr int PK_A = 128 * 128;   // A tile: 128 rows x 128 bytes, 128B-swizzled
 constexpr int PK_B = 256 * 128;   // B tile: 256 rows x 128 bytes
 constexpr int PK_SF = 512 + 1024; // scale tiles of A (128 rows) and B (256 rows)
-constexpr int PK_SMEM = PK_A + PK_B + PK_SF + 1024;
+// Dynamic shared memory requested per CTA: more than half of an SM's, so that exactly one CTA
+// runs per SM (only the first PK_A + PK_B + PK_SF bytes are used).
+constexpr int PK_SMEM = 120 * 1024;
+static_assert(PK_A + PK_B + PK_SF + 1024 <= PK_SMEM, "peak loop shared memory");
+constexpr long long PK_MAX_ITERS = 1000000;  // one launch stays well inside the bounded final wait
 constexpr uint32_t PK_SF_COL = 256;  // TMEM columns after the 128 x 256 fp32 accumulator
 }  // namespace
 
@@ -102,6 +106,7 @@ double tensor_peak_flops(bool mx, int num_sms, long long iters) {
 
 cudaError_t launch_tensor_peak(bool mx, long long iters, int scale_refresh, int num_sms, int* status,
                                cudaStream_t st) {
+  if (iters > PK_MAX_ITERS) return cudaErrorInvalidValue;
   auto kern = mx ? tensor_peak_kernel<true> : tensor_peak_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PK_SMEM);
   if (e != cudaSuccess) return e;
