@@ -67,18 +67,19 @@ def silu(g):
     return g * sigmoid(g)
 
 
-def gemm(A, B, precision: str) -> np.ndarray:
+def gemm(A, B, precision: str, scale_rule: str = "ceil") -> np.ndarray:
     """C = A @ B for A [M, K], B [K, N] with operands in the given precision.
 
-    mxfp8: A quantised in blocks of 32 along its axis 1 (K), B along its axis 0 (K).
+    mxfp8: A quantised in blocks of 32 along its axis 1 (K), B along its axis 0 (K), with the
+           shared-exponent rule ``scale_rule`` (oracle.mx).
     bf16:  both operands rounded to bf16.   fp64: used as given.
     The product is formed in fp64 (callers round it).
     """
     A = np.asarray(A, dtype=np.float64)
     B = np.asarray(B, dtype=np.float64)
     if precision == "mxfp8":
-        A = mx.fake_quant(A, axis=1)
-        B = mx.fake_quant(B, axis=0)
+        A = mx.fake_quant(A, axis=1, rule=scale_rule)
+        B = mx.fake_quant(B, axis=0, rule=scale_rule)
     elif precision == "bf16":
         A = bf16_round(A).astype(np.float64)
         B = bf16_round(B).astype(np.float64)
@@ -108,8 +109,9 @@ def _combine(rows_perm, src_to_sorted, T, k, precision):
     return bf16_round(acc)
 
 
-def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: int = 128):
-    """Returns (y [T, d], state) with the intermediates the backward needs."""
+def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: int = 128, scale_rule: str = "ceil"):
+    """Returns (y [T, d], state) with the intermediates the backward needs.  ``scale_rule`` is the
+    MXFP8 shared-exponent rule of every quantisation (forward and backward)."""
     x = np.asarray(x, dtype=np.float64)
     T, d = x.shape
     E, two_f, _ = w_gate_up.shape
@@ -138,14 +140,14 @@ def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: in
         pe[valid] = pflat[slots[valid]]
         W1 = np.asarray(w_gate_up[e], dtype=np.float64)
         W2 = np.asarray(w_down[e], dtype=np.float64)
-        h = gemm(Xe, W1.T, precision)
+        h = gemm(Xe, W1.T, precision, scale_rule)
         if precision != "fp64":
             h = f32(h)
         g, u = h[:, :f].astype(np.float64), h[:, f:].astype(np.float64)
         a = silu(g) * u * pe[:, None]
         if precision != "fp64":
             a = f32(a)
-        ye = gemm(a, W2.T, precision)
+        ye = gemm(a, W2.T, precision, scale_rule)
         y_perm[lo:hi] = _round_out(ye, precision)
         h_all[lo:hi] = h
         a_all[lo:hi] = a
@@ -153,7 +155,7 @@ def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: in
         p_perm[lo:hi] = pe
     y = _combine(y_perm, r["src_to_sorted"], T, k, precision)
     state = dict(route=r, x_perm=x_perm, p_perm=p_perm, h=h_all, a=a_all, y_perm=y_perm,
-                 T=T, d=d, f=f, E=E, k=k, precision=precision)
+                 T=T, d=d, f=f, E=E, k=k, precision=precision, scale_rule=scale_rule)
     return y, state
 
 
@@ -165,6 +167,7 @@ def backward(dy, state, w_gate_up, w_down):
     dW of an expert that received no tokens is exactly zero.
     """
     precision = state["precision"]
+    rule = state.get("scale_rule", "ceil")
     T, d, f, E, k = (state[n] for n in ("T", "d", "f", "E", "k"))
     r = state["route"]
     poff, split, s2src = r["poffsets"], r["split_sizes"], r["sorted_to_src"]
@@ -195,11 +198,11 @@ def backward(dy, state, w_gate_up, w_down):
         W2 = np.asarray(w_down[e], dtype=np.float64)
 
         # down projection: dgrad (K = d) and wgrad (K = tokens)
-        da = gemm(dYe, W2, precision)
+        da = gemm(dYe, W2, precision, rule)
         if precision != "fp64":
             da = f32(da)
         da = da.astype(np.float64)
-        dW2[e] = _round_out(gemm(dYe.T, a, precision), precision)
+        dW2[e] = _round_out(gemm(dYe.T, a, precision, rule), precision)
 
         # ScaledSwiGLU gradient
         s = sigmoid(g)
@@ -213,8 +216,8 @@ def backward(dy, state, w_gate_up, w_down):
             dp = f32(dp)
 
         # gate_up projection: dgrad (K = 2f) and wgrad (K = tokens)
-        dx_perm[lo:hi] = _round_out(gemm(dh, W1, precision), precision)
-        dW1[e] = _round_out(gemm(np.asarray(dh, dtype=np.float64).T, Xe, precision), precision)
+        dx_perm[lo:hi] = _round_out(gemm(dh, W1, precision, rule), precision)
+        dW1[e] = _round_out(gemm(np.asarray(dh, dtype=np.float64).T, Xe, precision, rule), precision)
         dp_perm[lo:hi] = dp
         dh_perm[lo:hi] = dh
 

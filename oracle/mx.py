@@ -13,6 +13,9 @@ protect the numerical range.  Everything else is a reading:
 * shared scale: the power of two 2**e with the smallest integer e such that
   amax <= 448 * 2**e (no element can saturate), clamped to [-127, 127] and
   stored as the biased byte e + 127.  An all-zero block gets byte 0.
+  Variant ("floor", the OCP MX v1.0 rule): e = floor(log2(amax)) - 8, 8 being
+  the exponent of E4M3's largest power of two; the block maximum then scales
+  into [256, 512) and elements above 448 saturate to 448.
 * a block holding a NaN gets scale byte 0xFF and NaN codes (outside the
   tested contract; inputs are finite).
 
@@ -70,23 +73,35 @@ def e4m3_decode(codes) -> np.ndarray:
     return _TABLE[np.asarray(codes, dtype=np.uint8)]
 
 
-def e8m0_exponent(amax) -> np.ndarray:
-    """Smallest integer e with amax <= 448 * 2**e, clamped to [-127, 127] (int64)."""
+SCALE_RULES = ("ceil", "floor")
+
+
+def e8m0_exponent(amax, rule: str = "ceil") -> np.ndarray:
+    """Shared exponent of a block with maximum magnitude ``amax`` (int64, clamped to [-127, 127]).
+
+    ceil:  the smallest integer e with amax <= 448 * 2**e.
+    floor: floor(log2(amax)) - 8 (OCP MX v1.0).
+    """
+    if rule not in SCALE_RULES:
+        raise ValueError(rule)
     amax = np.asarray(amax, dtype=np.float64)
     safe = np.where((amax > 0) & np.isfinite(amax), amax, 1.0)
     _, ex = np.frexp(safe)                  # safe = m * 2**ex, m in [0.5, 1)
     guess = ex.astype(np.int64) - 1 - 8     # floor(log2(amax)) - 8
-    e = guess + 2
-    # walk down while the next smaller exponent still covers amax (checks are exact in fp64)
-    for _ in range(4):
-        smaller_ok = safe <= E4M3_MAX * np.exp2((e - 1).astype(np.float64))
-        e = np.where(smaller_ok, e - 1, e)
+    if rule == "floor":
+        e = guess
+    else:
+        e = guess + 2
+        # walk down while the next smaller exponent still covers amax (checks are exact in fp64)
+        for _ in range(4):
+            smaller_ok = safe <= E4M3_MAX * np.exp2((e - 1).astype(np.float64))
+            e = np.where(smaller_ok, e - 1, e)
     e = np.where(amax > 0, e, -127)
     return np.clip(e, -127, 127)
 
 
-def quantize_blocks(x: np.ndarray):
-    """Quantise along the last axis in blocks of 32.
+def quantize_blocks(x: np.ndarray, rule: str = "ceil"):
+    """Quantise along the last axis in blocks of 32, with the shared-exponent ``rule``.
 
     Returns (codes uint8, same shape as x; scale bytes uint8, shape [..., n/32]).
     """
@@ -97,7 +112,7 @@ def quantize_blocks(x: np.ndarray):
     xb = x.reshape(x.shape[:-1] + (n // BLOCK, BLOCK))
     amax = np.max(np.abs(xb), axis=-1)
     has_nan = np.isnan(xb).any(axis=-1)
-    e = e8m0_exponent(np.where(has_nan, 0.0, amax))
+    e = e8m0_exponent(np.where(has_nan, 0.0, amax), rule)
     scaled = xb * np.exp2(-e.astype(np.float64))[..., None]
     codes = e4m3_encode(scaled)
     codes = np.where(has_nan[..., None], np.where(np.signbit(xb), 0xFF, 0x7F), codes).astype(np.uint8)
@@ -115,18 +130,18 @@ def dequantize_blocks(codes: np.ndarray, sbytes: np.ndarray) -> np.ndarray:
     return (vals * scale[..., None]).reshape(codes.shape)
 
 
-def quantize_rowwise(x: np.ndarray):
+def quantize_rowwise(x: np.ndarray, rule: str = "ceil"):
     """Blocks of 32 along each row (the last axis): codes [R, C], scales [R, C/32]."""
-    return quantize_blocks(x)
+    return quantize_blocks(x, rule)
 
 
-def quantize_colwise_t(x: np.ndarray):
+def quantize_colwise_t(x: np.ndarray, rule: str = "ceil"):
     """Blocks of 32 down each column, returned transposed: codes [C, R], scales [C, R/32]."""
-    return quantize_blocks(np.swapaxes(np.asarray(x), -1, -2))
+    return quantize_blocks(np.swapaxes(np.asarray(x), -1, -2), rule)
 
 
-def fake_quant(x: np.ndarray, axis: int) -> np.ndarray:
+def fake_quant(x: np.ndarray, axis: int, rule: str = "ceil") -> np.ndarray:
     """Dequantised value of x after MXFP8 quantisation with blocks of 32 along ``axis``."""
     xm = np.moveaxis(np.asarray(x, dtype=np.float64), axis, -1)
-    c, s = quantize_blocks(xm)
+    c, s = quantize_blocks(xm, rule)
     return np.moveaxis(dequantize_blocks(c, s), -1, axis)

@@ -39,24 +39,27 @@ MAX_DIFF_FRACTION = 1e-4
 
 
 # ---------------------------------------------------------------- independent numerics
-def _e8m0_exponent(amax: torch.Tensor) -> torch.Tensor:
+def _e8m0_exponent(amax: torch.Tensor, rule: str = "ceil") -> torch.Tensor:
     m, x = torch.frexp(amax)                 # amax = m * 2**x, 0.5 <= m < 1 (m = 0 for amax = 0)
-    e = x.to(torch.int64) - 9 + (m > 0.875).to(torch.int64)
+    e = x.to(torch.int64) - 9                # floor(log2 amax) - 8: the OCP rule
+    if rule == "ceil":                       # one more when amax > 448 * 2**(x - 9), i.e. m > 0.875
+        e = e + (m > 0.875).to(torch.int64)
     e = torch.where(amax > 0, e, torch.full_like(e, -127))
     return e.clamp(-127, 127)
 
 
-def _fq_mx(v: torch.Tensor, axis: int) -> torch.Tensor:
-    """MXFP8 fake quantisation with blocks of 32 along ``axis`` (zero-padded to a multiple of 32)."""
+def _fq_mx(v: torch.Tensor, axis: int, rule: str = "ceil") -> torch.Tensor:
+    """MXFP8 fake quantisation with blocks of 32 along ``axis`` (zero-padded to a multiple of 32);
+    elements beyond 448 after scaling (floor rule only) saturate."""
     vm = v.movedim(axis, -1)
     n = vm.shape[-1]
     pad = (-n) % 32
     if pad:
         vm = torch.nn.functional.pad(vm, (0, pad))
     blocks = vm.reshape(*vm.shape[:-1], -1, 32)
-    e = _e8m0_exponent(blocks.abs().amax(dim=-1, keepdim=True))
+    e = _e8m0_exponent(blocks.abs().amax(dim=-1, keepdim=True), rule)
     scale = torch.ldexp(torch.ones_like(blocks[..., :1]), e)
-    q = (blocks / scale).to(torch.float8_e4m3fn).to(torch.float64) * scale
+    q = (blocks / scale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).to(torch.float64) * scale
     q = q.reshape(vm.shape)[..., :n]
     return q.movedim(-1, axis)
 
@@ -73,7 +76,9 @@ ROUND = {"f32": _to_f32, "bf16": _to_bf16}
 
 
 def _operand(v, axis, mode):
-    return _fq_mx(v, axis) if mode == "mxfp8" else _to_bf16(v)
+    if mode == "bf16":
+        return _to_bf16(v)
+    return _fq_mx(v, axis, "floor" if mode == "mxfp8-floor" else "ceil")
 
 
 class _QuantLinear(torch.autograd.Function):
@@ -189,12 +194,16 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("mode", ["mxfp8", "bf16"])
+@pytest.mark.parametrize("mode", ["mxfp8", "bf16", "mxfp8-floor"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"T{s['T']}_E{s['E']}_k{s['k']}_{s['routing']}")
 def test_quantised_backward_matches_straight_through_autograd(shape, mode):
+    """mxfp8-floor: the oracle's OCP floor shared-exponent variant, in every quantisation."""
     inp = _inputs(**shape)
     args = [inp[n] for n in ("x", "topk_idx", "topk_prob", "w_gate_up", "w_down")]
-    y, st = moe.forward(*args, mode)
+    if mode == "mxfp8-floor":
+        y, st = moe.forward(*args, "mxfp8", scale_rule="floor")
+    else:
+        y, st = moe.forward(*args, mode)
     got = moe.backward(inp["dy"], st, inp["w_gate_up"], inp["w_down"])
     got["y"] = y
     ref = _reference(*args, inp["dy"], mode)
@@ -221,6 +230,8 @@ def test_fake_quantiser_matches_the_scale_rule_on_hand_values():
     assert int(_e8m0_exponent(torch.tensor([1.875], dtype=torch.float64))) == -7
     assert int(_e8m0_exponent(torch.tensor([448.0], dtype=torch.float64))) == 0
     assert int(_e8m0_exponent(torch.tensor([450.0], dtype=torch.float64))) == 1
+    assert int(_e8m0_exponent(torch.tensor([1.875], dtype=torch.float64), "floor")) == -8
+    assert int(_e8m0_exponent(torch.tensor([450.0], dtype=torch.float64), "floor")) == 0
     w = torch.zeros(1, 32, dtype=torch.float64)
     w[0, 0] = 450.0
     w[0, 1] = 1.0

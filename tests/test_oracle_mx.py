@@ -14,6 +14,7 @@ import torch
 from oracle import mx
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_hand_vectors.txt")
+GOLDEN_FLOOR = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_hand_vectors_floor.txt")
 
 
 def _parse_list(s):
@@ -28,9 +29,9 @@ def _parse_list(s):
     return out
 
 
-def _golden_cases():
+def _golden_cases(path=GOLDEN):
     cases = []
-    for line in open(GOLDEN):
+    for line in open(path):
         line = line.strip()
         if not line or line.startswith("#"):
             continue
@@ -48,6 +49,43 @@ def test_hand_vectors(case):
     q, s = mx.quantize_blocks(v[None, :])
     assert int(s[0, 0]) == sbyte
     assert [int(c) for c in q[0, :len(codes)]] == codes
+
+
+@pytest.mark.parametrize("case", _golden_cases(GOLDEN_FLOOR), ids=lambda c: c[0])
+def test_hand_vectors_floor_rule(case):
+    name, v, sbyte, codes = case
+    q, s = mx.quantize_blocks(v[None, :], rule="floor")
+    assert int(s[0, 0]) == sbyte
+    assert [int(c) for c in q[0, :len(codes)]] == codes
+
+
+def test_floor_rule_brute_force_and_relation_to_round_up():
+    """floor: 2**(e + 8) <= amax < 2**(e + 9) exactly; the round-up exponent is the floor one or one
+    more (one more exactly when amax > 448 * 2**e_floor, the blocks the floor rule saturates)."""
+    rng = np.random.default_rng(12)
+    amax = np.abs(rng.standard_normal(5000)) * 2.0 ** rng.integers(-60, 60, 5000)
+    amax = np.concatenate([amax, 448.0 * 2.0 ** np.arange(-20, 20), 2.0 ** np.arange(-20, 20),
+                           np.nextafter(2.0 ** np.arange(-20, 20), 0)])
+    ef = mx.e8m0_exponent(amax, "floor")
+    ec = mx.e8m0_exponent(amax, "ceil")
+    for a, f_, c_ in zip(amax, ef, ec):
+        assert 2.0 ** (f_ + 8) <= a < 2.0 ** (f_ + 9)
+        assert c_ == f_ + (1 if a > 448.0 * 2.0 ** f_ else 0)
+
+
+def test_floor_rule_top_binade_and_saturation():
+    rng = np.random.default_rng(13)
+    x = _bf16_block(rng, 512, spread=30)
+    q, s = mx.quantize_blocks(x, rule="floor")
+    scaled = np.abs(x) * 2.0 ** -(s[:, 0].astype(np.float64) - 127)[:, None]
+    assert np.all(np.max(scaled, axis=1) >= 256) and np.all(np.max(scaled, axis=1) < 512)
+    top = q[np.arange(x.shape[0]), np.argmax(np.abs(x), axis=1)] & 0x7F
+    assert np.all((top >= 0x78) & (top <= 0x7E))
+    sat = np.max(scaled, axis=1) > 448
+    assert sat.any() and np.all(top[sat] == 0x7E)
+    # torch's float8 conversion of the scaled, clamped values gives the same codes
+    ref = torch.from_numpy(np.clip(x * 2.0 ** -(s[:, :1].astype(np.float64) - 127), -448, 448).astype(np.float32))
+    assert np.array_equal(ref.to(torch.float8_e4m3fn).view(torch.uint8).numpy(), q)
 
 
 def test_decode_table_matches_torch_float8():
