@@ -58,6 +58,15 @@ typedef enum { MOE_PREC_BF16 = 0, MOE_PREC_MXFP8 = 1 } moe_precision_t;
 #define MXFP8_ROWWISE 1        /* blocks of 32 along each row                              */
 #define MXFP8_COLWISE_T 2      /* blocks of 32 down each column, written transposed        */
 #define MXFP8_SF_MMA_LAYOUT 4  /* scales in the tensor-core tile layout instead of row-major */
+#define MXFP8_FLAG_SCALE_FLOOR 8 /* shared exponent by the OCP floor rule instead of round-up   */
+
+/* Shared-exponent rules (moe_ctx_set_scale_rule).  ROUND_UP: e = the smallest integer with
+ * amax <= 448 * 2^e, so no element saturates (this library's default reading of "a scaling factor
+ * per block of 32 values" that protects the range: sitech.ge "Memory and quantization overhead").
+ * FLOOR: e = floor(log2 amax) - 8, the OCP MX v1.0 rule; the block maximum scales into [256, 512)
+ * and elements above 448 saturate to 448. */
+#define MXFP8_SCALE_ROUND_UP 0
+#define MXFP8_SCALE_FLOOR 1
 
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK 8
@@ -79,6 +88,11 @@ moe_status_t moe_get_status(moe_ctx_t ctx, void* stream);
  * epilogue writes the fp32 dh = [dg, du] it quantises into ``dh_f32`` [capacity, 2f]; pass
  * NULL to switch off.  The buffers must outlive every call that runs while set. */
 moe_status_t moe_ctx_set_debug_dump(moe_ctx_t ctx, float* a_f32, float* dh_f32);
+
+/* Shared-exponent rule of every MXFP8 quantisation the fused layer makes with this context
+ * (weights, x, dy and the epilogue requantisations of a and dh): MXFP8_SCALE_ROUND_UP (default) or
+ * MXFP8_SCALE_FLOOR.  Calls already enqueued are not affected. */
+moe_status_t moe_ctx_set_scale_rule(moe_ctx_t ctx, int rule);
 
 /* Test hook for the bounded in-kernel waits (tests only).  With ``stall`` non-zero, every CTA of
  * the persistent kernels (the grouped GEMMs and the TMA-fed quantiser) makes one extra wait on a
@@ -105,7 +119,8 @@ moe_status_t moe_ctx_set_launch_hook(moe_ctx_t ctx, moe_launch_hook_t hook, void
  * block of 32 consecutive values; ai4snews paragraph 2).
  *
  * x        bf16 [batch, rows, cols]
- * flags    MXFP8_ROWWISE and/or MXFP8_COLWISE_T, optionally | MXFP8_SF_MMA_LAYOUT
+ * flags    MXFP8_ROWWISE and/or MXFP8_COLWISE_T, optionally | MXFP8_SF_MMA_LAYOUT and
+ *          | MXFP8_FLAG_SCALE_FLOOR (the OCP floor rule below instead of round-up)
  * q_row    uint8 [batch, rows, cols] E4M3 codes, blocks of 32 along each row   (ROWWISE)
  * s_row    uint8 E8M0 bytes, [batch, rows, cols/32] row-major, or the MMA layout (ROWWISE)
  * q_colT   uint8 [batch, cols, rows] codes of blocks of 32 down each column, transposed
@@ -114,6 +129,8 @@ moe_status_t moe_ctx_set_launch_hook(moe_ctx_t ctx, moe_launch_hook_t hook, void
  * Scale rule: e = the smallest integer with amax <= 448 * 2^e over the block (clamped to
  * [-127, 127]), byte = e + 127; element code = E4M3(v * 2^-e) rounded to nearest-even,
  * saturating (no element can exceed 448 under this rule); all-zero blocks get byte 0.
+ * With MXFP8_FLAG_SCALE_FLOOR: e = floor(log2 amax) - 8, elements above 448 after scaling
+ * saturate to 448.
  *
  * MMA layout (MXFP8_SF_MMA_LAYOUT): a scale matrix S[R][KB] (R rows, KB = K/32 blocks) is
  * stored as 512-byte tiles, tile (R/128 index rb, KB/4 index kb4) at byte (rb*KB/4 + kb4)*512,

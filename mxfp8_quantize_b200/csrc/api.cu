@@ -21,6 +21,7 @@ struct moe_ctx_s {
   float* dbg_dh;
   moe_launch_hook_t hook;
   void* hook_user;
+  int scale_floor;          // MXFP8 shared-exponent rule of the fused layer (moe_ctx_set_scale_rule)
   int stall;                // test hook for the bounded waits (moe_ctx_set_test_stall)
   long long stall_limit;
 };
@@ -356,6 +357,7 @@ QuantArgs quant_args(moe_ctx_t ctx) {
   QuantArgs a;
   std::memset(&a, 0, sizeof(a));
   a.status = ctx->d_status;
+  a.scale_floor = ctx->scale_floor;
   if (ctx->stall) {
     a.stall_flag = ctx->d_status + kNeverSetWord;
     a.stall_limit = ctx->stall_limit;
@@ -367,6 +369,7 @@ GemmArgs gemm_args(moe_ctx_t ctx) {
   GemmArgs g;
   std::memset(&g, 0, sizeof(g));
   g.status = ctx->d_status;
+  g.epi.scale_floor = ctx->scale_floor;
   if (ctx->stall) {
     g.stall_flag = ctx->d_status + kNeverSetWord;
     g.stall_limit = ctx->stall_limit;
@@ -408,6 +411,7 @@ moe_status_t moe_ctx_create(moe_ctx_t* out, int device) {
   c->dbg_a = c->dbg_dh = nullptr;
   c->hook = nullptr;
   c->hook_user = nullptr;
+  c->scale_floor = 0;
   c->stall = 0;
   c->stall_limit = 0;
   if (cudaMalloc(&c->d_status, 256) != cudaSuccess) {
@@ -452,6 +456,12 @@ moe_status_t moe_ctx_set_test_stall(moe_ctx_t ctx, int stall, int64_t limit_cycl
   return MOE_OK;
 }
 
+moe_status_t moe_ctx_set_scale_rule(moe_ctx_t ctx, int rule) {
+  if (!ctx || (rule != MXFP8_SCALE_ROUND_UP && rule != MXFP8_SCALE_FLOOR)) return MOE_ERR_INVALID_ARG;
+  ctx->scale_floor = rule == MXFP8_SCALE_FLOOR ? 1 : 0;
+  return MOE_OK;
+}
+
 moe_status_t moe_get_status(moe_ctx_t ctx, void* stream) {
   if (!ctx) return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->device);
@@ -474,7 +484,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
                             uint8_t* q_row, uint8_t* s_row, uint8_t* q_colT, uint8_t* s_colT, void* stream) {
   if (!ctx || !x || batch <= 0 || rows <= 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
   const bool row = flags & MXFP8_ROWWISE, col = flags & MXFP8_COLWISE_T, mma = flags & MXFP8_SF_MMA_LAYOUT;
-  if ((flags & ~7) || !(row || col)) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~15) || !(row || col)) return MOE_ERR_INVALID_ARG;
   if (row && (!q_row || !s_row)) return MOE_ERR_INVALID_ARG;
   if (col && (!q_colT || !s_colT)) return MOE_ERR_INVALID_ARG;
   if (cols % 32) return MOE_ERR_SHAPE;
@@ -494,6 +504,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
   a.do_row = row;
   a.do_col = col;
   a.sf_mma = mma;
+  a.scale_floor = (flags & MXFP8_FLAG_SCALE_FLOOR) ? 1 : 0;
   a.q_row = q_row;
   a.s_row = s_row;
   a.q_colT = q_colT;
@@ -1111,6 +1122,7 @@ moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx,
   c.dbg_a = c.dbg_dh = nullptr;
   c.hook = nullptr;
   c.hook_user = nullptr;
+  c.scale_floor = 0;
   c.stall = 0;
   c.stall_limit = 0;
   // the scratch base is 256-aligned; the workspace carving aligns to 1 KiB inside the size bound

@@ -146,7 +146,8 @@ __device__ __forceinline__ void column_pass(const QuantArgs& a, const uint32_t* 
     m2 = absmax_bf16x2(m2, wv[i]);
   }
   if (a.mx) {
-    const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16), sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u);
+    const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16, a.scale_floor);
+    const uint32_t sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u, a.scale_floor);
     const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
     uint32_t q0[8], q1[8];
 #pragma unroll
@@ -266,7 +267,7 @@ quant_tile_kernel(const __grid_constant__ QuantArgs a) {
       uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w)));
       m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      const uint32_t sb = e8m0_from_amax_bits(m);
+      const uint32_t sb = e8m0_from_amax_bits(m, a.scale_floor);
       const float inv = e8m0_inv_scale(sb);
       if (valid) {
         const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
@@ -483,7 +484,7 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        const uint32_t sb = e8m0_from_amax_bits(m);
+        const uint32_t sb = e8m0_from_amax_bits(m, a.scale_floor);
         const float inv = e8m0_inv_scale(sb);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t q[4];
@@ -506,7 +507,8 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
           wv[i] = words[(rb * 32 + i) * 64 + p];
           m2 = absmax_bf16x2(m2, wv[i]);
         }
-        const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16), sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u);
+        const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16, a.scale_floor);
+        const uint32_t sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u, a.scale_floor);
         const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
         uint32_t q0[8], q1[8];
   #pragma unroll

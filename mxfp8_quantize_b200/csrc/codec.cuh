@@ -22,6 +22,7 @@ struct QuantArgs {
   int mx;                      // 1: MXFP8 codes + scales; 0: bf16 copies
   int64_t gate_up_half;        // >0: row-wise outputs in 256-row groups [128 rows < half | 128 rows >= half]
   int do_row, do_col, sf_mma;
+  int scale_floor;             // MXFP8 shared exponent: 0 round-up rule, 1 OCP floor rule
   uint8_t* q_row;
   uint8_t* s_row;
   uint8_t* q_colT;

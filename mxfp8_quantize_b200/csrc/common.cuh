@@ -29,10 +29,12 @@ __host__ __device__ inline int64_t sf_mma_offset(int64_t r, int64_t kb, int64_t 
 
 // E8M0 exponent e = the smallest integer with amax <= 448 * 2^e, from the fp32 bits of amax
 // (amax = (1 + m/2^23) * 2^E: e = E - 8, plus one when the mantissa exceeds 0.75), clamped to
-// [-127, 127].  Returns the biased byte e + 127.
-__device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t abits) {
+// [-127, 127].  With ``floor_rule`` (the OCP MX v1.0 variant) e = E - 8 = floor(log2 amax) - 8,
+// and the block's largest elements may exceed 448 after scaling (the conversion saturates them).
+// Returns the biased byte e + 127.
+__device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t abits, int floor_rule = 0) {
   const int E = static_cast<int>((abits >> 23) & 0xFFu) - 127;
-  int e = E - 8 + (((abits & 0x7FFFFFu) > 0x600000u) ? 1 : 0);
+  int e = E - 8 + ((!floor_rule && (abits & 0x7FFFFFu) > 0x600000u) ? 1 : 0);
   e = e < -127 ? -127 : (e > 127 ? 127 : e);
   return static_cast<uint32_t>(e + 127);
 }

@@ -83,8 +83,9 @@ struct SharedState {
   uint32_t tmem_base;
   int abort_flag;
   int total_tiles;
-  int tile_prefix[MOE_MAX_EXPERTS + 1];
-  int poff[MOE_MAX_EXPERTS + 1];
+  int tile_prefix[MOE_MAX_EXPERTS + 1];  // tiles before the i-th expert of ``order``
+  int poff[MOE_MAX_EXPERTS + 1];         // padded row offsets, by expert id
+  int order[MOE_MAX_EXPERTS];            // expert ids in tile-list order
 };
 
 struct Tile {
@@ -93,14 +94,22 @@ struct Tile {
   int k0;     // first K coordinate (K-grouped: the expert's first token row)
 };
 
+// The i-th tile of this CTA: tiles are dealt out in rounds of gridDim.x, in boustrophedon order
+// (even rounds to CTAs 0, 1, ..., odd rounds in reverse), so that with the tile list sorted from
+// the most to the least work every CTA gets a similar total.
+__device__ __forceinline__ int tile_of(int i) {
+  const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+  return i * G + ((i & 1) ? G - 1 - b : b);
+}
+
 __device__ __forceinline__ void decode_tile(int t, const SharedState& s, const GemmArgs& g, bool mx, Tile& o) {
-  int lo = 0, hi = g.E;  // largest e with prefix[e] <= t (experts without tiles are skipped)
+  int lo = 0, hi = g.E;  // largest i with prefix[i] <= t (experts without tiles are skipped)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (s.tile_prefix[mid] <= t) lo = mid; else hi = mid;
   }
-  const int e = lo;
-  const int local = t - s.tile_prefix[e];
+  const int e = s.order[lo];
+  const int local = t - s.tile_prefix[lo];
   const int P = s.poff[e + 1] - s.poff[e];
   const int bk = mx ? 128 : 64;  // K elements per stage (128 bytes)
   o.e = e;
@@ -147,11 +156,11 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
 
 // MXFP8 of 32 values with the scale of their own amax: 32 codes stored at q (32-byte aligned);
 // returns the E8M0 byte.
-__device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q) {
+__device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q, int floor_rule) {
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) m = max(m, __float_as_uint(v[i]) & 0x7FFFFFFFu);
-  const uint32_t sb = e8m0_from_amax_bits(m);
+  const uint32_t sb = e8m0_from_amax_bits(m, floor_rule);
   const float inv = e8m0_inv_scale(sb);
   uint32_t w[8];
 #pragma unroll
@@ -187,14 +196,14 @@ __device__ __forceinline__ void column_passes(const float* v, float* stage, F&& 
 // tile-layout scale matrix with sf_KB columns.
 template <int P>
 __device__ __forceinline__ void colwise_mx(const float* v, float* stage, uint8_t* colT, int64_t ld, uint8_t* sf,
-                                           int64_t sf_row0, int64_t sf_kb, int64_t sf_KB) {
+                                           int64_t sf_row0, int64_t sf_kb, int64_t sf_KB, int floor_rule) {
   column_passes<P>(v, stage, [&](int h, int cl, int rg, const float* col) {
     uint32_t m = 0;
 #pragma unroll
     for (int i = 0; i < P; ++i) m = max(m, __float_as_uint(col[i]) & 0x7FFFFFFFu);
 #pragma unroll
     for (int s = P; s < 32; s <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, s));
-    const uint32_t sb = e8m0_from_amax_bits(m);
+    const uint32_t sb = e8m0_from_amax_bits(m, floor_rule);
     const float inv = e8m0_inv_scale(sb);
     uint32_t w[P / 4];
 #pragma unroll
@@ -248,14 +257,27 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
 
   // ---- set-up: tile prefix over experts, barriers, TMEM
   if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int e = 0; e < g.E; ++e) {
-      const int p0 = g.poffsets[e], p1 = g.poffsets[e + 1];
-      s.poff[e] = p0;
-      s.tile_prefix[e] = acc;
-      acc += g.kgrouped ? g.m_tiles * g.n_tiles : ((p1 - p0) / BM) * g.n_tiles;
+    for (int e = 0; e <= g.E; ++e) s.poff[e] = g.poffsets[e];
+    // tile list order: experts in id order, except for K-grouped GEMMs, whose tiles cost in
+    // proportion to the expert's token count: there the experts go from most to fewest tokens
+    // (stable insertion sort), so that skewed routing does not leave a tail of long tiles
+    for (int i = 0; i < g.E; ++i) {
+      int j = i;
+      if (g.kgrouped) {
+        const int P = s.poff[i + 1] - s.poff[i];
+        while (j > 0 && s.poff[s.order[j - 1] + 1] - s.poff[s.order[j - 1]] < P) {
+          s.order[j] = s.order[j - 1];
+          --j;
+        }
+      }
+      s.order[j] = i;
     }
-    s.poff[g.E] = g.poffsets[g.E];
+    int acc = 0;
+    for (int i = 0; i < g.E; ++i) {
+      const int e = s.order[i];
+      s.tile_prefix[i] = acc;
+      acc += g.kgrouped ? g.m_tiles * g.n_tiles : ((s.poff[e + 1] - s.poff[e]) / BM) * g.n_tiles;
+    }
     s.tile_prefix[g.E] = acc;
     s.total_tiles = acc;
     s.abort_flag = 0;
@@ -302,7 +324,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     bool h_issued = false;
     bool stalled = false;
     const uint32_t tx = S::A_BYTES + S::B_BYTES + (MX ? 512 + S::SFB_BYTES : 0);
-    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+    for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
       const int bk = MX ? 128 : 64;
@@ -379,7 +401,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     const uint64_t bdesc0 = ptx::smem_desc(smem0 + S::OFF_B, 16, 1024, ptx::kSwizzle128B);
     const uint64_t sfadesc0 = ptx::smem_desc(smem0 + S::OFF_SFA, 0, 128, ptx::kSwizzleNone);
     const uint64_t sfbdesc0 = ptx::smem_desc(smem0 + S::OFF_SFB, 0, 128, ptx::kSwizzleNone);
-    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+    for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
       if (tl.nk == 0) continue;
@@ -438,7 +460,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
                                                 (warp - 4) * S::STAGING_PER_WARP);
     const EpiArgs& ep = g.epi;
     int local = 0;
-    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+    for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
       const int64_t row_w = tl.a_row + 32 * q;  // first row of this warp
@@ -523,11 +545,11 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             for (int i = 0; i < 8; ++i) dd[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
           }
           if (MX) {
-            const uint32_t sb = quant32_store(gv, ep.q_row + row * f + j);
+            const uint32_t sb = quant32_store(gv, ep.q_row + row * f + j, ep.scale_floor);
             ep.s_row[sf_mma_offset(row, j / 32, f / 32)] = static_cast<uint8_t>(sb);
             if (ep.q_colT)
               colwise_mx<S::PASS>(gv, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
-                                  ep.cap / 32);
+                                  ep.cap / 32, ep.scale_floor);
           } else {
             bf16* dst = ep.o_row + row * f + j;
 #pragma unroll
@@ -620,14 +642,14 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             }
           }
           if (MX) {
-            uint32_t sb = quant32_store(dg, ep.q_row + row * f2 + j);
+            uint32_t sb = quant32_store(dg, ep.q_row + row * f2 + j, ep.scale_floor);
             ep.s_row[sf_mma_offset(row, j / 32, f2 / 32)] = static_cast<uint8_t>(sb);
-            sb = quant32_store(du, ep.q_row + row * f2 + f + j);
+            sb = quant32_store(du, ep.q_row + row * f2 + f + j, ep.scale_floor);
             ep.s_row[sf_mma_offset(row, (f + j) / 32, f2 / 32)] = static_cast<uint8_t>(sb);
             colwise_mx<S::PASS>(dg, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
-                                ep.cap / 32);
+                                ep.cap / 32, ep.scale_floor);
             colwise_mx<S::PASS>(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j,
-                                row_w / 32, ep.cap / 32);
+                                row_w / 32, ep.cap / 32, ep.scale_floor);
           } else {
             bf16* d0 = ep.o_row + row * f2 + j;
             bf16* d1 = d0 + f;

@@ -29,6 +29,7 @@ struct EpiArgs {
   bf16* o_row;        // BF16 path equivalents
   bf16* o_colT;
   float* dump;        // debug: fp32 values before quantisation
+  int scale_floor;    // MXFP8 shared exponent of the requantisations: 0 round-up rule, 1 OCP floor rule
   float* dp_part;     // DSWIGLU: [parts * n_tiles, cap] partial sums of the probability gradient
 };
 

@@ -142,3 +142,37 @@ def test_unpermute_bit_exact(with_probs):
                           probs=prob.cuda() if with_probs else None)
     ref = oracle_unpermute(rows.float().numpy(), r["src_to_sorted"], T, k, probs=prob.numpy() if with_probs else None)
     assert np.array_equal(y.float().cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("rows,cols,colwise,mma", [
+    (64, 128, True, False), (100, 96, False, False), (128, 256, True, True), (4096, 512, True, True),
+])
+def test_quantize_floor_rule_bit_exact(rows, cols, colwise, mma):
+    """The OCP floor shared-exponent variant (MXFP8_FLAG_SCALE_FLOOR), both quantiser kernels."""
+    x = _spread_bf16(rows, cols, seed=7 * rows + cols)
+    out = moe.mxfp8_quantize(x.cuda(), rowwise=True, colwise=colwise, mma_layout=mma, scale_rule="floor")
+    torch.cuda.synchronize()
+    xf = x.float().numpy()
+    q, s = mx.quantize_rowwise(xf, rule="floor")
+    assert np.array_equal(out["q_row"].cpu().numpy(), q)
+    s_gpu = out["s_row"].cpu().numpy()
+    assert np.array_equal(unswizzle_scales(s_gpu, rows, cols // 32) if mma else s_gpu, s)
+    if colwise:
+        qc, sc = mx.quantize_colwise_t(xf, rule="floor")
+        assert np.array_equal(out["q_colT"].cpu().numpy(), qc)
+        sc_gpu = out["s_colT"].cpu().numpy()
+        assert np.array_equal(unswizzle_scales(sc_gpu, cols, rows // 32) if mma else sc_gpu, sc)
+
+
+def test_golden_floor_vectors_on_gpu():
+    from tests.test_oracle_mx import GOLDEN_FLOOR, _golden_cases
+    cases = _golden_cases(GOLDEN_FLOOR)
+    x = np.zeros((len(cases), 32))
+    for i, (_, v, _, _) in enumerate(cases):
+        x[i] = v
+    out = moe.mxfp8_quantize(torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).cuda(), rowwise=True,
+                             scale_rule="floor")
+    q, s = out["q_row"].cpu().numpy(), out["s_row"].cpu().numpy()
+    for i, (name, v, sbyte, codes) in enumerate(cases):
+        assert int(s[i, 0]) == sbyte, name
+        assert [int(c) for c in q[i, :len(codes)]] == codes, name

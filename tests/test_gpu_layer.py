@@ -232,3 +232,38 @@ def test_few_tokens_forward_backward(T, precision):
     for e in range(cfg.E):
         if e not in used:
             assert not bf16_np(g["dw1"][e]).any() and not bf16_np(g["dw2"][e]).any()
+
+
+def test_floor_scale_rule_layer():
+    """The fused layer with the OCP floor shared-exponent rule in every quantisation
+    (moe_ctx_set_scale_rule): quantised operands and the epilogue requantisations bit-exact against
+    the oracle's floor-rule codec, outputs within tolerance of the oracle's floor-rule layer."""
+    precision = "mxfp8"
+    cfg = workloads.scaled_config(workloads.CONFIGS["small_mxfp8"], T=1024, seed=41)
+    moe.set_scale_rule(0, "floor")
+    try:
+        g = _run(cfg, precision)
+    finally:
+        moe.set_scale_rule(0, "ceil")
+    np_in = {n: (t.float().numpy() if t.dtype == torch.bfloat16 else t.numpy()) for n, t in g["inp"].items()}
+    y, st = omoe.forward(np_in["x"], np_in["topk_idx"], np_in["topk_prob"], np_in["w_gate_up"], np_in["w_down"],
+                         precision, scale_rule="floor")
+    gr = omoe.backward(np_in["dy"], st, np_in["w_gate_up"], np_in["w_down"])
+    E, d, f, cap = cfg.E, cfg.d, cfg.f, g["cap"]
+    Tp = int(st["route"]["poffsets"][E])
+    w2 = np_in["w_down"]
+    q = _view(g["ws"], 1, "w2_q", cfg, precision, True, E * d * f).cpu().numpy().reshape(E * d, f)
+    assert np.array_equal(q, mx.quantize_rowwise(w2.reshape(E * d, f), rule="floor")[0])
+    q = _view(g["ws"], 1, "x_q", cfg, precision, True, cap * d).cpu().numpy().reshape(cap, d)
+    assert np.array_equal(q[:Tp], mx.quantize_rowwise(st["x_perm"], rule="floor")[0])
+    a32 = g["dump_a"].cpu().numpy()[:Tp]
+    q = _view(g["ws"], 1, "a_q", cfg, precision, True, cap * f).cpu().numpy().reshape(cap, f)
+    assert np.array_equal(q[:Tp], mx.quantize_rowwise(a32, rule="floor")[0])
+    dh32 = g["dump_dh"].cpu().numpy()[:Tp]
+    q = _view(g["bws"], 2, "dhT_q", cfg, precision, True, 2 * f * cap).cpu().numpy().reshape(2 * f, cap)
+    assert np.array_equal(q[:, :Tp], mx.quantize_colwise_t(dh32, rule="floor")[0])
+    for name, ref in (("y", y), ("dx", gr["dx"]), ("dw1", gr["dw_gate_up"]), ("dw2", gr["dw_down"]),
+                      ("dp", gr["d_topk_prob"])):
+        got = g[name]
+        got = got.float().cpu().numpy() if got.dtype == torch.bfloat16 else got.cpu().numpy()
+        parity(f"small_floor_rule.{name}", got, ref, TOL[precision])
