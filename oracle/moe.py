@@ -31,7 +31,10 @@ Precision modes and the readings they encode:
   routing probability is applied once, inside ScaledSwiGLU, so the final
   combine is an unweighted sum.  Straight-through: gradients flow through the
   quantisers as identity; each backward GEMM quantises its own operands along
-  its own K (so dgrad uses the weights quantised down the columns).
+  its own K (so dgrad uses the weights quantised down the columns).  Variants:
+  the OCP floor shared-exponent rule (``scale_rule="floor"``) in every
+  quantisation, and E5M2 elements for the gradient operands dy and dh of the
+  backward GEMMs (``grad_format="e5m2"``; weights and activations stay E4M3).
 * "bf16": the same chain with bf16 GEMM operands (a, dh rounded to bf16) and
   fp32 products.
 * "fp64": no quantisation and no rounding anywhere (used to pin the algebra
@@ -67,18 +70,19 @@ def silu(g):
     return g * sigmoid(g)
 
 
-def gemm(A, B, precision: str, scale_rule: str = "ceil") -> np.ndarray:
+def gemm(A, B, precision: str, scale_rule: str = "ceil", a_fmt: str = "e4m3") -> np.ndarray:
     """C = A @ B for A [M, K], B [K, N] with operands in the given precision.
 
-    mxfp8: A quantised in blocks of 32 along its axis 1 (K), B along its axis 0 (K), with the
-           shared-exponent rule ``scale_rule`` (oracle.mx).
+    mxfp8: A quantised in blocks of 32 along its axis 1 (K) with elements ``a_fmt``, B along its
+           axis 0 (K) with E4M3 elements, both with the shared-exponent rule ``scale_rule``
+           (oracle.mx).
     bf16:  both operands rounded to bf16.   fp64: used as given.
     The product is formed in fp64 (callers round it).
     """
     A = np.asarray(A, dtype=np.float64)
     B = np.asarray(B, dtype=np.float64)
     if precision == "mxfp8":
-        A = mx.fake_quant(A, axis=1, rule=scale_rule)
+        A = mx.fake_quant(A, axis=1, rule=scale_rule, fmt=a_fmt)
         B = mx.fake_quant(B, axis=0, rule=scale_rule)
     elif precision == "bf16":
         A = bf16_round(A).astype(np.float64)
@@ -109,9 +113,11 @@ def _combine(rows_perm, src_to_sorted, T, k, precision):
     return bf16_round(acc)
 
 
-def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: int = 128, scale_rule: str = "ceil"):
+def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: int = 128, scale_rule: str = "ceil",
+            grad_format: str = "e4m3"):
     """Returns (y [T, d], state) with the intermediates the backward needs.  ``scale_rule`` is the
-    MXFP8 shared-exponent rule of every quantisation (forward and backward)."""
+    MXFP8 shared-exponent rule of every quantisation (forward and backward); ``grad_format`` the
+    element format of the gradient operands (dy, dh) of the four backward GEMMs."""
     x = np.asarray(x, dtype=np.float64)
     T, d = x.shape
     E, two_f, _ = w_gate_up.shape
@@ -155,7 +161,7 @@ def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: in
         p_perm[lo:hi] = pe
     y = _combine(y_perm, r["src_to_sorted"], T, k, precision)
     state = dict(route=r, x_perm=x_perm, p_perm=p_perm, h=h_all, a=a_all, y_perm=y_perm,
-                 T=T, d=d, f=f, E=E, k=k, precision=precision, scale_rule=scale_rule)
+                 T=T, d=d, f=f, E=E, k=k, precision=precision, scale_rule=scale_rule, grad_format=grad_format)
     return y, state
 
 
@@ -168,6 +174,7 @@ def backward(dy, state, w_gate_up, w_down):
     """
     precision = state["precision"]
     rule = state.get("scale_rule", "ceil")
+    gf = state.get("grad_format", "e4m3")   # element format of the gradient operand (A) of each GEMM
     T, d, f, E, k = (state[n] for n in ("T", "d", "f", "E", "k"))
     r = state["route"]
     poff, split, s2src = r["poffsets"], r["split_sizes"], r["sorted_to_src"]
@@ -198,11 +205,11 @@ def backward(dy, state, w_gate_up, w_down):
         W2 = np.asarray(w_down[e], dtype=np.float64)
 
         # down projection: dgrad (K = d) and wgrad (K = tokens)
-        da = gemm(dYe, W2, precision, rule)
+        da = gemm(dYe, W2, precision, rule, gf)
         if precision != "fp64":
             da = f32(da)
         da = da.astype(np.float64)
-        dW2[e] = _round_out(gemm(dYe.T, a, precision, rule), precision)
+        dW2[e] = _round_out(gemm(dYe.T, a, precision, rule, gf), precision)
 
         # ScaledSwiGLU gradient
         s = sigmoid(g)
@@ -216,8 +223,8 @@ def backward(dy, state, w_gate_up, w_down):
             dp = f32(dp)
 
         # gate_up projection: dgrad (K = 2f) and wgrad (K = tokens)
-        dx_perm[lo:hi] = _round_out(gemm(dh, W1, precision, rule), precision)
-        dW1[e] = _round_out(gemm(np.asarray(dh, dtype=np.float64).T, Xe, precision, rule), precision)
+        dx_perm[lo:hi] = _round_out(gemm(dh, W1, precision, rule, gf), precision)
+        dW1[e] = _round_out(gemm(np.asarray(dh, dtype=np.float64).T, Xe, precision, rule, gf), precision)
         dp_perm[lo:hi] = dp
         dh_perm[lo:hi] = dh
 

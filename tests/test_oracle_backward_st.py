@@ -48,6 +48,27 @@ def _e8m0_exponent(amax: torch.Tensor, rule: str = "ceil") -> torch.Tensor:
     return e.clamp(-127, 127)
 
 
+def _e8m0_exponent_e5m2(amax: torch.Tensor) -> torch.Tensor:
+    """E5M2 elements: the smallest e with amax <= 57344 * 2**e = 0.875 * 2**(16 + e)."""
+    m, x = torch.frexp(amax)
+    e = x.to(torch.int64) - 16 + (m > 0.875).to(torch.int64)
+    e = torch.where(amax > 0, e, torch.full_like(e, -127))
+    return e.clamp(-127, 127)
+
+
+def _fq_mx5(v: torch.Tensor, axis: int) -> torch.Tensor:
+    """MXFP8 fake quantisation with E5M2 elements (gradient operands), blocks of 32 along ``axis``."""
+    vm = v.movedim(axis, -1)
+    n = vm.shape[-1]
+    pad = (-n) % 32
+    if pad:
+        vm = torch.nn.functional.pad(vm, (0, pad))
+    blocks = vm.reshape(*vm.shape[:-1], -1, 32)
+    scale = torch.ldexp(torch.ones_like(blocks[..., :1]), _e8m0_exponent_e5m2(blocks.abs().amax(dim=-1, keepdim=True)))
+    q = (blocks / scale).clamp(-57344.0, 57344.0).to(torch.float8_e5m2).to(torch.float64) * scale
+    return q.reshape(vm.shape)[..., :n].movedim(-1, axis)
+
+
 def _fq_mx(v: torch.Tensor, axis: int, rule: str = "ceil") -> torch.Tensor:
     """MXFP8 fake quantisation with blocks of 32 along ``axis`` (zero-padded to a multiple of 32);
     elements beyond 448 after scaling (floor rule only) saturate."""
@@ -81,6 +102,11 @@ def _operand(v, axis, mode):
     return _fq_mx(v, axis, "floor" if mode == "mxfp8-floor" else "ceil")
 
 
+def _grad_operand(v, axis, mode):
+    """The gradient operand of a backward product (E5M2 elements in the gradient-format variant)."""
+    return _fq_mx5(v, axis) if mode == "mxfp8-e5m2grad" else _operand(v, axis, mode)
+
+
 class _QuantLinear(torch.autograd.Function):
     """C = A B^T with A [M, K], B [N, K].  Forward: both operands quantised along K.  Backward:
     dA = dC B with dC and B quantised along N; dB = dC^T A with dC and A quantised down the M
@@ -96,8 +122,8 @@ class _QuantLinear(torch.autograd.Function):
     def backward(ctx, dC):
         A, B = ctx.saved_tensors
         mode = ctx.mode
-        dA = _operand(dC, 1, mode) @ _operand(B, 0, mode)
-        dB = _operand(dC, 0, mode).T @ _operand(A, 0, mode)
+        dA = _grad_operand(dC, 1, mode) @ _operand(B, 0, mode)
+        dB = _grad_operand(dC, 0, mode).T @ _operand(A, 0, mode)
         return ROUND[ctx.da_round](dA), _to_bf16(dB), None, None, None
 
 
@@ -194,14 +220,17 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("mode", ["mxfp8", "bf16", "mxfp8-floor"])
+@pytest.mark.parametrize("mode", ["mxfp8", "bf16", "mxfp8-floor", "mxfp8-e5m2grad"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"T{s['T']}_E{s['E']}_k{s['k']}_{s['routing']}")
 def test_quantised_backward_matches_straight_through_autograd(shape, mode):
-    """mxfp8-floor: the oracle's OCP floor shared-exponent variant, in every quantisation."""
+    """mxfp8-floor: the oracle's OCP floor shared-exponent variant, in every quantisation;
+    mxfp8-e5m2grad: E5M2 elements for the gradient operand of every backward product."""
     inp = _inputs(**shape)
     args = [inp[n] for n in ("x", "topk_idx", "topk_prob", "w_gate_up", "w_down")]
     if mode == "mxfp8-floor":
         y, st = moe.forward(*args, "mxfp8", scale_rule="floor")
+    elif mode == "mxfp8-e5m2grad":
+        y, st = moe.forward(*args, "mxfp8", grad_format="e5m2")
     else:
         y, st = moe.forward(*args, mode)
     got = moe.backward(inp["dy"], st, inp["w_gate_up"], inp["w_down"])

@@ -15,6 +15,7 @@ from oracle import mx
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_hand_vectors.txt")
 GOLDEN_FLOOR = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_hand_vectors_floor.txt")
+GOLDEN_E5M2 = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_e5m2_hand_vectors.txt")
 
 
 def _parse_list(s):
@@ -222,3 +223,61 @@ def test_fake_quant_error_bound():
     e = mx.e8m0_exponent(amax[:, 0])[:, None].astype(np.float64)
     bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** (e - 10))
     assert np.all(err <= bound + 0.0)
+
+
+# ---------------------------------------------------------------- E5M2 elements (gradient variant)
+@pytest.mark.parametrize("case", _golden_cases(GOLDEN_E5M2), ids=lambda c: c[0])
+def test_hand_vectors_e5m2(case):
+    name, v, sbyte, codes = case
+    q, s = mx.quantize_blocks(v[None, :], fmt="e5m2")
+    assert int(s[0, 0]) == sbyte
+    assert [int(c) for c in q[0, :len(codes)]] == codes
+
+
+def test_e5m2_decode_table_matches_torch_float8():
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e5m2).to(torch.float64).numpy()
+    ours = mx.e5m2_decode_table()
+    assert np.array_equal(np.isnan(ref), np.isnan(ours)) and np.array_equal(np.isinf(ref), np.isinf(ours))
+    fin = np.isfinite(ref)
+    assert np.array_equal(ref[fin], ours[fin])
+    assert ours[0x7B] == 57344.0 and ours[0x01] == 2.0 ** -16
+
+
+def test_e5m2_encode_matches_torch_rne_in_range():
+    rng = np.random.default_rng(20)
+    pos = mx.e5m2_decode_table()[:0x7C]
+    mids = (pos[:-1] + pos[1:]) / 2
+    v = np.concatenate([pos, mids, -pos, -mids, rng.uniform(-57344, 57344, 20000),
+                        rng.standard_normal(20000) * 2.0 ** rng.integers(-20, 14, 20000)]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert np.array_equal(ref, mx.e5m2_encode(v))
+    assert mx.e5m2_encode(np.array([57344.0, 60000.0, 1e9, -1e9])).tolist() == [0x7B, 0x7B, 0x7B, 0xFB]
+
+
+@pytest.mark.parametrize("rule", ["ceil", "floor"])
+def test_e5m2_exponent_rules_brute_force(rule):
+    rng = np.random.default_rng(21)
+    amax = np.abs(rng.standard_normal(5000)) * 2.0 ** rng.integers(-60, 60, 5000)
+    amax = np.concatenate([amax, 57344.0 * 2.0 ** np.arange(-20, 20), 2.0 ** np.arange(-20, 20)])
+    e = mx.e8m0_exponent(amax, rule, "e5m2")
+    for a, ei in zip(amax, e):
+        if rule == "ceil":
+            assert 57344.0 * 2.0 ** (ei - 1) < a <= 57344.0 * 2.0 ** ei
+        else:
+            assert 2.0 ** (ei + 15) <= a < 2.0 ** (ei + 16)
+
+
+def test_e5m2_blocks_roundtrip_grid_values_and_never_saturate():
+    rng = np.random.default_rng(22)
+    table = mx.e5m2_decode_table()
+    codes = rng.integers(0, 0x7C, (64, 32)).astype(np.uint8)
+    codes[:, 0] = 0x7B                      # every block's amax is 57344 * 2**sb
+    codes |= (rng.integers(0, 2, codes.shape) * 0x80).astype(np.uint8)
+    sb = rng.integers(-20, 20, 64)
+    x = table[codes] * 2.0 ** sb[:, None]
+    q, s = mx.quantize_blocks(x, fmt="e5m2")
+    assert np.array_equal(q, codes) and np.array_equal(s[:, 0].astype(int), sb + 127)
+    assert np.array_equal(mx.dequantize_blocks(q, s, fmt="e5m2"), x)
+    y = _bf16_block(rng, 256, spread=30)
+    q, s = mx.quantize_blocks(y, fmt="e5m2")
+    assert not np.any((q & 0x7F) > 0x7B)    # no infinity or NaN code
