@@ -59,6 +59,11 @@ typedef enum { MOE_PREC_BF16 = 0, MOE_PREC_MXFP8 = 1 } moe_precision_t;
 #define MXFP8_COLWISE_T 2      /* blocks of 32 down each column, written transposed        */
 #define MXFP8_SF_MMA_LAYOUT 4  /* scales in the tensor-core tile layout instead of row-major */
 #define MXFP8_FLAG_SCALE_FLOOR 8 /* shared exponent by the OCP floor rule instead of round-up   */
+#define MXFP8_FLAG_E5M2 16       /* E5M2 elements (max 57344) instead of E4M3                   */
+
+/* Element format of the gradient operands (dy, dh) of the backward GEMMs (moe_ctx_set_grad_format). */
+#define MOE_GRAD_E4M3 0
+#define MOE_GRAD_E5M2 1
 
 /* Shared-exponent rules (moe_ctx_set_scale_rule).  ROUND_UP: e = the smallest integer with
  * amax <= 448 * 2^e, so no element saturates (this library's default reading of "a scaling factor
@@ -94,6 +99,15 @@ moe_status_t moe_ctx_set_debug_dump(moe_ctx_t ctx, float* a_f32, float* dh_f32);
  * MXFP8_SCALE_FLOOR.  Calls already enqueued are not affected. */
 moe_status_t moe_ctx_set_scale_rule(moe_ctx_t ctx, int rule);
 
+/* Element format of the MXFP8 gradient operands of the fused layer's backward with this context
+ * (ai4snews paragraph 2: FP8 and MXFP8 training): MOE_GRAD_E4M3 (default) or MOE_GRAD_E5M2.
+ * With E5M2, dy (quantised along d and along the tokens) and the requantised dh take E5M2
+ * elements (round to nearest even, saturating at 57344) with the same E8M0 scales per 32 values,
+ * the shared exponent computed against 57344 (round-up: the smallest e with amax <= 57344 * 2^e;
+ * floor rule: floor(log2 amax) - 15); every backward GEMM then multiplies an E5M2 A operand by an
+ * E4M3 B operand (weights, a, x).  The forward is unchanged. */
+moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt);
+
 /* Test hook for the bounded in-kernel waits (tests only).  With ``stall`` non-zero, every CTA of
  * the persistent kernels (the grouped GEMMs and the TMA-fed quantiser) makes one extra wait on a
  * word of the context's status block that nothing ever sets, bounded by ``limit_cycles`` SM clock
@@ -121,6 +135,7 @@ moe_status_t moe_ctx_set_launch_hook(moe_ctx_t ctx, moe_launch_hook_t hook, void
  * x        bf16 [batch, rows, cols]
  * flags    MXFP8_ROWWISE and/or MXFP8_COLWISE_T, optionally | MXFP8_SF_MMA_LAYOUT and
  *          | MXFP8_FLAG_SCALE_FLOOR (the OCP floor rule below instead of round-up)
+ *          | MXFP8_FLAG_E5M2 (E5M2 element codes; 57344 replaces 448 and 15 replaces 8 below)
  * q_row    uint8 [batch, rows, cols] E4M3 codes, blocks of 32 along each row   (ROWWISE)
  * s_row    uint8 E8M0 bytes, [batch, rows, cols/32] row-major, or the MMA layout (ROWWISE)
  * q_colT   uint8 [batch, cols, rows] codes of blocks of 32 down each column, transposed
@@ -144,7 +159,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
                             int flags, uint8_t* q_row, uint8_t* s_row, uint8_t* q_colT, uint8_t* s_colT,
                             void* stream);
 
-/* Inverse of mxfp8_quantize for row-wise data (tests): out[r][c] = decode(q[r][c]) * 2^(s-127),
+/* Inverse of mxfp8_quantize for row-wise E4M3 data (tests): out[r][c] = decode(q[r][c]) * 2^(s-127),
  * fp32 [rows, cols]; ``sf_mma_layout`` says how ``s`` is laid out.  cols % 32 == 0. */
 moe_status_t mxfp8_dequantize(moe_ctx_t ctx, const uint8_t* q, const uint8_t* s, int64_t rows, int64_t cols,
                               int sf_mma_layout, float* out, void* stream);

@@ -20,7 +20,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmoemx.so")
 
 MOE_ROW_ALIGN = 128
-MXFP8_ROWWISE, MXFP8_COLWISE_T, MXFP8_SF_MMA_LAYOUT, MXFP8_FLAG_SCALE_FLOOR = 1, 2, 4, 8
+MXFP8_ROWWISE, MXFP8_COLWISE_T, MXFP8_SF_MMA_LAYOUT, MXFP8_FLAG_SCALE_FLOOR, MXFP8_FLAG_E5M2 = 1, 2, 4, 8, 16
+GRAD_FORMATS = {"e4m3": 0, "e5m2": 1}
 SCALE_RULES = {"ceil": 0, "floor": 1}
 PRECISIONS = {"bf16": 0, "mxfp8": 1}
 STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "unsupported", 4: "cuda", 5: "device", 6: "timeout",
@@ -31,7 +32,8 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_get_status", "moe_ctx_set_d
            "mxfp8_quantize", "mxfp8_dequantize", "moe_capacity_rows", "moe_permute", "moe_unpermute",
            "moe_saved_size", "moe_fwd_workspace_size", "moe_bwd_workspace_size", "moe_grouped_mlp_fwd",
            "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook", "moe_grouped_mlp_fwd_noalloc",
-           "moe_ctx_set_test_stall", "moe_tensor_peak_loop", "moe_tensor_peak_flops", "moe_ctx_set_scale_rule"]
+           "moe_ctx_set_test_stall", "moe_tensor_peak_loop", "moe_tensor_peak_flops", "moe_ctx_set_scale_rule",
+           "moe_ctx_set_grad_format"]
 
 LAUNCH_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
@@ -63,6 +65,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ctx_set_debug_dump": (c_int, [c_vp, c_vp, c_vp]),
         "moe_ctx_set_test_stall": (c_int, [c_vp, c_int, c_i64]),
         "moe_ctx_set_scale_rule": (c_int, [c_vp, c_int]),
+        "moe_ctx_set_grad_format": (c_int, [c_vp, c_int]),
         "moe_tensor_peak_loop": (c_int, [c_vp, c_int, c_i64, c_int, c_vp]),
         "moe_tensor_peak_flops": (ctypes.c_double, [c_vp, c_int, c_i64]),
         "moe_status_string": (ctypes.c_char_p, [c_int]),
@@ -165,8 +168,14 @@ def set_scale_rule(device: int, rule: str):
     _check("moe_ctx_set_scale_rule", L.moe_ctx_set_scale_rule(context(device), SCALE_RULES[rule]))
 
 
+def set_grad_format(device: int, fmt: str):
+    """Element format of the MXFP8 gradient operands of the backward on ``device``: "e4m3" or "e5m2"."""
+    L = load_library()
+    _check("moe_ctx_set_grad_format", L.moe_ctx_set_grad_format(context(device), GRAD_FORMATS[fmt]))
+
+
 def mxfp8_quantize(x: torch.Tensor, rowwise: bool = True, colwise: bool = False, mma_layout: bool = False,
-                   scale_rule: str = "ceil"):
+                   scale_rule: str = "ceil", fmt: str = "e4m3"):
     """x bf16 [..., rows, cols] -> dict(q_row, s_row, q_colT, s_colT) (uint8; absent parts are None)."""
     assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() >= 2
     dev = _device_index(x)
@@ -178,6 +187,7 @@ def mxfp8_quantize(x: torch.Tensor, rowwise: bool = True, colwise: bool = False,
     out = dict(q_row=None, s_row=None, q_colT=None, s_colT=None)
     flags = (MXFP8_ROWWISE if rowwise else 0) | (MXFP8_COLWISE_T if colwise else 0) | (MXFP8_SF_MMA_LAYOUT if mma_layout else 0)
     flags |= MXFP8_FLAG_SCALE_FLOOR if scale_rule == "floor" else 0
+    flags |= MXFP8_FLAG_E5M2 if fmt == "e5m2" else 0
     if rowwise:
         out["q_row"] = torch.empty(lead + (rows, cols), dtype=torch.uint8, device=x.device)
         out["s_row"] = torch.empty(lead + (rows, cols // 32), dtype=torch.uint8, device=x.device)

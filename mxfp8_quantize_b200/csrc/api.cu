@@ -22,6 +22,7 @@ struct moe_ctx_s {
   moe_launch_hook_t hook;
   void* hook_user;
   int scale_floor;          // MXFP8 shared-exponent rule of the fused layer (moe_ctx_set_scale_rule)
+  int grad_e5m2;            // MXFP8 gradient operands in E5M2 (moe_ctx_set_grad_format)
   int stall;                // test hook for the bounded waits (moe_ctx_set_test_stall)
   long long stall_limit;
 };
@@ -412,6 +413,7 @@ moe_status_t moe_ctx_create(moe_ctx_t* out, int device) {
   c->hook = nullptr;
   c->hook_user = nullptr;
   c->scale_floor = 0;
+  c->grad_e5m2 = 0;
   c->stall = 0;
   c->stall_limit = 0;
   if (cudaMalloc(&c->d_status, 256) != cudaSuccess) {
@@ -462,6 +464,12 @@ moe_status_t moe_ctx_set_scale_rule(moe_ctx_t ctx, int rule) {
   return MOE_OK;
 }
 
+moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt) {
+  if (!ctx || (fmt != MOE_GRAD_E4M3 && fmt != MOE_GRAD_E5M2)) return MOE_ERR_INVALID_ARG;
+  ctx->grad_e5m2 = fmt == MOE_GRAD_E5M2 ? 1 : 0;
+  return MOE_OK;
+}
+
 moe_status_t moe_get_status(moe_ctx_t ctx, void* stream) {
   if (!ctx) return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->device);
@@ -484,7 +492,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
                             uint8_t* q_row, uint8_t* s_row, uint8_t* q_colT, uint8_t* s_colT, void* stream) {
   if (!ctx || !x || batch <= 0 || rows <= 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
   const bool row = flags & MXFP8_ROWWISE, col = flags & MXFP8_COLWISE_T, mma = flags & MXFP8_SF_MMA_LAYOUT;
-  if ((flags & ~15) || !(row || col)) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~31) || !(row || col)) return MOE_ERR_INVALID_ARG;
   if (row && (!q_row || !s_row)) return MOE_ERR_INVALID_ARG;
   if (col && (!q_colT || !s_colT)) return MOE_ERR_INVALID_ARG;
   if (cols % 32) return MOE_ERR_SHAPE;
@@ -505,6 +513,7 @@ moe_status_t mxfp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t
   a.do_col = col;
   a.sf_mma = mma;
   a.scale_floor = (flags & MXFP8_FLAG_SCALE_FLOOR) ? 1 : 0;
+  a.e5m2 = (flags & MXFP8_FLAG_E5M2) ? 1 : 0;
   a.q_row = q_row;
   a.s_row = s_row;
   a.q_colT = q_colT;
@@ -848,6 +857,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     if (D.mx) {
       a.mx = 1;
       a.sf_mma = 1;
+      a.e5m2 = ctx->grad_e5m2;  // dy is a gradient operand
       a.q_row = w.dy_q;
       a.s_row = w.dy_s;
       a.q_colT = w.dyT_q;
@@ -911,6 +921,8 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     ep.h = s.h;
     ep.dump = ctx->dbg_dh;
     ep.dp_part = w.dp_part;
+    ep.grad_e5m2 = ctx->grad_e5m2;  // dh is the gradient operand of both gate_up backward GEMMs
+    g.a_e5m2 = ctx->grad_e5m2;      // A = dy
     if (D.mx) {
       ep.q_row = w.dh_q;
       ep.s_row = w.dh_s;
@@ -942,6 +954,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     if (D.mx && !sf_maps(g, d, f, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
     g.epi.ldo = f;
     for (int e = 0; e < E; ++e) g.epi.out_ptrs.p[e] = dw_down[e];
+    g.a_e5m2 = ctx->grad_e5m2;  // A is a gradient operand (dy or dh)
     MOE_LAUNCH(ctx, "gemm_wgrad_down", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
   }
   // 4. dgrad of gate_up: dx_perm = dh W1 (K = 2f)
@@ -964,6 +977,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     if (D.mx && !sf_maps(g, D.cap, E * d, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
     g.epi.out = w.dx_perm;
     g.epi.ldo = d;
+    g.a_e5m2 = ctx->grad_e5m2;  // A is a gradient operand (dy or dh)
     MOE_LAUNCH(ctx, "gemm_dgrad_gate_up", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
   }
   // 5. wgrad of gate_up: dW1_e [2f, d] = dh_e^T x_e
@@ -986,12 +1000,14 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     if (D.mx && !sf_maps(g, 2 * f, d, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
     g.epi.ldo = d;
     for (int e = 0; e < E; ++e) g.epi.out_ptrs.p[e] = dw_gate_up[e];
+    g.a_e5m2 = ctx->grad_e5m2;  // A is a gradient operand (dy or dh)
     MOE_LAUNCH(ctx, "gemm_wgrad_gate_up", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
   }
   // 6. combine dx, reduce the probability gradient
   MOE_LAUNCH(ctx, "unpermute_dx", st, launch_unpermute(w.dx_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(dx), ctx->num_sms, st));
-  MOE_LAUNCH(ctx, "dprob_reduce", st, launch_dprob_reduce(w.dp_part, static_cast<int>(gemm_dswiglu_parts() * (f / gemm_tile_n(EPI_DSWIGLU))), D.cap, s.src2s, D.Tk,
-                                           d_topk_prob, st));
+  MOE_LAUNCH(ctx, "dprob_reduce", st,
+             launch_dprob_reduce(w.dp_part, static_cast<int>(gemm_dswiglu_parts() * (f / gemm_tile_n(EPI_DSWIGLU))),
+                                 D.cap, s.s2src, D.cap, s.src2s, D.Tk, d_topk_prob, st));
   return MOE_OK;
 }
 
@@ -1123,6 +1139,7 @@ moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx,
   c.hook = nullptr;
   c.hook_user = nullptr;
   c.scale_floor = 0;
+  c.grad_e5m2 = 0;
   c.stall = 0;
   c.stall_limit = 0;
   // the scratch base is 256-aligned; the workspace carving aligns to 1 KiB inside the size bound

@@ -38,19 +38,27 @@ route_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ top
   const int hi = min(Tk, lo + per_warp);
   const unsigned lt_mask = (1u << lane) - 1u;
 
-  // pass 1: per-warp histograms
-  for (int base = lo; base < hi; base += 32) {
-    const int s = base + lane;
-    int e = -1;
-    if (s < hi) {
-      e = topk_idx[s];
-      if (e < 0 || e >= E) {
+  // pass 1: per-warp histograms (each lane loads RB slots of a chunk before using any)
+  constexpr int RB = 16;
+  for (int base = lo; base < hi; base += 32 * RB) {
+    int ev[RB];
+#pragma unroll
+    for (int i = 0; i < RB; ++i) {
+      const int s = base + 32 * i + lane;
+      ev[i] = s < hi ? topk_idx[s] : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < RB; ++i) {
+      const int s = base + 32 * i + lane;
+      int e = ev[i];
+      if (s < hi && (e < 0 || e >= E)) {
         s_bad = 1;
         e = -1;
       }
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && (peers & lt_mask) == 0) wcnt[warp * E + e] += __popc(peers);
+      __syncwarp();
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && (peers & lt_mask) == 0) wcnt[warp * E + e] += __popc(peers);
   }
   __syncthreads();
 
@@ -78,26 +86,32 @@ route_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ top
   for (int e = tid; e <= E; e += blockDim.x) poffsets[e] = s_poff[e];
   if (tid == 0 && s_bad) atomicOr(status, kStatusDevice);
 
-  // pass 2: positions
-  for (int base = lo; base < hi; base += 32) {
-    const int s = base + lane;
-    int e = -1;
-    if (s < hi) {
-      e = topk_idx[s];
-      if (e < 0 || e >= E) e = -1;
+  // pass 2: positions (same chunking)
+  for (int base = lo; base < hi; base += 32 * RB) {
+    int ev[RB];
+#pragma unroll
+    for (int i = 0; i < RB; ++i) {
+      const int s = base + 32 * i + lane;
+      ev[i] = s < hi ? topk_idx[s] : -1;
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    int pos = -1;
-    if (e >= 0) pos = s_poff[e] + wcnt[warp * E + e] + __popc(peers & lt_mask);
-    __syncwarp();
-    if (e >= 0 && (peers & lt_mask) == 0) wcnt[warp * E + e] += __popc(peers);
-    __syncwarp();
-    if (e >= 0) {
-      sorted_to_src[pos] = s;
-      src_to_sorted[s] = pos;
-      if (prob_perm) prob_perm[pos] = topk_prob[s];
-    } else if (s < hi) {
-      src_to_sorted[s] = -1;
+#pragma unroll
+    for (int i = 0; i < RB; ++i) {
+      const int s = base + 32 * i + lane;
+      int e = ev[i];
+      if (e < 0 || e >= E) e = -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      int pos = -1;
+      if (e >= 0) pos = s_poff[e] + wcnt[warp * E + e] + __popc(peers & lt_mask);
+      __syncwarp();
+      if (e >= 0 && (peers & lt_mask) == 0) wcnt[warp * E + e] += __popc(peers);
+      __syncwarp();
+      if (e >= 0) {
+        sorted_to_src[pos] = s;
+        src_to_sorted[s] = pos;
+        if (prob_perm) prob_perm[pos] = topk_prob[s];
+      } else if (s < hi) {
+        src_to_sorted[s] = -1;
+      }
     }
   }
 }
@@ -127,9 +141,6 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
 // fp32 bits of the larger half of a bf16 pair of non-negative values
 __device__ __forceinline__ uint32_t fold_halves(uint32_t m2) { return max(m2 << 16, m2 & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
-}
 }  // namespace
 
 // Column-wise outputs of one thread: columns (2p, 2p+1) of the tile and 32-row block rb (each smem
@@ -146,19 +157,19 @@ __device__ __forceinline__ void column_pass(const QuantArgs& a, const uint32_t* 
     m2 = absmax_bf16x2(m2, wv[i]);
   }
   if (a.mx) {
-    const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16, a.scale_floor);
-    const uint32_t sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u, a.scale_floor);
+    const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16, a.scale_floor, a.e5m2);
+    const uint32_t sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u, a.scale_floor, a.e5m2);
     const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
     uint32_t q0[8], q1[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t lo0 = e4m3x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0);
+      const uint32_t lo0 = fp8x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0, a.e5m2);
       const uint32_t hi0 =
-          e4m3x2(__uint_as_float(wv[4 * i + 2] << 16) * inv0, __uint_as_float(wv[4 * i + 3] << 16) * inv0);
-      const uint32_t lo1 = e4m3x2(__uint_as_float(wv[4 * i] & 0xFFFF0000u) * inv1,
-                                  __uint_as_float(wv[4 * i + 1] & 0xFFFF0000u) * inv1);
-      const uint32_t hi1 = e4m3x2(__uint_as_float(wv[4 * i + 2] & 0xFFFF0000u) * inv1,
-                                  __uint_as_float(wv[4 * i + 3] & 0xFFFF0000u) * inv1);
+          fp8x2(__uint_as_float(wv[4 * i + 2] << 16) * inv0, __uint_as_float(wv[4 * i + 3] << 16) * inv0, a.e5m2);
+      const uint32_t lo1 = fp8x2(__uint_as_float(wv[4 * i] & 0xFFFF0000u) * inv1,
+                                  __uint_as_float(wv[4 * i + 1] & 0xFFFF0000u) * inv1, a.e5m2);
+      const uint32_t hi1 = fp8x2(__uint_as_float(wv[4 * i + 2] & 0xFFFF0000u) * inv1,
+                                  __uint_as_float(wv[4 * i + 3] & 0xFFFF0000u) * inv1, a.e5m2);
       q0[i] = lo0 | (hi0 << 16);
       q1[i] = lo1 | (hi1 << 16);
     }
@@ -267,14 +278,14 @@ quant_tile_kernel(const __grid_constant__ QuantArgs a) {
       uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w)));
       m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      const uint32_t sb = e8m0_from_amax_bits(m, a.scale_floor);
+      const uint32_t sb = e8m0_from_amax_bits(m, a.scale_floor, a.e5m2);
       const float inv = e8m0_inv_scale(sb);
       if (valid) {
         const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
         uint32_t q[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
+          q[j] = fp8x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv, a.e5m2);
         const uint2 qq = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
         if (a.tma_store) {  // row lr, bytes 8*cchunk.. of the swizzled 128-byte row
           uint8_t* rowp = qdyn + lr * 128;
@@ -484,13 +495,13 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         uint32_t m = fold_halves(absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        const uint32_t sb = e8m0_from_amax_bits(m, a.scale_floor);
+        const uint32_t sb = e8m0_from_amax_bits(m, a.scale_floor, a.e5m2);
         const float inv = e8m0_inv_scale(sb);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t q[4];
   #pragma unroll
         for (int j = 0; j < 4; ++j)
-          q[j] = e4m3x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
+          q[j] = fp8x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv, a.e5m2);
         *reinterpret_cast<uint2*>(qrow + lr * 128 + (((cchunk >> 1) ^ (lr & 7)) << 4) + ((cchunk & 1) << 3)) =
             make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
         if ((cchunk & 3) == 0) satom_row[sf_mma_offset(lr, (cchunk >> 2) & 3, 4)] = static_cast<uint8_t>(sb);
@@ -507,20 +518,20 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
           wv[i] = words[(rb * 32 + i) * 64 + p];
           m2 = absmax_bf16x2(m2, wv[i]);
         }
-        const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16, a.scale_floor);
-        const uint32_t sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u, a.scale_floor);
+        const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16, a.scale_floor, a.e5m2);
+        const uint32_t sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u, a.scale_floor, a.e5m2);
         const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
         uint32_t q0[8], q1[8];
   #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint32_t lo0 =
-              e4m3x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0);
+              fp8x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0, a.e5m2);
           const uint32_t hi0 =
-              e4m3x2(__uint_as_float(wv[4 * i + 2] << 16) * inv0, __uint_as_float(wv[4 * i + 3] << 16) * inv0);
-          const uint32_t lo1 = e4m3x2(__uint_as_float(wv[4 * i] & 0xFFFF0000u) * inv1,
-                                      __uint_as_float(wv[4 * i + 1] & 0xFFFF0000u) * inv1);
-          const uint32_t hi1 = e4m3x2(__uint_as_float(wv[4 * i + 2] & 0xFFFF0000u) * inv1,
-                                      __uint_as_float(wv[4 * i + 3] & 0xFFFF0000u) * inv1);
+              fp8x2(__uint_as_float(wv[4 * i + 2] << 16) * inv0, __uint_as_float(wv[4 * i + 3] << 16) * inv0, a.e5m2);
+          const uint32_t lo1 = fp8x2(__uint_as_float(wv[4 * i] & 0xFFFF0000u) * inv1,
+                                      __uint_as_float(wv[4 * i + 1] & 0xFFFF0000u) * inv1, a.e5m2);
+          const uint32_t hi1 = fp8x2(__uint_as_float(wv[4 * i + 2] & 0xFFFF0000u) * inv1,
+                                      __uint_as_float(wv[4 * i + 3] & 0xFFFF0000u) * inv1, a.e5m2);
           q0[i] = lo0 | (hi0 << 16);
           q1[i] = lo1 | (hi1 << 16);
         }
@@ -631,19 +642,33 @@ unpermute_kernel(const bf16* __restrict__ rows, const int32_t* __restrict__ src_
   }
 }
 
-// d_topk_prob[t][j] = sum over n-tiles (ascending) of the partial row sums of the
-// ScaledSwiGLU probability gradient, read at row(t, j).
+// d_topk_prob[t][j] = sum over n-tiles (ascending) of the partial row sums of the ScaledSwiGLU
+// probability gradient at row(t, j).  Threads walk the rows (consecutive threads read consecutive
+// words of every partial) and write the sum to the row's slot; slots the routing rejected (no row)
+// get zero.
 __global__ void dprob_reduce_kernel(const float* __restrict__ part, int n_parts, int64_t part_stride,
+                                    const int32_t* __restrict__ sorted_to_src, int64_t rows,
                                     const int32_t* __restrict__ src_to_sorted, int64_t Tk,
                                     float* __restrict__ d_prob) {
-  for (int64_t s = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; s < Tk;
-       s += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = src_to_sorted[s];
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  for (int64_t r = i0; r < rows; r += stride) {
+    const int32_t s = sorted_to_src[r];
+    if (s < 0) continue;  // padding row
     float acc = 0.f;
-    if (r >= 0)  // a rejected slot has no row and gets a zero gradient
-      for (int n = 0; n < n_parts; ++n) acc = __fadd_rn(acc, part[n * part_stride + r]);
+    int n = 0;
+    for (; n + 8 <= n_parts; n += 8) {  // eight independent loads in flight, summed in order
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __ldg(part + (n + q) * part_stride + r);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc = __fadd_rn(acc, v[q]);
+    }
+    for (; n < n_parts; ++n) acc = __fadd_rn(acc, __ldg(part + n * part_stride + r));
     d_prob[s] = acc;
   }
+  for (int64_t s = i0; s < Tk; s += stride)
+    if (src_to_sorted[s] < 0) d_prob[s] = 0.f;
 }
 
 // Row-wise MXFP8 -> fp32 (tests).
@@ -707,12 +732,13 @@ cudaError_t launch_unpermute(const bf16* rows, const int32_t* src_to_sorted, con
   return cudaGetLastError();
 }
 
-cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_stride, const int32_t* src_to_sorted,
-                                int64_t Tk, float* d_prob, cudaStream_t st) {
+cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_stride, const int32_t* sorted_to_src,
+                                int64_t rows, const int32_t* src_to_sorted, int64_t Tk, float* d_prob,
+                                cudaStream_t st) {
   if (Tk == 0) return cudaSuccess;
-  const int64_t blocks = std::min<int64_t>(ceil_div(Tk, 256), 4096);
-  dprob_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(part, n_parts, part_stride, src_to_sorted, Tk,
-                                                                      d_prob);
+  const int64_t blocks = std::min<int64_t>(ceil_div(std::max(rows, Tk), 256), 4096);
+  dprob_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(part, n_parts, part_stride, sorted_to_src, rows,
+                                                                      src_to_sorted, Tk, d_prob);
   return cudaGetLastError();
 }
 

@@ -23,6 +23,7 @@ struct QuantArgs {
   int64_t gate_up_half;        // >0: row-wise outputs in 256-row groups [128 rows < half | 128 rows >= half]
   int do_row, do_col, sf_mma;
   int scale_floor;             // MXFP8 shared exponent: 0 round-up rule, 1 OCP floor rule
+  int e5m2;                    // MXFP8 element format: 0 E4M3, 1 E5M2
   uint8_t* q_row;
   uint8_t* s_row;
   uint8_t* q_colT;
@@ -55,8 +56,9 @@ cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk
 cudaError_t launch_quant(const QuantArgs& a, int batch, int num_sms, cudaStream_t st);
 cudaError_t launch_unpermute(const bf16* rows, const int32_t* src_to_sorted, const float* probs, int64_t T, int k,
                              int64_t d, bf16* y, int num_sms, cudaStream_t st);
-cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_stride, const int32_t* src_to_sorted,
-                                int64_t Tk, float* d_prob, cudaStream_t st);
+cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_stride, const int32_t* sorted_to_src,
+                                int64_t rows, const int32_t* src_to_sorted, int64_t Tk, float* d_prob,
+                                cudaStream_t st);
 cudaError_t launch_dequant(const uint8_t* q, const uint8_t* s, int64_t R, int64_t C, int sf_mma, float* out,
                            int num_sms, cudaStream_t st);
 

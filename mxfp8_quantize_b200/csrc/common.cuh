@@ -1,6 +1,7 @@
 // Internal definitions shared by the kernels and the C ABI layer of libmoemx.
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -31,12 +32,19 @@ __host__ __device__ inline int64_t sf_mma_offset(int64_t r, int64_t kb, int64_t 
 // (amax = (1 + m/2^23) * 2^E: e = E - 8, plus one when the mantissa exceeds 0.75), clamped to
 // [-127, 127].  With ``floor_rule`` (the OCP MX v1.0 variant) e = E - 8 = floor(log2 amax) - 8,
 // and the block's largest elements may exceed 448 after scaling (the conversion saturates them).
+// For E5M2 elements (``e5m2``) the largest finite value is 57344 = 1.75 * 2^15: 15 replaces 8.
 // Returns the biased byte e + 127.
-__device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t abits, int floor_rule = 0) {
+__device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t abits, int floor_rule = 0, int e5m2 = 0) {
   const int E = static_cast<int>((abits >> 23) & 0xFFu) - 127;
-  int e = E - 8 + ((!floor_rule && (abits & 0x7FFFFFu) > 0x600000u) ? 1 : 0);
+  int e = E - (e5m2 ? 15 : 8) + ((!floor_rule && (abits & 0x7FFFFFu) > 0x600000u) ? 1 : 0);
   e = e < -127 ? -127 : (e > 127 ? 127 : e);
   return static_cast<uint32_t>(e + 127);
+}
+// Two fp32 values -> two 8-bit codes (low byte first), round to nearest even, saturating: E4M3, or
+// E5M2 when ``e5m2``.
+__device__ __forceinline__ uint32_t fp8x2(float lo, float hi, int e5m2) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, e5m2 ? __NV_E5M2 : __NV_E4M3));
 }
 // 2^-(byte-127) as an fp32 (byte <= 253 for every finite input).
 __device__ __forceinline__ float e8m0_inv_scale(uint32_t byte) {

@@ -150,22 +150,18 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 v, float* o) {
     o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
-  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
-}
-
-// MXFP8 of 32 values with the scale of their own amax: 32 codes stored at q (32-byte aligned);
-// returns the E8M0 byte.
-__device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q, int floor_rule) {
+// MXFP8 of 32 values with the scale of their own amax: 32 codes (E4M3, or E5M2 when ``e5m2``)
+// stored at q (32-byte aligned); returns the E8M0 byte.
+__device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q, int floor_rule, int e5m2) {
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) m = max(m, __float_as_uint(v[i]) & 0x7FFFFFFFu);
-  const uint32_t sb = e8m0_from_amax_bits(m, floor_rule);
+  const uint32_t sb = e8m0_from_amax_bits(m, floor_rule, e5m2);
   const float inv = e8m0_inv_scale(sb);
   uint32_t w[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    w[i] = e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv) | (e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv) << 16);
+    w[i] = fp8x2(v[4 * i] * inv, v[4 * i + 1] * inv, e5m2) | (fp8x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv, e5m2) << 16);
   ptx::st_global_v8(q, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
   return sb;
 }
@@ -196,19 +192,20 @@ __device__ __forceinline__ void column_passes(const float* v, float* stage, F&& 
 // tile-layout scale matrix with sf_KB columns.
 template <int P>
 __device__ __forceinline__ void colwise_mx(const float* v, float* stage, uint8_t* colT, int64_t ld, uint8_t* sf,
-                                           int64_t sf_row0, int64_t sf_kb, int64_t sf_KB, int floor_rule) {
+                                           int64_t sf_row0, int64_t sf_kb, int64_t sf_KB, int floor_rule, int e5m2) {
   column_passes<P>(v, stage, [&](int h, int cl, int rg, const float* col) {
     uint32_t m = 0;
 #pragma unroll
     for (int i = 0; i < P; ++i) m = max(m, __float_as_uint(col[i]) & 0x7FFFFFFFu);
 #pragma unroll
     for (int s = P; s < 32; s <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, s));
-    const uint32_t sb = e8m0_from_amax_bits(m, floor_rule);
+    const uint32_t sb = e8m0_from_amax_bits(m, floor_rule, e5m2);
     const float inv = e8m0_inv_scale(sb);
     uint32_t w[P / 4];
 #pragma unroll
     for (int i = 0; i < P / 4; ++i)
-      w[i] = e4m3x2(col[4 * i] * inv, col[4 * i + 1] * inv) | (e4m3x2(col[4 * i + 2] * inv, col[4 * i + 3] * inv) << 16);
+      w[i] = fp8x2(col[4 * i] * inv, col[4 * i + 1] * inv, e5m2) |
+             (fp8x2(col[4 * i + 2] * inv, col[4 * i + 3] * inv, e5m2) << 16);
     const int c = P * h + cl;
     uint8_t* dst = colT + c * ld + P * rg;
     if constexpr (P == 16) {
@@ -401,6 +398,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     const uint64_t bdesc0 = ptx::smem_desc(smem0 + S::OFF_B, 16, 1024, ptx::kSwizzle128B);
     const uint64_t sfadesc0 = ptx::smem_desc(smem0 + S::OFF_SFA, 0, 128, ptx::kSwizzleNone);
     const uint64_t sfbdesc0 = ptx::smem_desc(smem0 + S::OFF_SFB, 0, 128, ptx::kSwizzleNone);
+    const uint32_t a_fmt = ptx::idesc_a_format(g.a_e5m2 ? ptx::kFmtE5M2 : ptx::kFmtE4M3);  // A's element format
     for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
       Tile tl;
       decode_tile(t, s, g, MX, tl);
@@ -428,8 +426,8 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           for (int i = 0; i < BN / 128; ++i) ptx::tc_cp_32x128b_warpx4(sfb_t + 4 * i, sfbdesc0 + soff + 32 * i);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            ptx::tc_mma_mxf8(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(BM, BN, k, k), sfa_t, sfb_t,
-                             (kb | k) != 0);
+            ptx::tc_mma_mxf8(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(BM, BN, k, k) | a_fmt, sfa_t,
+                             sfb_t, (kb | k) != 0);
         } else {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
@@ -545,11 +543,11 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             for (int i = 0; i < 8; ++i) dd[i] = make_float4(gv[4 * i], gv[4 * i + 1], gv[4 * i + 2], gv[4 * i + 3]);
           }
           if (MX) {
-            const uint32_t sb = quant32_store(gv, ep.q_row + row * f + j, ep.scale_floor);
+            const uint32_t sb = quant32_store(gv, ep.q_row + row * f + j, ep.scale_floor, 0);
             ep.s_row[sf_mma_offset(row, j / 32, f / 32)] = static_cast<uint8_t>(sb);
             if (ep.q_colT)
               colwise_mx<S::PASS>(gv, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
-                                  ep.cap / 32, ep.scale_floor);
+                                  ep.cap / 32, ep.scale_floor, 0);
           } else {
             bf16* dst = ep.o_row + row * f + j;
 #pragma unroll
@@ -642,14 +640,14 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             }
           }
           if (MX) {
-            uint32_t sb = quant32_store(dg, ep.q_row + row * f2 + j, ep.scale_floor);
+            uint32_t sb = quant32_store(dg, ep.q_row + row * f2 + j, ep.scale_floor, ep.grad_e5m2);
             ep.s_row[sf_mma_offset(row, j / 32, f2 / 32)] = static_cast<uint8_t>(sb);
-            sb = quant32_store(du, ep.q_row + row * f2 + f + j, ep.scale_floor);
+            sb = quant32_store(du, ep.q_row + row * f2 + f + j, ep.scale_floor, ep.grad_e5m2);
             ep.s_row[sf_mma_offset(row, (f + j) / 32, f2 / 32)] = static_cast<uint8_t>(sb);
             colwise_mx<S::PASS>(dg, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
-                                ep.cap / 32, ep.scale_floor);
+                                ep.cap / 32, ep.scale_floor, ep.grad_e5m2);
             colwise_mx<S::PASS>(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j,
-                                row_w / 32, ep.cap / 32, ep.scale_floor);
+                                row_w / 32, ep.cap / 32, ep.scale_floor, ep.grad_e5m2);
           } else {
             bf16* d0 = ep.o_row + row * f2 + j;
             bf16* d1 = d0 + f;

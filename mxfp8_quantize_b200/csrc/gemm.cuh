@@ -30,6 +30,7 @@ struct EpiArgs {
   bf16* o_colT;
   float* dump;        // debug: fp32 values before quantisation
   int scale_floor;    // MXFP8 shared exponent of the requantisations: 0 round-up rule, 1 OCP floor rule
+  int grad_e5m2;      // DSWIGLU: dh requantised with E5M2 elements (gradient-format variant)
   float* dp_part;     // DSWIGLU: [parts * n_tiles, cap] partial sums of the probability gradient
 };
 
@@ -55,6 +56,7 @@ struct GemmArgs {
   const uint8_t* sfb;
   int64_t sfb_kb4;
   int64_t sfb_expert_rows;  // rows of B per expert (M-grouped), for the scale tile index
+  int a_e5m2;          // MXFP8: A's elements are E5M2 (B's stay E4M3)
   int* status;
   // test hook: a device flag nothing sets; when non-null the producer of each CTA waits on it once,
   // for at most stall_limit cycles, after issuing the first stages of its first tile

@@ -205,8 +205,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N) {
          | ((N >> 3) << 17)   // N / 8
          | ((M >> 4) << 24);  // M / 16
 }
+// Element formats of kind::mxf8f6f4 operands (instruction descriptor fields at bits 7-9 for A and
+// 10-12 for B); A and B may differ.
+constexpr uint32_t kFmtE4M3 = 0;
+constexpr uint32_t kFmtE5M2 = 1;
+__host__ __device__ constexpr uint32_t idesc_a_format(uint32_t fmt) { return (fmt & 7u) << 7; }
 // Instruction descriptor, kind::mxf8f6f4 with E4M3 A/B, E8M0 scales, K-major; the scale-factor
-// ids select which byte of each 32-bit TMEM scale cell an MMA reads.
+// ids select which byte of each 32-bit TMEM scale cell an MMA reads.  OR in idesc_a_format for an
+// A operand of another format.
 __host__ __device__ constexpr uint32_t idesc_mxf8(uint32_t M, uint32_t N, uint32_t sfa_id, uint32_t sfb_id) {
   return ((sfb_id & 3u) << 4)  // B scale-factor id
          | (0u << 7)           // A E4M3

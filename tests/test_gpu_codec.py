@@ -176,3 +176,36 @@ def test_golden_floor_vectors_on_gpu():
     for i, (name, v, sbyte, codes) in enumerate(cases):
         assert int(s[i, 0]) == sbyte, name
         assert [int(c) for c in q[i, :len(codes)]] == codes, name
+
+
+@pytest.mark.parametrize("rule", ["ceil", "floor"])
+@pytest.mark.parametrize("rows,cols,colwise,mma", [(64, 128, True, False), (128, 256, True, True), (4096, 512, True, True)])
+def test_quantize_e5m2_bit_exact(rows, cols, colwise, mma, rule):
+    """E5M2 element codes (MXFP8_FLAG_E5M2, the gradient format), both quantiser kernels, both rules."""
+    x = _spread_bf16(rows, cols, seed=3 * rows + cols)
+    out = moe.mxfp8_quantize(x.cuda(), rowwise=True, colwise=colwise, mma_layout=mma, scale_rule=rule, fmt="e5m2")
+    torch.cuda.synchronize()
+    xf = x.float().numpy()
+    q, s = mx.quantize_rowwise(xf, rule=rule, fmt="e5m2")
+    assert np.array_equal(out["q_row"].cpu().numpy(), q)
+    s_gpu = out["s_row"].cpu().numpy()
+    assert np.array_equal(unswizzle_scales(s_gpu, rows, cols // 32) if mma else s_gpu, s)
+    if colwise:
+        qc, sc = mx.quantize_colwise_t(xf, rule=rule, fmt="e5m2")
+        assert np.array_equal(out["q_colT"].cpu().numpy(), qc)
+        sc_gpu = out["s_colT"].cpu().numpy()
+        assert np.array_equal(unswizzle_scales(sc_gpu, cols, rows // 32) if mma else sc_gpu, sc)
+
+
+def test_golden_e5m2_vectors_on_gpu():
+    from tests.test_oracle_mx import GOLDEN_E5M2, _golden_cases
+    cases = _golden_cases(GOLDEN_E5M2)
+    x = np.zeros((len(cases), 32))
+    for i, (_, v, _, _) in enumerate(cases):
+        x[i] = v
+    out = moe.mxfp8_quantize(torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).cuda(), rowwise=True,
+                             fmt="e5m2")
+    q, s = out["q_row"].cpu().numpy(), out["s_row"].cpu().numpy()
+    for i, (name, v, sbyte, codes) in enumerate(cases):
+        assert int(s[i, 0]) == sbyte, name
+        assert [int(c) for c in q[i, :len(codes)]] == codes, name

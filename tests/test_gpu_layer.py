@@ -267,3 +267,40 @@ def test_floor_scale_rule_layer():
         got = g[name]
         got = got.float().cpu().numpy() if got.dtype == torch.bfloat16 else got.cpu().numpy()
         parity(f"small_floor_rule.{name}", got, ref, TOL[precision])
+
+
+def test_e5m2_gradient_format_layer():
+    """The backward with E5M2 gradient operands (moe_ctx_set_grad_format): dy quantised both ways
+    and the dSwiGLU requantisation of dh bit-exact against the oracle's E5M2 codec, the backward
+    GEMMs multiplying E5M2 A by E4M3 B, outputs within tolerance of the oracle's e5m2 layer."""
+    precision = "mxfp8"
+    cfg = workloads.scaled_config(workloads.CONFIGS["small_mxfp8"], T=1024, seed=42)
+    moe.set_grad_format(0, "e5m2")
+    try:
+        g = _run(cfg, precision)
+    finally:
+        moe.set_grad_format(0, "e4m3")
+    np_in = {n: (t.float().numpy() if t.dtype == torch.bfloat16 else t.numpy()) for n, t in g["inp"].items()}
+    y, st = omoe.forward(np_in["x"], np_in["topk_idx"], np_in["topk_prob"], np_in["w_gate_up"], np_in["w_down"],
+                         precision, grad_format="e5m2")
+    gr = omoe.backward(np_in["dy"], st, np_in["w_gate_up"], np_in["w_down"])
+    d, f, cap = cfg.d, cfg.f, g["cap"]
+    Tp = int(st["route"]["poffsets"][cfg.E])
+    dyp = routing.permute_rows(np_in["dy"], st["route"]["sorted_to_src"], cfg.k)
+    q = _view(g["bws"], 2, "dy_q", cfg, precision, True, cap * d).cpu().numpy().reshape(cap, d)
+    assert np.array_equal(q[:Tp], mx.quantize_rowwise(dyp, fmt="e5m2")[0])
+    q = _view(g["bws"], 2, "dyT_q", cfg, precision, True, d * cap).cpu().numpy().reshape(d, cap)
+    assert np.array_equal(q[:, :Tp], mx.quantize_colwise_t(dyp, fmt="e5m2")[0])
+    dh32 = g["dump_dh"].cpu().numpy()[:Tp]
+    q = _view(g["bws"], 2, "dh_q", cfg, precision, True, cap * 2 * f).cpu().numpy().reshape(cap, 2 * f)
+    s = _view(g["bws"], 2, "dh_s", cfg, precision, True, cap * 2 * f // 32).cpu().numpy()
+    rq, rs = mx.quantize_rowwise(dh32, fmt="e5m2")
+    assert np.array_equal(q[:Tp], rq)
+    assert np.array_equal(unswizzle_scales(s, cap, 2 * f // 32)[:Tp], rs)
+    q = _view(g["bws"], 2, "dhT_q", cfg, precision, True, 2 * f * cap).cpu().numpy().reshape(2 * f, cap)
+    assert np.array_equal(q[:, :Tp], mx.quantize_colwise_t(dh32, fmt="e5m2")[0])
+    assert rel_err(bf16_np(g["y"]), y) <= TOL[precision]          # the forward is unchanged
+    for name, ref in (("dx", gr["dx"]), ("dw1", gr["dw_gate_up"]), ("dw2", gr["dw_down"]), ("dp", gr["d_topk_prob"])):
+        got = g[name]
+        got = got.float().cpu().numpy() if got.dtype == torch.bfloat16 else got.cpu().numpy()
+        parity(f"small_e5m2_grads.{name}", got, ref, TOL[precision])
