@@ -97,7 +97,7 @@ int64_t uniform_stride(const void* const* p, int E, int64_t min_bytes);
 void quant_load_map(QuantArgs& a, int batch) {
   a.tma_load = 0;
   a.tma_gather = 0;
-  const bool outputs_ok = a.mx ? (a.do_row && a.do_col) : (a.do_col && !a.do_row);  // the kernel's two modes
+  const bool outputs_ok = a.mx ? a.do_row : (a.do_col && !a.do_row);  // the kernel's modes
   if (a.rows % 128 || a.cols % 128 || !outputs_ok) return;
   if (a.sorted_to_src) {
     // MXFP8 gather of one [src_rows, cols] source: rows fetched four at a time by tile::gather4

@@ -355,7 +355,7 @@ quant_tile_kernel(const __grid_constant__ QuantArgs a) {
 }
 
 // ------------------------------------------------------------------------------------------
-// The same MXFP8 quantisation (tensor-core scale layout, row-wise and column-wise) for a uniformly
+// The same MXFP8 quantisation (tensor-core scale layout, row-wise and optionally column-wise) for a uniformly
 // strided [batch, rows, cols] source whose rows and cols are multiples of 128, as a persistent
 // kernel: QW_CTAS_PER_SM CTAs per SM walk the 128 x 128 tiles (column tiles fastest); each source
 // tile arrives by a TMA tensor load into a QW_NIN-deep ring issued QW_NIN tiles ahead, and the
@@ -394,9 +394,21 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
     const int64_t hf = a.gate_up_half;
     return r < hf ? (r / 128) * 256 + (r % 128) : ((r - hf) / 128) * 256 + 128 + ((r - hf) % 128);
   };
+  // gather: the four source rows lane ``tid`` of warp 0 fetches for tile t (padding rows point past
+  // the last source row, where the copy reads zeros)
+  auto gather_rows = [&](int t, int32_t (&y)[4]) {
+    int b, rt, ct;
+    coords(t, b, rt, ct);
+    const int64_t r0 = static_cast<int64_t>(rt) * QT_ROWS + 4 * (tid & 31);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int32_t s = a.sorted_to_src[r0 + j];
+      y[j] = s < 0 ? static_cast<int32_t>(a.src_rows) : s / a.k;
+    }
+  };
   // source tile t into ring slot ``slot``: one 3-D box (thread 0), or, for a gather, 32 gather4
-  // loads of four rows each (one per lane of warp 0)
-  auto issue = [&](int t, int slot) {
+  // loads of four rows each (one per lane of warp 0, rows ``y``)
+  auto issue = [&](int t, int slot, const int32_t (&y)[4]) {
     int b, rt, ct;
     coords(t, b, rt, ct);
     if (!a.tma_gather) {
@@ -405,13 +417,6 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
       return;
     }
     const int lane = tid & 31;
-    const int64_t r0 = static_cast<int64_t>(rt) * QT_ROWS + 4 * lane;
-    int32_t y[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int32_t s = a.sorted_to_src[r0 + j];
-      y[j] = s < 0 ? static_cast<int32_t>(a.src_rows) : s / a.k;  // padding: past the last row -> zeros
-    }
     if (lane == 0) ptx::mbar_arrive_expect_tx(&full[slot], QW_IN_BYTES);
     ptx::tma_gather4(in_base + slot * QW_IN_BYTES + lane * 4 * 256, &a.tmap_src, ct * QT_COLS, y[0], y[1], y[2], y[3],
                      &full[slot]);
@@ -425,14 +430,21 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
   }
   __syncthreads();
   int issued_last = 0;  // last tile whose load was issued (waited for at exit only after an abort)
-  if (issuer)
+  // gather: rows of the next tile to be issued, loaded one refill ahead so that the index loads'
+  // latency overlaps a tile's work instead of delaying the refill
+  int32_t y_next[4] = {0, 0, 0, 0};
+  if (issuer) {
     for (int j = 0; j < QW_NIN; ++j) {
       const int t = blockIdx.x + j * gridDim.x;
       if (t < tiles) {
-        issue(t, j);
+        if (a.tma_gather) gather_rows(t, y_next);
+        issue(t, j, y_next);
         issued_last = t;
       }
     }
+    const int tn = blockIdx.x + QW_NIN * gridDim.x;
+    if (a.tma_gather && tn < tiles) gather_rows(tn, y_next);
+  }
   int it = 0;
   for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
     const int slot = it % QW_NIN;
@@ -508,7 +520,7 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
       }
 
       // ---- column-wise: thread -> columns (2p, 2p+1), 32-row block rb
-      {
+      if (a.do_col) {
         const int p = tid & 63, rb = tid >> 6;
         const uint32_t* words = reinterpret_cast<const uint32_t*>(in);  // 64 bf16 pairs per row
         uint32_t wv[32];
@@ -556,11 +568,12 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
                      "r"(static_cast<int32_t>(col0)), "r"(static_cast<int32_t>(b * R + dst_row(row0))),
                      "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qrow)))
                      : "memory");
-        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                         reinterpret_cast<uint64_t>(&a.tmap_qcol)),
-                     "r"(static_cast<int32_t>(row0)), "r"(static_cast<int32_t>(b * C + col0)),
-                     "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qcol)))
-                     : "memory");
+        if (a.do_col)
+          asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                           reinterpret_cast<uint64_t>(&a.tmap_qcol)),
+                       "r"(static_cast<int32_t>(row0)), "r"(static_cast<int32_t>(b * C + col0)),
+                       "r"(static_cast<uint32_t>(__cvta_generic_to_shared(qcol)))
+                       : "memory");
       } else {  // the transposed bf16 tile: two boxes of 64 columns x 128 rows
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -575,8 +588,9 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
     if (issuer) {
       const int tn = t + QW_NIN * gridDim.x;  // refill the slot just consumed
       if (tn < tiles) {
-        issue(tn, slot);
+        issue(tn, slot, y_next);
         issued_last = tn;
+        if (a.tma_gather && tn + static_cast<int>(gridDim.x) < tiles) gather_rows(tn + gridDim.x, y_next);
       }
     } else if (a.mx && tid >= 32 && tid < 64) {  // warp 1: the two 512-byte scale tiles, 16 bytes per lane
       const int l = tid - 32;
@@ -584,9 +598,11 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         uint8_t* sr = a.s_row + static_cast<int64_t>(b) * R * KBr;
         reinterpret_cast<uint4*>(sr + ((dst_row(row0) / 128) * (KBr / 4) + col0 / 128) * 512)[l] =
             reinterpret_cast<const uint4*>(satom_row)[l];
-        uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
-        reinterpret_cast<uint4*>(sc + ((col0 / 128) * (KBc / 4) + row0 / 128) * 512)[l] =
-            reinterpret_cast<const uint4*>(satom_col)[l];
+        if (a.do_col) {
+          uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
+          reinterpret_cast<uint4*>(sc + ((col0 / 128) * (KBc / 4) + row0 / 128) * 512)[l] =
+              reinterpret_cast<const uint4*>(satom_col)[l];
+        }
       }
     }
   }
@@ -704,7 +720,7 @@ cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk
 
 cudaError_t launch_quant(const QuantArgs& a, int batch, int num_sms, cudaStream_t st) {
   if (a.rows == 0 || a.cols == 0 || batch == 0) return cudaSuccess;
-  if (a.tma_load && a.tma_store && (a.mx ? (a.do_row && a.do_col) : (a.do_col && !a.do_row))) {
+  if (a.tma_load && a.tma_store && (a.mx ? a.do_row : (a.do_col && !a.do_row))) {
     const int64_t tiles = (a.rows / QT_ROWS) * (a.cols / QT_COLS) * batch;
     cudaError_t e = cudaFuncSetAttribute(quant_w_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QW_SMEM);
     if (e != cudaSuccess) return e;

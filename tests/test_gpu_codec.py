@@ -34,6 +34,7 @@ def _spread_bf16(rows, cols, seed):
 @pytest.mark.parametrize("rows,cols,colwise,mma", [
     (32, 32, True, False), (64, 128, True, False), (100, 96, False, False), (256, 384, True, False),
     (128, 256, True, True), (384, 1024, True, True), (1000, 4096, False, False), (4096, 512, True, True),
+    (256, 512, False, True), (4096, 384, False, True),   # row-wise only through the TMA-fed kernel
 ])
 def test_quantize_bit_exact(rows, cols, colwise, mma):
     x = _spread_bf16(rows, cols, seed=rows + cols)
