@@ -235,6 +235,52 @@ def measure_peaks(args):
     print(json.dumps(out))
 
 
+# ------------------------------------------------------------------------------ context: torch loop
+def torch_loop_context(cfg, device: int, steps: int = 5, warmup: int = 2):
+    """The pages' baseline structure (ai4snews paragraph 1; sitech.ge "Grouped experts instead of a
+    Python loop"): a Python loop over experts, each gathering its tokens and running
+    gate_up -> SwiGLU * p -> down with plain PyTorch BF16 ops (cuBLAS GEMMs), autograd for the
+    backward.  Timed on the same GPU and workload shape as context for the grouped path; it is a
+    library path, not this build's kernels.  Returns TFLOP/s and ms per fwd+bwd step."""
+    dev = torch.device("cuda", device)
+    inp = workloads.make_inputs(cfg, with_dy=True)
+    x = inp["x"].to(dev)
+    idx = inp["topk_idx"].to(dev).long()
+    prob = inp["topk_prob"].to(dev).to(torch.bfloat16)
+    dy = inp["dy"].to(dev)
+    w1 = inp["w_gate_up"].to(dev).requires_grad_(True)
+    w2 = inp["w_down"].to(dev).requires_grad_(True)
+    f = cfg.f
+
+    def step():
+        xs = x.detach().requires_grad_(True)
+        p = prob.detach().requires_grad_(True)
+        y = torch.zeros_like(xs)
+        for e in range(cfg.E):
+            tok, j = torch.where(idx == e)
+            if tok.numel() == 0:
+                continue
+            h = xs[tok] @ w1[e].t()
+            a = torch.nn.functional.silu(h[:, :f]) * h[:, f:] * p[tok, j].unsqueeze(1)
+            y = y.index_add(0, tok, a @ w2[e].t())
+        y.backward(dy)
+        w1.grad = None
+        w2.grad = None
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    return {"kind": "torch per-expert loop, bf16, autograd (cuBLAS GEMMs)", "tflops": round(cfg.flops_fwd_bwd() / (ms * 1e-3) / 1e12, 1),
+            "ms_per_step": round(ms, 3), "steps": steps}
+
+
 # ------------------------------------------------------------------------------ replicas
 def max_over_ranks(value: float, world: int, device=None) -> float:
     """Largest ``value`` over all ranks (the job's step time is the slowest replica's)."""
@@ -289,12 +335,12 @@ def run_ours(args, cfg, rank, world, local_rank):
     # the tensor peak of this GPU, measured live just before the timed region: a 0.1 s burst, and a
     # run as long as the timed region itself (same power-cap and clock regime as the GEMMs in it)
     stream0 = torch.cuda.current_stream(dev)
-    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    w0.record(stream0)
+    est0, est1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    est0.record(stream0)
     step(x, idx, prob, dy)
-    w1.record(stream0)
+    est1.record(stream0)
     torch.cuda.synchronize(dev)
-    timed_ms_est = w0.elapsed_time(w1) * args.steps
+    timed_ms_est = est0.elapsed_time(est1) * args.steps
     peak_burst, _ = tensor_peak(moe, local_rank, cfg.precision, 100.0)
     loop_tflops, loop_ms = tensor_peak(moe, local_rank, cfg.precision, min(max(timed_ms_est, 100.0), 4000.0))
     step(x, idx, prob, dy)
@@ -468,6 +514,8 @@ def main():
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling cases)")
     ap.add_argument("--clocks-dir", default=tempfile.gettempdir(), help="where the nvidia-smi clock samples go")
     ap.add_argument("--peaks", action="store_true", help="measure the tensor-core peak loop (burst and sustained)")
+    ap.add_argument("--context-torch-loop", action="store_true",
+                    help="also time a plain PyTorch per-expert loop (BF16, autograd) on the same workload shape")
     args = ap.parse_args()
     if args.peaks:
         measure_peaks(args)
@@ -525,6 +573,8 @@ def main():
             "tokens_per_s": round(world * cfg.T / (res["ms"] * 1e-3), 1),
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["launches"],
             "clocks": res["clocks"], "tensor_peaks": res["tensor_peaks"], "kernels": res["kernels"]}
+    if args.context_torch_loop and world == 1:
+        line["context_torch_loop"] = torch_loop_context(workloads.scaled_config(cfg, precision="bf16"), local_rank)
     print(json.dumps(line))
 
 
