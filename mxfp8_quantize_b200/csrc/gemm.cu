@@ -11,12 +11,12 @@
 // loop while handling uneven counts in one launch (andresseo.expert, "Fragmented Expert
 // Kernels") is what the tile list provides.
 //
-// One CTA per SM, 4 + EPI_WARPS warps:
+// One CTA per SM, LEAD + EPI_WARPS warps:
 //   warp 0  TMA producer (one thread): operand tiles + scale tiles into a STAGES-deep smem ring
 //           (scale tiles as 3-D tensor-map boxes over the tile-layout scale buffers)
 //   warp 1  MMA issuer (one thread): scale tiles smem->TMEM, 4 MMAs per stage, commits
-//   warp 2  TMEM allocator
-//   warps 4.. epilogue: TMEM -> registers -> fused math -> global stores
+//   warp 2  TMEM allocator (warp 0 when LEAD = 2)
+//   warps LEAD.. epilogue: TMEM -> registers -> fused math -> global stores
 // The bf16-store and gate_up kernels use 128 x 256 tiles with one TMEM accumulator (two
 // 256-column accumulators would leave no room for the per-stage scale tiles); the dSwiGLU kernel
 // uses 128 x 128 tiles with two, so that its heavy epilogue overlaps the next tile's MMAs.  Plain
@@ -40,13 +40,17 @@ constexpr uint32_t TMEM_COLS = 512;
 // Tile shape and thread layout of one kernel instance.
 //   EPI_WARPS epilogue warps (a multiple of 4: each TMEM lane quadrant gets EPI_WARPS/4 warps that
 //   split the tile's columns); PASS columns per pass of the column-wise transpose buffer.
-template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_, bool HTILE_ = false>
+//   LEAD warps before the epilogue warps: 4 (producer, MMA issuer, TMEM allocator, idle) or 2 (the
+//   producer's warp also allocates TMEM), the latter leaving more registers per thread.
+template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_, bool HTILE_ = false, int LEAD_ = 4>
 struct Shape {
   static constexpr int BN = BN_;
   static constexpr int NBUF = NBUF_;
   static constexpr int STAGES = STAGES_;
   static constexpr int EPI_WARPS = EPI_WARPS_;
-  static constexpr int NUM_THREADS = 32 * (4 + EPI_WARPS);
+  static constexpr int LEAD = LEAD_;
+  static constexpr int ALLOC_WARP = LEAD == 4 ? 2 : 0;
+  static constexpr int NUM_THREADS = 32 * (LEAD + EPI_WARPS);
   static constexpr int PASS = PASS_;
   static constexpr int PITCH = PASS + 1;  // odd pitch: conflict-free row writes and column reads
   static constexpr int A_BYTES = BM * 128;
@@ -66,7 +70,7 @@ struct Shape {
   static constexpr int SMEM_DYN = OFF_STAGING + EPI_WARPS * STAGING_PER_WARP + 1024;
   static_assert(NBUF * BN + STAGES * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
   static_assert(SMEM_DYN + 4096 <= 232448, "shared memory budget");
-  static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0, "thread layout");
+  static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0 && (LEAD == 4 || LEAD == 2), "thread layout");
 };
 using ShapeStore = Shape<256, 1, 4, false, 8, 16>;    // plain bf16-store epilogues
 using ShapeSwiglu = Shape<256, 1, 4, true, 16, 8>;    // gate_up + ScaledSwiGLU: one 32-column group per thread
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     }
     if (S::HTILE) ptx::prefetch_tmap(&g.tmap_h);
   }
-  if (warp == 2) {
+  if (warp == S::ALLOC_WARP) {
     ptx::tmem_alloc(&s.tmem_base, TMEM_COLS);
     ptx::tmem_relinquish();
   }
@@ -449,13 +453,13 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       volatile int never = 0;
       ptx::mbar_wait(&s.drain, 0, &never, lim);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= S::LEAD) {
     // ================= epilogue
-    const int q = warp & 3;          // TMEM lane quadrant this warp may read
-    const int ch = (warp - 4) >> 2;  // which of the quadrant's EPI_WARPS/4 column parts this warp owns
+    const int q = warp & 3;               // TMEM lane quadrant this warp may read
+    const int ch = (warp - S::LEAD) >> 2;  // which of the quadrant's EPI_WARPS/4 column parts this warp owns
     constexpr int NPART = S::EPI_WARPS / 4;
     float* stage_buf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(staging_base) +
-                                                (warp - 4) * S::STAGING_PER_WARP);
+                                                (warp - S::LEAD) * S::STAGING_PER_WARP);
     const EpiArgs& ep = g.epi;
     int local = 0;
     for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
@@ -667,7 +671,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
 
   __syncthreads();
   if (threadIdx.x == 0 && s.abort_flag) atomicOr(g.status, kStatusTimeout);
-  if (warp == 2) {
+  if (warp == S::ALLOC_WARP) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TMEM_COLS);
   }
