@@ -35,6 +35,11 @@ Precision modes and the readings they encode:
   the OCP floor shared-exponent rule (``scale_rule="floor"``) in every
   quantisation, and E5M2 elements for the gradient operands dy and dh of the
   backward GEMMs (``grad_format="e5m2"``; weights and activations stay E4M3).
+  Memory variant for long sequences (andresseo.expert "Memory Pressure From
+  Long Sequences"; sitech.ge "Memory and quantization overhead"): h saved as
+  MXFP8 instead of bf16 (``saved_h="mxfp8"``: E4M3, blocks of 32 along 2f,
+  which never straddle the gate and up halves since f % 32 == 0); the
+  backward then reads g and u dequantised from it.
 * "bf16": the same chain with bf16 GEMM operands (a, dh rounded to bf16) and
   fp32 products.
 * "fp64": no quantisation and no rounding anywhere (used to pin the algebra
@@ -114,10 +119,13 @@ def _combine(rows_perm, src_to_sorted, T, k, precision):
 
 
 def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: int = 128, scale_rule: str = "ceil",
-            grad_format: str = "e4m3"):
+            grad_format: str = "e4m3", saved_h: str = "bf16"):
     """Returns (y [T, d], state) with the intermediates the backward needs.  ``scale_rule`` is the
     MXFP8 shared-exponent rule of every quantisation (forward and backward); ``grad_format`` the
-    element format of the gradient operands (dy, dh) of the four backward GEMMs."""
+    element format of the gradient operands (dy, dh) of the four backward GEMMs; ``saved_h`` the
+    format h is kept in for the backward ("bf16" or "mxfp8")."""
+    if saved_h not in ("bf16", "mxfp8"):
+        raise ValueError(saved_h)
     x = np.asarray(x, dtype=np.float64)
     T, d = x.shape
     E, two_f, _ = w_gate_up.shape
@@ -161,7 +169,8 @@ def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: in
         p_perm[lo:hi] = pe
     y = _combine(y_perm, r["src_to_sorted"], T, k, precision)
     state = dict(route=r, x_perm=x_perm, p_perm=p_perm, h=h_all, a=a_all, y_perm=y_perm,
-                 T=T, d=d, f=f, E=E, k=k, precision=precision, scale_rule=scale_rule, grad_format=grad_format)
+                 T=T, d=d, f=f, E=E, k=k, precision=precision, scale_rule=scale_rule, grad_format=grad_format,
+                 saved_h=saved_h)
     return y, state
 
 
@@ -198,8 +207,8 @@ def backward(dy, state, w_gate_up, w_down):
         pe = state["p_perm"][lo:hi][:, None]
         a = state["a"][lo:hi].astype(np.float64)
         h = state["h"][lo:hi]
-        if precision != "fp64":
-            h = bf16_round(h)           # the backward reads h as saved (bf16)
+        if precision != "fp64":          # the backward reads h as saved: bf16, or MXFP8 along 2f
+            h = bf16_round(h) if state.get("saved_h", "bf16") == "bf16" else mx.fake_quant(h, axis=1, rule=rule)
         g, u = h[:, :f].astype(np.float64), h[:, f:].astype(np.float64)
         W1 = np.asarray(w_gate_up[e], dtype=np.float64)
         W2 = np.asarray(w_down[e], dtype=np.float64)

@@ -137,11 +137,14 @@ class _ScaledSwiGLU(torch.autograd.Function):
         f = h.shape[1] // 2
         return _to_f32(torch.nn.functional.silu(h[:, :f]) * h[:, f:] * p)
 
+    saved_h = "bf16"   # format h is read back in for the backward ("mxfp8": E4M3 blocks of 32 along 2f)
+
     @staticmethod
     def backward(ctx, da):
         h, p = ctx.saved_tensors
         f = h.shape[1] // 2
-        hb = _to_bf16(h).detach().requires_grad_(True)
+        hs = _fq_mx(h, 1) if _ScaledSwiGLU.saved_h == "mxfp8" else _to_bf16(h)
+        hb = hs.detach().requires_grad_(True)
         pp = p.detach().requires_grad_(True)
         with torch.enable_grad():
             a = torch.nn.functional.silu(hb[:, :f]) * hb[:, f:] * pp
@@ -220,22 +223,29 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("mode", ["mxfp8", "bf16", "mxfp8-floor", "mxfp8-e5m2grad"])
+@pytest.mark.parametrize("mode", ["mxfp8", "bf16", "mxfp8-floor", "mxfp8-e5m2grad", "mxfp8-savedh"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"T{s['T']}_E{s['E']}_k{s['k']}_{s['routing']}")
 def test_quantised_backward_matches_straight_through_autograd(shape, mode):
     """mxfp8-floor: the oracle's OCP floor shared-exponent variant, in every quantisation;
-    mxfp8-e5m2grad: E5M2 elements for the gradient operand of every backward product."""
+    mxfp8-e5m2grad: E5M2 elements for the gradient operand of every backward product;
+    mxfp8-savedh: h kept as MXFP8 for the backward (the long-sequence memory variant)."""
     inp = _inputs(**shape)
     args = [inp[n] for n in ("x", "topk_idx", "topk_prob", "w_gate_up", "w_down")]
     if mode == "mxfp8-floor":
         y, st = moe.forward(*args, "mxfp8", scale_rule="floor")
     elif mode == "mxfp8-e5m2grad":
         y, st = moe.forward(*args, "mxfp8", grad_format="e5m2")
+    elif mode == "mxfp8-savedh":
+        y, st = moe.forward(*args, "mxfp8", saved_h="mxfp8")
     else:
         y, st = moe.forward(*args, mode)
     got = moe.backward(inp["dy"], st, inp["w_gate_up"], inp["w_down"])
     got["y"] = y
-    ref = _reference(*args, inp["dy"], mode)
+    _ScaledSwiGLU.saved_h = "mxfp8" if mode == "mxfp8-savedh" else "bf16"
+    try:
+        ref = _reference(*args, inp["dy"], "mxfp8" if mode == "mxfp8-savedh" else mode)
+    finally:
+        _ScaledSwiGLU.saved_h = "bf16"
     got["dh_slot"] = got["dh_perm"][st["route"]["src_to_sorted"]]
     for name in ("y", "dx", "dw_gate_up", "dw_down", "d_topk_prob", "dh_slot"):
         r = ref[name].numpy()
