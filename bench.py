@@ -309,10 +309,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     w1 = inp["w_gate_up"].to(dev)
     w2 = inp["w_down"].to(dev)
     T, d, f, E, k = cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
-    sz = moe.sizes(T, d, f, E, k, cfg.precision, True)
+    sz = moe.sizes(T, d, f, E, k, cfg.precision, True, args.saved_h)
     fws = torch.empty(sz["fwd_ws"], dtype=torch.uint8, device=dev)
     bws = torch.empty(sz["bwd_ws"], dtype=torch.uint8, device=dev)
-    saved = moe.Saved(torch.empty(sz["saved"], dtype=torch.uint8, device=dev), (T, d, f, E, k, cfg.precision))
+    saved = moe.Saved(torch.empty(sz["saved"], dtype=torch.uint8, device=dev), (T, d, f, E, k, cfg.precision),
+                      args.saved_h)
     y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     dx = torch.empty_like(y)
     dw1 = torch.empty_like(w1)
@@ -321,7 +322,7 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     def step(xi, idxi, probi, dyi, yo=y, dxo=dx, dpo=dp):
         moe.moe_grouped_mlp_fwd(xi, idxi, probi, w1, w2, precision=cfg.precision, training=True, workspace=fws,
-                                saved=saved, y=yo)
+                                saved=saved, y=yo, saved_h=args.saved_h)
         moe.moe_grouped_mlp_bwd(dyi, saved, w1, w2, workspace=bws, dx=dxo, dw_gate_up=dw1, dw_down=dw2,
                                 d_topk_prob=dpo)
 
@@ -490,7 +491,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     tensor_peaks = {"matched_tflops": round(loop_tflops, 1), "matched_ms": round(loop_ms, 1),
                     "burst_tflops": round(peak_burst, 1), "nominal_rule_tflops": round(nominal_rule, 1)}
     return dict(ms=ms, kernels=kern, roofline=roofline, clocks=clk, e2e=e2e, launches=launches,
-                tensor_peaks=tensor_peaks)
+                tensor_peaks=tensor_peaks, memory={"saved_h": args.saved_h, "saved_bytes": sz["saved"],
+                                                   "fwd_workspace_bytes": sz["fwd_ws"], "bwd_workspace_bytes": sz["bwd_ws"]})
 
 
 def config_desc(cfg):
@@ -514,6 +516,8 @@ def main():
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling cases)")
     ap.add_argument("--clocks-dir", default=tempfile.gettempdir(), help="where the nvidia-smi clock samples go")
     ap.add_argument("--peaks", action="store_true", help="measure the tensor-core peak loop (burst and sustained)")
+    ap.add_argument("--saved-h", default="bf16", choices=["bf16", "mxfp8"],
+                    help="format h is saved in for the backward (long-sequence memory mode)")
     ap.add_argument("--context-torch-loop", action="store_true",
                     help="also time a plain PyTorch per-expert loop (BF16, autograd) on the same workload shape")
     args = ap.parse_args()
@@ -572,7 +576,8 @@ def main():
             "data": "synthetic", "config": config_desc(cfg),
             "tokens_per_s": round(world * cfg.T / (res["ms"] * 1e-3), 1),
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["launches"],
-            "clocks": res["clocks"], "tensor_peaks": res["tensor_peaks"], "kernels": res["kernels"]}
+            "clocks": res["clocks"], "tensor_peaks": res["tensor_peaks"], "memory": res["memory"],
+            "kernels": res["kernels"]}
     if args.context_torch_loop and world == 1:
         line["context_torch_loop"] = torch_loop_context(workloads.scaled_config(cfg, precision="bf16"), local_rank)
     print(json.dumps(line))

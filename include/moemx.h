@@ -108,6 +108,20 @@ moe_status_t moe_ctx_set_scale_rule(moe_ctx_t ctx, int rule);
  * E4M3 B operand (weights, a, x).  The forward is unchanged. */
 moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt);
 
+/* Format of the gate/up pre-activations h that a training forward with this context saves for the
+ * backward (the backward must run with the same setting).  Long sequences make h the largest saved
+ * tensor (4*T*k*f bytes in bf16; andresseo.expert "Memory Pressure From Long Sequences", sitech.ge
+ * "Memory and quantization overhead"):
+ *   MOE_SAVED_H_BF16  (default) bf16 h [capacity, 2f];
+ *   MOE_SAVED_H_MXFP8 MXFP8 h: E4M3 codes [capacity, 2f] with one E8M0 scale per 32 values along
+ *                     2f (row-major [capacity, 2f/32]), quantised in the gate_up GEMM's epilogue with
+ *                     the context's scale rule; the dSwiGLU epilogue reads g and u dequantised from
+ *                     it.  About half the bytes; MXFP8 precision only (MOE_ERR_UNSUPPORTED for BF16).
+ * moe_saved_size_ex gives the saved-buffer size for a mode. */
+#define MOE_SAVED_H_BF16 0
+#define MOE_SAVED_H_MXFP8 1
+moe_status_t moe_ctx_set_saved_h(moe_ctx_t ctx, int mode);
+
 /* Test hook for the bounded in-kernel waits (tests only).  With ``stall`` non-zero, every CTA of
  * the persistent kernels (the grouped GEMMs and the TMA-fed quantiser) makes one extra wait on a
  * word of the context's status block that nothing ever sets, bounded by ``limit_cycles`` SM clock
@@ -220,6 +234,9 @@ moe_status_t moe_unpermute(moe_ctx_t ctx, const void* y_perm, const int32_t* src
  * Neither may be shared by two calls in flight at once.
  */
 size_t moe_saved_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec);
+/* Saved-buffer size when h is saved in format ``saved_h`` (see moe_ctx_set_saved_h); 0 for an
+ * unsupported combination. */
+size_t moe_saved_size_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int saved_h);
 size_t moe_fwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training);
 size_t moe_bwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec);
 
@@ -287,7 +304,7 @@ double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters)
  * a forward workspace (which = 1) or a backward workspace (which = 2) laid out for these
  * dimensions, given the buffer's base address ``base``; NULL for an unknown name.  Names:
  * saved: split_sizes poffsets sorted_to_src src_to_sorted prob_perm w1c_q w1c_s w2c_q w2c_s
- *        xT_q xT_s aT_q aT_s xT aT h
+ *        xT_q xT_s aT_q aT_s xT aT h (h_q h_s with moe_buffer_address_ex and MOE_SAVED_H_MXFP8)
  * forward workspace: w1_q w1_s w2_q w2_s x_q x_s a_q a_s x_perm a y_perm (+ the routing names
  *        when training == 0)
  * backward workspace: dy_q dy_s dyT_q dyT_s dh_q dh_s dhT_q dhT_s dy_perm dyT dh dhT w1T w2T
@@ -295,6 +312,9 @@ double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters)
  * Scales (*_s) are in the tensor-core tile layout described at mxfp8_quantize. */
 void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
                          int which, void* base, const char* name);
+/* The same for a saved buffer laid out for the saved-h format ``saved_h``. */
+void* moe_buffer_address_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
+                            int saved_h, int which, void* base, const char* name);
 
 #ifdef __cplusplus
 }

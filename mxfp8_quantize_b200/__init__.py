@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(HERE, "libmoemx.so")
 MOE_ROW_ALIGN = 128
 MXFP8_ROWWISE, MXFP8_COLWISE_T, MXFP8_SF_MMA_LAYOUT, MXFP8_FLAG_SCALE_FLOOR, MXFP8_FLAG_E5M2 = 1, 2, 4, 8, 16
 GRAD_FORMATS = {"e4m3": 0, "e5m2": 1}
+SAVED_H = {"bf16": 0, "mxfp8": 1}
 SCALE_RULES = {"ceil": 0, "floor": 1}
 PRECISIONS = {"bf16": 0, "mxfp8": 1}
 STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "unsupported", 4: "cuda", 5: "device", 6: "timeout",
@@ -33,7 +34,7 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_get_status", "moe_ctx_set_d
            "moe_saved_size", "moe_fwd_workspace_size", "moe_bwd_workspace_size", "moe_grouped_mlp_fwd",
            "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook", "moe_grouped_mlp_fwd_noalloc",
            "moe_ctx_set_test_stall", "moe_tensor_peak_loop", "moe_tensor_peak_flops", "moe_ctx_set_scale_rule",
-           "moe_ctx_set_grad_format"]
+           "moe_ctx_set_grad_format", "moe_ctx_set_saved_h", "moe_saved_size_ex", "moe_buffer_address_ex"]
 
 LAUNCH_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
@@ -66,6 +67,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ctx_set_test_stall": (c_int, [c_vp, c_int, c_i64]),
         "moe_ctx_set_scale_rule": (c_int, [c_vp, c_int]),
         "moe_ctx_set_grad_format": (c_int, [c_vp, c_int]),
+        "moe_ctx_set_saved_h": (c_int, [c_vp, c_int]),
+        "moe_saved_size_ex": (c_size, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int]),
+        "moe_buffer_address_ex": (c_vp, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_vp,
+                                         ctypes.c_char_p]),
         "moe_tensor_peak_loop": (c_int, [c_vp, c_int, c_i64, c_int, c_vp]),
         "moe_tensor_peak_flops": (ctypes.c_double, [c_vp, c_int, c_i64]),
         "moe_status_string": (ctypes.c_char_p, [c_int]),
@@ -267,28 +272,30 @@ def _ptr_array(ws: Weights, E: int):
 
 
 class Saved:
-    """Opaque buffer a training forward leaves for the backward, plus the call's dimensions."""
+    """Opaque buffer a training forward leaves for the backward, plus the call's dimensions and the
+    format h was saved in."""
 
-    def __init__(self, buf: torch.Tensor, dims: tuple):
+    def __init__(self, buf: torch.Tensor, dims: tuple, saved_h: str = "bf16"):
         self.buf = buf
         self.dims = dims
+        self.saved_h = saved_h
 
 
-def sizes(T: int, d: int, f: int, E: int, k: int, precision: str, training: bool):
+def sizes(T: int, d: int, f: int, E: int, k: int, precision: str, training: bool, saved_h: str = "bf16"):
     L = load_library()
     p = PRECISIONS[precision]
-    return dict(saved=int(L.moe_saved_size(T, k, E, d, f, p)),
+    return dict(saved=int(L.moe_saved_size_ex(T, k, E, d, f, p, SAVED_H[saved_h])),
                 fwd_ws=int(L.moe_fwd_workspace_size(T, k, E, d, f, p, int(training))),
                 bwd_ws=int(L.moe_bwd_workspace_size(T, k, E, d, f, p)))
 
 
 def buffer_view(buf: torch.Tensor, which: int, name: str, dims: tuple, training: bool, nbytes: int,
-                dtype=torch.uint8) -> torch.Tensor:
+                dtype=torch.uint8, saved_h: str = "bf16") -> torch.Tensor:
     """A view of the named intermediate inside ``buf`` (a saved / workspace buffer); tests only."""
     T, d, f, E, k, precision = dims
     L = load_library()
-    p = L.moe_buffer_address(T, k, E, d, f, PRECISIONS[precision], int(training), which, buf.data_ptr(),
-                             name.encode())
+    p = L.moe_buffer_address_ex(T, k, E, d, f, PRECISIONS[precision], int(training), SAVED_H[saved_h], which,
+                                buf.data_ptr(), name.encode())
     if not p:
         raise KeyError(name)
     off = p - buf.data_ptr()
@@ -299,26 +306,31 @@ def buffer_view(buf: torch.Tensor, which: int, name: str, dims: tuple, training:
 def moe_grouped_mlp_fwd(x: torch.Tensor, topk_idx: torch.Tensor, topk_prob: torch.Tensor, w_gate_up: Weights,
                         w_down: Weights, precision: str = "mxfp8", training: bool = False,
                         split_sizes: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                        saved: Optional[Saved] = None, y: Optional[torch.Tensor] = None):
+                        saved: Optional[Saved] = None, y: Optional[torch.Tensor] = None, saved_h: str = "bf16"):
     """y = sum_j p_j * W2_e (silu(W1g_e x) * W1u_e x) over each token's k experts.
 
     Returns (y, saved) where saved is a Saved for the backward when ``training`` else None.
+    ``saved_h``: the format h is saved in for the backward ("bf16" or "mxfp8").
     """
     dev = _device_index(x)
     T, d = x.shape
     E = len(w_gate_up)
     f = w_down[0].shape[1]
     k = topk_idx.shape[1]
-    sz = sizes(T, d, f, E, k, precision, training)
+    sz = sizes(T, d, f, E, k, precision, training, saved_h)
     if sz["fwd_ws"] == 0:
         raise MoeError("moe_grouped_mlp_fwd (sizes)", 2)
     if workspace is None:
         workspace = torch.empty(sz["fwd_ws"], dtype=torch.uint8, device=x.device)
     if training and saved is None:
-        saved = Saved(torch.empty(sz["saved"], dtype=torch.uint8, device=x.device), (T, d, f, E, k, precision))
+        saved = Saved(torch.empty(sz["saved"], dtype=torch.uint8, device=x.device), (T, d, f, E, k, precision),
+                      saved_h)
+    if training:
+        saved.saved_h = saved_h
     if y is None:
         y = torch.empty((T, d), dtype=torch.bfloat16, device=x.device)
     L = load_library()
+    _check("moe_ctx_set_saved_h", L.moe_ctx_set_saved_h(context(dev), SAVED_H[saved_h] if training else 0))
     _check("moe_grouped_mlp_fwd", L.moe_grouped_mlp_fwd(
         context(dev), x.data_ptr(), topk_idx.data_ptr(), topk_prob.data_ptr(), _ptr(split_sizes),
         _ptr_array(w_gate_up, E), _ptr_array(w_down, E), T, d, f, E, k, PRECISIONS[precision], int(training),
@@ -371,6 +383,7 @@ def moe_grouped_mlp_bwd(dy: torch.Tensor, saved: Saved, w_gate_up: Weights, w_do
     if d_topk_prob is None:
         d_topk_prob = torch.empty((T, k), dtype=torch.float32, device=dy.device)
     L = load_library()
+    _check("moe_ctx_set_saved_h", L.moe_ctx_set_saved_h(context(dev), SAVED_H[saved.saved_h]))
     _check("moe_grouped_mlp_bwd", L.moe_grouped_mlp_bwd(
         context(dev), dy.data_ptr(), saved.buf.data_ptr(), saved.buf.numel(), _ptr_array(w_gate_up, E),
         _ptr_array(w_down, E), T, d, f, E, k, PRECISIONS[precision], dx.data_ptr(), _ptr_array(dw_gate_up, E),

@@ -23,6 +23,7 @@ struct moe_ctx_s {
   void* hook_user;
   int scale_floor;          // MXFP8 shared-exponent rule of the fused layer (moe_ctx_set_scale_rule)
   int grad_e5m2;            // MXFP8 gradient operands in E5M2 (moe_ctx_set_grad_format)
+  int saved_h;              // format of the h a training forward saves (moe_ctx_set_saved_h)
   int stall;                // test hook for the bounded waits (moe_ctx_set_test_stall)
   long long stall_limit;
 };
@@ -197,6 +198,7 @@ struct Dims {
   int64_t T, d, f, cap, Tk;
   int E, k;
   bool mx;
+  int saved_h;  // MOE_SAVED_H_BF16 or MOE_SAVED_H_MXFP8
 };
 
 // Everything a training forward leaves for the backward.
@@ -206,7 +208,8 @@ struct Saved {
   uint8_t *w1c_q, *w1c_s, *w2c_q, *w2c_s;  // MXFP8: weights quantised down the columns, transposed
   uint8_t *xT_q, *xT_s, *aT_q, *aT_s;      // MXFP8: token-axis quantised x and a, transposed
   bf16 *xT, *aT;                           // BF16: transposed copies
-  bf16* h;                                 // [cap, 2f] gate/up pre-activations
+  bf16* h;                                 // [cap, 2f] gate/up pre-activations (bf16) ...
+  uint8_t *h_q, *h_s;                      // ... or as MXFP8: codes [cap, 2f], scales [cap, 2f/32]
 };
 void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
   s.split = c.take<int32_t>(D.E * 4);
@@ -217,6 +220,7 @@ void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
   s.w1c_q = s.w1c_s = s.w2c_q = s.w2c_s = s.xT_q = s.xT_s = s.aT_q = s.aT_s = nullptr;
   s.xT = s.aT = nullptr;
   s.h = nullptr;
+  s.h_q = s.h_s = nullptr;
   if (!full) return;  // inference: routing bookkeeping only
   if (D.mx) {
     s.w1c_q = c.take<uint8_t>(D.E * D.d * 2 * D.f);
@@ -231,7 +235,12 @@ void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
     s.xT = c.take<bf16>(D.d * D.cap * 2);
     s.aT = c.take<bf16>(D.f * D.cap * 2);
   }
-  s.h = c.take<bf16>(D.cap * 2 * D.f * 2);
+  if (D.saved_h == MOE_SAVED_H_MXFP8) {
+    s.h_q = c.take<uint8_t>(D.cap * 2 * D.f);
+    s.h_s = c.take<uint8_t>(D.cap * 2 * D.f / 32);
+  } else {
+    s.h = c.take<bf16>(D.cap * 2 * D.f * 2);
+  }
 }
 
 struct FwdWs {
@@ -300,8 +309,9 @@ moe_status_t check_dims(int64_t T, int64_t d, int64_t f, int E, int k) {
   return MOE_OK;
 }
 
-Dims make_dims(int64_t T, int64_t d, int64_t f, int E, int k, moe_precision_t prec) {
+Dims make_dims(int64_t T, int64_t d, int64_t f, int E, int k, moe_precision_t prec, int saved_h = 0) {
   Dims D;
+  D.saved_h = saved_h;
   D.T = T;
   D.d = d;
   D.f = f;
@@ -414,6 +424,7 @@ moe_status_t moe_ctx_create(moe_ctx_t* out, int device) {
   c->hook_user = nullptr;
   c->scale_floor = 0;
   c->grad_e5m2 = 0;
+  c->saved_h = MOE_SAVED_H_BF16;
   c->stall = 0;
   c->stall_limit = 0;
   if (cudaMalloc(&c->d_status, 256) != cudaSuccess) {
@@ -467,6 +478,12 @@ moe_status_t moe_ctx_set_scale_rule(moe_ctx_t ctx, int rule) {
 moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt) {
   if (!ctx || (fmt != MOE_GRAD_E4M3 && fmt != MOE_GRAD_E5M2)) return MOE_ERR_INVALID_ARG;
   ctx->grad_e5m2 = fmt == MOE_GRAD_E5M2 ? 1 : 0;
+  return MOE_OK;
+}
+
+moe_status_t moe_ctx_set_saved_h(moe_ctx_t ctx, int mode) {
+  if (!ctx || (mode != MOE_SAVED_H_BF16 && mode != MOE_SAVED_H_MXFP8)) return MOE_ERR_INVALID_ARG;
+  ctx->saved_h = mode;
   return MOE_OK;
 }
 
@@ -578,13 +595,18 @@ moe_status_t moe_unpermute(moe_ctx_t ctx, const void* y_perm, const int32_t* src
   return MOE_OK;
 }
 
-size_t moe_saved_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec) {
+size_t moe_saved_size_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int saved_h) {
   if (check_dims(T, d, f, E, k) != MOE_OK) return 0;
-  Dims D = make_dims(T, d, f, E, k, prec);
+  if (saved_h != MOE_SAVED_H_BF16 && (saved_h != MOE_SAVED_H_MXFP8 || prec != MOE_PREC_MXFP8)) return 0;
+  Dims D = make_dims(T, d, f, E, k, prec, saved_h);
   Carve c(nullptr);
   Saved s;
   carve_saved(c, D, s);
   return c.off + 1024;
+}
+
+size_t moe_saved_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec) {
+  return moe_saved_size_ex(T, k, E, d, f, prec, MOE_SAVED_H_BF16);
 }
 
 size_t moe_fwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training) {
@@ -622,12 +644,14 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
   for (int e = 0; e < E; ++e)
     if (!w_gate_up[e] || !w_down[e] || !aligned16(w_gate_up[e]) || !aligned16(w_down[e])) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  const int saved_h = training ? ctx->saved_h : MOE_SAVED_H_BF16;
+  if (saved_h == MOE_SAVED_H_MXFP8 && prec != MOE_PREC_MXFP8) return MOE_ERR_UNSUPPORTED;
   if (workspace_bytes < moe_fwd_workspace_size(T, k, E, d, f, prec, training)) return MOE_ERR_WORKSPACE;
-  if (training && saved_bytes < moe_saved_size(T, k, E, d, f, prec)) return MOE_ERR_WORKSPACE;
+  if (training && saved_bytes < moe_saved_size_ex(T, k, E, d, f, prec, saved_h)) return MOE_ERR_WORKSPACE;
 
   DeviceGuard guard(ctx->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Dims D = make_dims(T, d, f, E, k, prec);
+  const Dims D = make_dims(T, d, f, E, k, prec, saved_h);
   Carve cw(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(workspace), 1024)));
   FwdWs w;
   carve_fwd(cw, D, w);
@@ -774,7 +798,9 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     ep.f = f;
     ep.cap = D.cap;
     ep.p_perm = s.pperm;
-    ep.h = training ? s.h : nullptr;
+    ep.h = training ? s.h : nullptr;  // (null when h is saved as MXFP8)
+    ep.h_q = training ? s.h_q : nullptr;
+    ep.h_s = training ? s.h_s : nullptr;
     ep.dump = ctx->dbg_a;
     if (D.mx) {
       ep.q_row = w.a_q;
@@ -829,12 +855,14 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
         !aligned16(dw_down[e]) || !aligned16(w_gate_up[e]) || !aligned16(w_down[e]))
       return MOE_ERR_INVALID_ARG;
   if (!aligned16(dy) || !aligned16(dx)) return MOE_ERR_INVALID_ARG;
-  if (saved_bytes < moe_saved_size(T, k, E, d, f, prec)) return MOE_ERR_WORKSPACE;
+  const int saved_h = ctx->saved_h;
+  if (saved_h == MOE_SAVED_H_MXFP8 && prec != MOE_PREC_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (saved_bytes < moe_saved_size_ex(T, k, E, d, f, prec, saved_h)) return MOE_ERR_WORKSPACE;
   if (workspace_bytes < moe_bwd_workspace_size(T, k, E, d, f, prec)) return MOE_ERR_WORKSPACE;
 
   DeviceGuard guard(ctx->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const Dims D = make_dims(T, d, f, E, k, prec);
+  const Dims D = make_dims(T, d, f, E, k, prec, saved_h);
   Saved s;
   Carve cs(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(saved), 1024)));
   carve_saved(cs, D, s);
@@ -901,7 +929,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     GemmArgs g = gemm_args(ctx);
     const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dy_q) : w.dy_perm, D.mx, d, D.cap, d * es) &&
                     map_3d(&g.tmap_b, w2c, D.mx, d, f, E, d * es, f * d * es, gemm_tile_n(EPI_DSWIGLU)) &&
-                    map_2d(&g.tmap_h, s.h, false, 2 * f, D.cap, 2 * f * 2);  // bf16 boxes of 128 rows x 64 columns
+                    (s.h_q || map_2d(&g.tmap_h, s.h, false, 2 * f, D.cap, 2 * f * 2));  // bf16 boxes, 128 x 64
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
@@ -918,7 +946,9 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     ep.f = f;
     ep.cap = D.cap;
     ep.p_perm = s.pperm;
-    ep.h = s.h;
+    ep.h = s.h;      // bf16 h staged by TMA, or
+    ep.h_q = s.h_q;  // MXFP8 h read by the epilogue (the kernel instance without h staging)
+    ep.h_s = s.h_s;
     ep.dump = ctx->dbg_dh;
     ep.dp_part = w.dp_part;
     ep.grad_e5m2 = ctx->grad_e5m2;  // dh is the gradient operand of both gate_up backward GEMMs
@@ -1027,10 +1057,10 @@ double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters)
   return tensor_peak_flops(prec == MOE_PREC_MXFP8, ctx->num_sms, iters);
 }
 
-void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
-                         int which, void* base, const char* name) {
+void* moe_buffer_address_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
+                            int saved_h, int which, void* base, const char* name) {
   if (!base || !name || check_dims(T, d, f, E, k) != MOE_OK) return nullptr;
-  const Dims D = make_dims(T, d, f, E, k, prec);
+  const Dims D = make_dims(T, d, f, E, k, prec, saved_h);
   Carve c(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(base), 1024)));
   struct Named {
     const char* n;
@@ -1047,7 +1077,7 @@ void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_prec
                          {"src_to_sorted", s.src2s}, {"prob_perm", s.pperm}, {"w1c_q", s.w1c_q},
                          {"w1c_s", s.w1c_s}, {"w2c_q", s.w2c_q}, {"w2c_s", s.w2c_s}, {"xT_q", s.xT_q},
                          {"xT_s", s.xT_s}, {"aT_q", s.aT_q}, {"aT_s", s.aT_s}, {"xT", s.xT}, {"aT", s.aT},
-                         {"h", s.h}};
+                         {"h", s.h},       {"h_q", s.h_q},     {"h_s", s.h_s}};
     for (const Named& e : tab)
       if (!std::strcmp(e.n, name) && e.p) return e.p;
     if (which == 0) return nullptr;
@@ -1075,6 +1105,11 @@ void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_prec
       if (!std::strcmp(e.n, name) && e.p) return e.p;
   }
   return nullptr;
+}
+
+void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
+                         int which, void* base, const char* name) {
+  return moe_buffer_address_ex(T, k, E, d, f, prec, training, MOE_SAVED_H_BF16, which, base, name);
 }
 
 // ---- forward without allocation: file-scope scratch, looked up once per device
@@ -1140,6 +1175,7 @@ moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx,
   c.hook_user = nullptr;
   c.scale_floor = 0;
   c.grad_e5m2 = 0;
+  c.saved_h = MOE_SAVED_H_BF16;
   c.stall = 0;
   c.stall_limit = 0;
   // the scratch base is 256-aligned; the workspace carving aligns to 1 KiB inside the size bound

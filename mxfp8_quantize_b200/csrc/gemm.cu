@@ -26,6 +26,7 @@
 // outputs leave in 256-bit stores (a whole 32-byte sector per lane).
 // Every wait is bounded: on expiry the kernel records MOE_ERR_TIMEOUT and all roles stop; copies
 // and MMAs already issued are waited for before TMEM is freed.
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "gemm.cuh"
@@ -75,6 +76,7 @@ struct Shape {
 using ShapeStore = Shape<256, 1, 4, false, 8, 16>;    // plain bf16-store epilogues
 using ShapeSwiglu = Shape<256, 1, 4, true, 16, 8>;    // gate_up + ScaledSwiGLU: one 32-column group per thread
 using ShapeDswiglu = Shape<128, 2, 4, true, 8, 16, true>;  // dgrad of down + dSwiGLU: epilogue overlaps the next tile
+using ShapeDswigluG = Shape<128, 2, 4, true, 8, 16, false>;  // ... reading the saved h from global memory (MXFP8 h)
 
 struct SharedState {
   uint64_t full[8];
@@ -154,6 +156,26 @@ __device__ __forceinline__ void unpack_bf16x8(uint4 v, float* o) {
     o[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
+// Eight E4M3 codes (bytes of lo then hi) -> fp32 values times ``scale`` (exact: every E4M3 value
+// is an fp16 value, and the scale is a power of two).
+__device__ __forceinline__ void e4m3x8_to_float(uint32_t lo, uint32_t hi, float scale, float* o) {
+  const uint32_t w[2] = {lo, hi};
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __half2_raw r =
+          __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>((w[k] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
+      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&r));
+      o[4 * k + 2 * h] = v.x * scale;
+      o[4 * k + 2 * h + 1] = v.y * scale;
+    }
+}
+// 2^(byte - 127) as an fp32 (byte 0: 2^-127, a subnormal).
+__device__ __forceinline__ float e8m0_scale(uint32_t byte) {
+  return byte ? __uint_as_float(byte << 23) : __uint_as_float(0x00400000u);
+}
+
 // MXFP8 of 32 values with the scale of their own amax: 32 codes (E4M3, or E5M2 when ``e5m2``)
 // stored at q (32-byte aligned); returns the E8M0 byte.
 __device__ __forceinline__ uint32_t quant32_store(const float* v, uint8_t* q, int floor_rule, int e5m2) {
@@ -531,7 +553,12 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
           }
-          if (ep.h) {  // saved gate/up pre-activations: 64 bytes of each per row, in 32-byte stores
+          if (ep.h_q) {  // saved as MXFP8: 32 codes and one scale per 32 gate (and up) values
+            const uint32_t sbg = quant32_store(gv, ep.h_q + row * 2 * f + j, ep.scale_floor, 0);
+            const uint32_t sbu = quant32_store(uv, ep.h_q + row * 2 * f + f + j, ep.scale_floor, 0);
+            ep.h_s[row * (2 * f / 32) + j / 32] = static_cast<uint8_t>(sbg);
+            ep.h_s[row * (2 * f / 32) + (f + j) / 32] = static_cast<uint8_t>(sbu);
+          } else if (ep.h) {  // saved gate/up pre-activations: 64 bytes of each per row, in 32-byte stores
             bf16* hg = ep.h + row * 2 * f + j;
             bf16* hu = hg + f;
 #pragma unroll
@@ -565,9 +592,11 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         const float p = ep.p_perm[row];
         const int64_t f = ep.f, f2 = 2 * ep.f;
         const int64_t j0 = static_cast<int64_t>(tl.nb) * BN + CPT * ch;
+        const bool mxh = !S::HTILE && ep.h_q != nullptr;  // h saved as MXFP8
         const bf16* hrow = ep.h + row * f2;
         // saved gate/up values: 16-byte chunk c (of this thread's 32-column group cc) of the gate part
-        // and of the up part, from the TMA-staged tile in smem (128B-swizzled rows) or from global
+        // and of the up part, from the TMA-staged tile in smem (128B-swizzled rows) or from global.
+        // MXFP8 h: chunks 0 and 1 are the group's 32 codes, chunk 2 holds its scale byte.
         const int rl = 32 * q + lane;  // row within the tile
         auto h_chunk = [&](int up, int cc, int c) -> uint4 {
           if (S::HTILE) {
@@ -576,7 +605,22 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             const int chunk = ((col % 64) / 8) ^ (rl & 7);
             return *reinterpret_cast<const uint4*>(box + rl * 128 + chunk * 16);
           }
+          if (mxh) {
+            const int64_t col = (up ? f : 0) + j0 + 32 * cc;
+            if (c < 2) return reinterpret_cast<const uint4*>(ep.h_q + row * f2 + col)[c];
+            if (c == 2) return make_uint4(ep.h_s[row * (f2 / 32) + col / 32], 0u, 0u, 0u);
+            return make_uint4(0u, 0u, 0u, 0u);
+          }
           return reinterpret_cast<const uint4*>(hrow + (up ? f : 0) + j0 + 32 * cc)[c];
+        };
+        // eight gate (or up) values of chunk i from the group's raw chunks
+        auto h_values = [&](const uint4 (&hv)[4], int i, float* o) {
+          if (mxh) {
+            const uint4 c = hv[i >> 1];
+            e4m3x8_to_float((i & 1) ? c.z : c.x, (i & 1) ? c.w : c.y, e8m0_scale(hv[2].x), o);
+          } else {
+            unpack_bf16x8(hv[i], o);
+          }
         };
         uint4 hg[4], hu[4];
         if (!S::HTILE) {
@@ -612,8 +656,8 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float gg[8], uu[8];
-            unpack_bf16x8(hg[i], gg);
-            unpack_bf16x8(hu[i], uu);
+            h_values(hg, i, gg);
+            h_values(hu, i, uu);
 #pragma unroll
             for (int q8 = 0; q8 < 8; ++q8) {
               const float gx = gg[q8], ux = uu[q8], d = da[8 * i + q8];
@@ -698,6 +742,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_
   if (mx) {
     if (epi == EPI_STORE) return launch_t<true, EPI_STORE, ShapeStore>(args, num_sms, st);
     if (epi == EPI_SWIGLU) return launch_t<true, EPI_SWIGLU, ShapeSwiglu>(args, num_sms, st);
+    if (args.epi.h_q) return launch_t<true, EPI_DSWIGLU, ShapeDswigluG>(args, num_sms, st);
     return launch_t<true, EPI_DSWIGLU, ShapeDswiglu>(args, num_sms, st);
   }
   if (epi == EPI_STORE) return launch_t<false, EPI_STORE, ShapeStore>(args, num_sms, st);

@@ -22,6 +22,8 @@ struct EpiArgs {
   int64_t cap;        // padded row capacity (token axis of the transposed outputs)
   const float* p_perm;
   bf16* h;            // [cap, 2f] saved gate/up pre-activations (written by SWIGLU, read by DSWIGLU)
+  uint8_t* h_q;       // ... or saved as MXFP8 (E4M3 codes [cap, 2f], blocks of 32 along 2f)
+  uint8_t* h_s;       //     with their E8M0 scales, row-major [cap, 2f/32]
   uint8_t* q_row;     // MXFP8 row-wise codes ([cap, f] for a, [cap, 2f] for dh)
   uint8_t* s_row;     // their scales, tensor-core tile layout
   uint8_t* q_colT;    // MXFP8 codes transposed ([f, cap] / [2f, cap])

@@ -304,3 +304,46 @@ def test_e5m2_gradient_format_layer():
         got = g[name]
         got = got.float().cpu().numpy() if got.dtype == torch.bfloat16 else got.cpu().numpy()
         parity(f"small_e5m2_grads.{name}", got, ref, TOL[precision])
+
+
+def test_saved_h_mxfp8_layer():
+    """h saved as MXFP8 for the backward (moe_ctx_set_saved_h): the saved buffer holds E4M3 codes
+    with one scale per 32 values of h (within tolerance of the oracle's h once dequantised), the
+    dSwiGLU epilogue reads g and u from them, and every gradient is within tolerance of the oracle
+    run with saved_h='mxfp8'; the dh requantisation stays bit-exact against its dumped input."""
+    precision = "mxfp8"
+    cfg = workloads.scaled_config(workloads.CONFIGS["small_mxfp8"], T=1024, seed=43)
+    T, d, f, E, k = cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
+    inp = workloads.make_inputs(cfg, with_dy=True)
+    dev = {n: t.cuda() for n, t in inp.items()}
+    cap = moe.capacity_rows(T, k, E)
+    dump_dh = torch.full((cap, 2 * f), float("nan"), dtype=torch.float32, device="cuda")
+    moe.set_debug_dump(0, None, dump_dh)
+    bws = torch.zeros(moe.sizes(T, d, f, E, k, precision, True)["bwd_ws"], dtype=torch.uint8, device="cuda")
+    try:
+        y, saved = moe.moe_grouped_mlp_fwd(dev["x"], dev["topk_idx"], dev["topk_prob"], dev["w_gate_up"],
+                                           dev["w_down"], precision=precision, training=True, saved_h="mxfp8")
+        dx, dw1, dw2, dp = moe.moe_grouped_mlp_bwd(dev["dy"], saved, dev["w_gate_up"], dev["w_down"], workspace=bws)
+        moe.get_status(0)
+    finally:
+        moe.set_debug_dump(0, None, None)
+    assert saved.buf.numel() == moe.sizes(T, d, f, E, k, precision, True, "mxfp8")["saved"]
+    assert saved.buf.numel() < moe.sizes(T, d, f, E, k, precision, True, "bf16")["saved"]
+    np_in = {n: (t.float().numpy() if t.dtype == torch.bfloat16 else t.numpy()) for n, t in inp.items()}
+    ry, st = omoe.forward(np_in["x"], np_in["topk_idx"], np_in["topk_prob"], np_in["w_gate_up"], np_in["w_down"],
+                          precision, saved_h="mxfp8")
+    gr = omoe.backward(np_in["dy"], st, np_in["w_gate_up"], np_in["w_down"])
+    Tp = int(st["route"]["poffsets"][E])
+    dims = (T, d, f, E, k, precision)
+    hq = moe.buffer_view(saved.buf, 0, "h_q", dims, True, cap * 2 * f, saved_h="mxfp8").cpu().numpy()
+    hs = moe.buffer_view(saved.buf, 0, "h_s", dims, True, cap * 2 * f // 32, saved_h="mxfp8").cpu().numpy()
+    h_deq = mx.dequantize_blocks(hq.reshape(cap, 2 * f)[:Tp], hs.reshape(cap, 2 * f // 32)[:Tp])
+    parity("small_saved_h_mxfp8.h", h_deq, mx.fake_quant(st["h"], axis=1), TOL[precision])
+    dh32 = dump_dh.cpu().numpy()[:Tp]
+    q = moe.buffer_view(bws, 2, "dh_q", dims, True, cap * 2 * f).cpu().numpy().reshape(cap, 2 * f)
+    assert np.array_equal(q[:Tp], mx.quantize_rowwise(dh32)[0])
+    parity("small_saved_h_mxfp8.dh", dh32, gr["dh_perm"], TOL[precision])
+    parity("small_saved_h_mxfp8.y", bf16_np(y), ry, TOL[precision])
+    for name, got, ref in (("dx", bf16_np(dx), gr["dx"]), ("dw1", bf16_np(dw1), gr["dw_gate_up"]),
+                           ("dw2", bf16_np(dw2), gr["dw_down"]), ("dp", dp.cpu().numpy(), gr["d_topk_prob"])):
+        parity(f"small_saved_h_mxfp8.{name}", got, ref, TOL[precision])
