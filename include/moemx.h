@@ -122,6 +122,16 @@ moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt);
 #define MOE_SAVED_H_MXFP8 1
 moe_status_t moe_ctx_set_saved_h(moe_ctx_t ctx, int mode);
 
+/* Forward GEMMs in one launch (hyper.ai: gate-up projection, SwiGLU, routing-weight scaling and the
+ * down projection fused into a single GroupedMLP kernel).  With ``on`` non-zero the fused layer's
+ * forward runs one persistent kernel that walks the gate_up tiles and then the down tiles; each
+ * down tile's loads wait (bounded, MOE_ERR_TIMEOUT on expiry) until every gate_up tile of its
+ * 128-row block has written its rows of a, which the gate_up epilogues release through one
+ * counter per row block in the forward workspace.  The kernel keeps one CTA on every SM for its
+ * whole run and its CTAs wait on one another, so it needs the GPU to itself: kernels of other
+ * streams that hold SMs meanwhile can make those waits expire.  Default off. */
+moe_status_t moe_ctx_set_fused_forward(moe_ctx_t ctx, int on);
+
 /* Test hook for the bounded in-kernel waits (tests only).  With ``stall`` non-zero, every CTA of
  * the persistent kernels (the grouped GEMMs and the TMA-fed quantiser) makes one extra wait on a
  * word of the context's status block that nothing ever sets, bounded by ``limit_cycles`` SM clock

@@ -34,7 +34,8 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_get_status", "moe_ctx_set_d
            "moe_saved_size", "moe_fwd_workspace_size", "moe_bwd_workspace_size", "moe_grouped_mlp_fwd",
            "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook", "moe_grouped_mlp_fwd_noalloc",
            "moe_ctx_set_test_stall", "moe_tensor_peak_loop", "moe_tensor_peak_flops", "moe_ctx_set_scale_rule",
-           "moe_ctx_set_grad_format", "moe_ctx_set_saved_h", "moe_saved_size_ex", "moe_buffer_address_ex"]
+           "moe_ctx_set_grad_format", "moe_ctx_set_saved_h", "moe_saved_size_ex", "moe_buffer_address_ex",
+           "moe_ctx_set_fused_forward"]
 
 LAUNCH_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
@@ -68,6 +69,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ctx_set_scale_rule": (c_int, [c_vp, c_int]),
         "moe_ctx_set_grad_format": (c_int, [c_vp, c_int]),
         "moe_ctx_set_saved_h": (c_int, [c_vp, c_int]),
+        "moe_ctx_set_fused_forward": (c_int, [c_vp, c_int]),
         "moe_saved_size_ex": (c_size, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int]),
         "moe_buffer_address_ex": (c_vp, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_vp,
                                          ctypes.c_char_p]),
@@ -171,6 +173,12 @@ def set_scale_rule(device: int, rule: str):
     """MXFP8 shared-exponent rule of the fused layer on ``device``: "ceil" (default) or "floor" (OCP)."""
     L = load_library()
     _check("moe_ctx_set_scale_rule", L.moe_ctx_set_scale_rule(context(device), SCALE_RULES[rule]))
+
+
+def set_fused_forward(device: int, on: bool):
+    """Run the forward's two GEMMs as one persistent launch on ``device`` (see moemx.h)."""
+    L = load_library()
+    _check("moe_ctx_set_fused_forward", L.moe_ctx_set_fused_forward(context(device), int(on)))
 
 
 def set_grad_format(device: int, fmt: str):

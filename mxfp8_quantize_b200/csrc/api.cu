@@ -24,6 +24,7 @@ struct moe_ctx_s {
   int scale_floor;          // MXFP8 shared-exponent rule of the fused layer (moe_ctx_set_scale_rule)
   int grad_e5m2;            // MXFP8 gradient operands in E5M2 (moe_ctx_set_grad_format)
   int saved_h;              // format of the h a training forward saves (moe_ctx_set_saved_h)
+  int fused_fwd;            // both forward GEMMs in one launch (moe_ctx_set_fused_forward)
   int stall;                // test hook for the bounded waits (moe_ctx_set_test_stall)
   long long stall_limit;
 };
@@ -247,6 +248,7 @@ struct FwdWs {
   uint8_t *w1_q, *w1_s, *w2_q, *w2_s, *x_q, *x_s, *a_q, *a_s;
   bf16 *x_perm, *a, *w1_copy, *w2_copy;
   bf16* y_perm;
+  int* mblk;  // fused forward: completion counters per 128-row block
 };
 void carve_fwd(Carve& c, const Dims& D, FwdWs& w) {
   std::memset(&w, 0, sizeof(w));
@@ -266,6 +268,7 @@ void carve_fwd(Carve& c, const Dims& D, FwdWs& w) {
     w.w2_copy = c.take<bf16>(D.E * D.d * D.f * 2);
   }
   w.y_perm = c.take<bf16>(D.cap * D.d * 2);
+  w.mblk = c.take<int>(D.cap / 128 * sizeof(int));
 }
 
 struct BwdWs {
@@ -425,6 +428,7 @@ moe_status_t moe_ctx_create(moe_ctx_t* out, int device) {
   c->scale_floor = 0;
   c->grad_e5m2 = 0;
   c->saved_h = MOE_SAVED_H_BF16;
+  c->fused_fwd = 0;
   c->stall = 0;
   c->stall_limit = 0;
   if (cudaMalloc(&c->d_status, 256) != cudaSuccess) {
@@ -484,6 +488,12 @@ moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt) {
 moe_status_t moe_ctx_set_saved_h(moe_ctx_t ctx, int mode) {
   if (!ctx || (mode != MOE_SAVED_H_BF16 && mode != MOE_SAVED_H_MXFP8)) return MOE_ERR_INVALID_ARG;
   ctx->saved_h = mode;
+  return MOE_OK;
+}
+
+moe_status_t moe_ctx_set_fused_forward(moe_ctx_t ctx, int on) {
+  if (!ctx) return MOE_ERR_INVALID_ARG;
+  ctx->fused_fwd = on ? 1 : 0;
   return MOE_OK;
 }
 
@@ -811,29 +821,43 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       ep.o_row = w.a;
       ep.o_colT = training ? s.aT : nullptr;
     }
-    MOE_LAUNCH(ctx, "gemm_gate_up_swiglu", st, launch_grouped_gemm(g, D.mx, EPI_SWIGLU, ctx->num_sms, st));
-  }
-  // 4. down GEMM
-  {
-    GemmArgs g = gemm_args(ctx);
-    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.a_q) : w.a, D.mx, f, D.cap,
-                           f * (D.mx ? 1 : 2)) &&
-                    map_3d(&g.tmap_b, w2_base, D.mx, f, d, E, f * (D.mx ? 1 : 2), w2_stride, gemm_tile_n(EPI_STORE));
-    if (!ok) return MOE_ERR_CUDA;
-    g.kgrouped = 0;
-    g.E = E;
-    g.K = static_cast<int>(f);
-    g.n_tiles = static_cast<int>(d / 256);
-    g.poffsets = s.poff;
-    g.sfa = w.a_s;
-    g.sfa_kb4 = f / 128;
-    g.sfb = w.w2_s;
-    g.sfb_kb4 = f / 128;
-    g.sfb_expert_rows = d;
-    if (D.mx && !sf_maps(g, D.cap, E * d, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
-    g.epi.out = w.y_perm;
-    g.epi.ldo = d;
-    MOE_LAUNCH(ctx, "gemm_down", st, launch_grouped_gemm(g, D.mx, EPI_STORE, ctx->num_sms, st));
+    // 4. down GEMM: its own launch, or (fused forward) the tiles that follow in the same launch
+    GemmArgs g2 = gemm_args(ctx);
+    const bool ok2 = map_2d(&g2.tmap_a, D.mx ? static_cast<const void*>(w.a_q) : w.a, D.mx, f, D.cap,
+                            f * (D.mx ? 1 : 2)) &&
+                     map_3d(&g2.tmap_b, w2_base, D.mx, f, d, E, f * (D.mx ? 1 : 2), w2_stride, gemm_tile_n(EPI_STORE));
+    if (!ok2) return MOE_ERR_CUDA;
+    g2.kgrouped = 0;
+    g2.E = E;
+    g2.K = static_cast<int>(f);
+    g2.n_tiles = static_cast<int>(d / 256);
+    g2.poffsets = s.poff;
+    g2.sfa = w.a_s;
+    g2.sfa_kb4 = f / 128;
+    g2.sfb = w.w2_s;
+    g2.sfb_kb4 = f / 128;
+    g2.sfb_expert_rows = d;
+    if (D.mx && !sf_maps(g2, D.cap, E * d, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
+    g2.epi.out = w.y_perm;
+    g2.epi.ldo = d;
+    if (ctx->fused_fwd) {
+      // one persistent launch: gate_up tiles, then down tiles that wait for their 128-row blocks of a
+      g.tmap_a2 = g2.tmap_a;
+      g.tmap_b2 = g2.tmap_b;
+      g.tmap_sfa2 = g2.tmap_sfa;
+      g.tmap_sfb2 = g2.tmap_sfb;
+      g.K2 = g2.K;
+      g.n_tiles2 = g2.n_tiles;
+      g.sfb_expert_rows2 = g2.sfb_expert_rows;
+      g.epi.out = g2.epi.out;
+      g.epi.ldo = g2.epi.ldo;
+      g.mblock_done = w.mblk;
+      MOE_CUDA(cudaMemsetAsync(w.mblk, 0, static_cast<size_t>(D.cap / 128) * sizeof(int), st));
+      MOE_LAUNCH(ctx, "gemm_fused_forward", st, launch_grouped_gemm(g, D.mx, EPI_FUSED_FWD, ctx->num_sms, st));
+    } else {
+      MOE_LAUNCH(ctx, "gemm_gate_up_swiglu", st, launch_grouped_gemm(g, D.mx, EPI_SWIGLU, ctx->num_sms, st));
+      MOE_LAUNCH(ctx, "gemm_down", st, launch_grouped_gemm(g2, D.mx, EPI_STORE, ctx->num_sms, st));
+    }
   }
   // 5. combine (probabilities were applied in ScaledSwiGLU)
   MOE_LAUNCH(ctx, "unpermute_y", st, launch_unpermute(w.y_perm, s.src2s, nullptr, T, k, d, static_cast<bf16*>(y), ctx->num_sms, st));
@@ -1176,6 +1200,7 @@ moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx,
   c.scale_floor = 0;
   c.grad_e5m2 = 0;
   c.saved_h = MOE_SAVED_H_BF16;
+  c.fused_fwd = 0;
   c.stall = 0;
   c.stall_limit = 0;
   // the scratch base is 256-aligned; the workspace carving aligns to 1 KiB inside the size bound

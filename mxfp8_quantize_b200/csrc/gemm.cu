@@ -70,7 +70,7 @@ struct Shape {
   static constexpr int OFF_STAGING = OFF_H + H_BYTES;
   static constexpr int SMEM_DYN = OFF_STAGING + EPI_WARPS * STAGING_PER_WARP + 1024;
   static_assert(NBUF * BN + STAGES * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
-  static_assert(SMEM_DYN + 4096 <= 232448, "shared memory budget");
+  static_assert(SMEM_DYN + 6144 <= 232448, "shared memory budget");  // + the static SharedState
   static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0 && (LEAD == 4 || LEAD == 2), "thread layout");
 };
 using ShapeStore = Shape<256, 1, 4, false, 8, 16>;    // plain bf16-store epilogues
@@ -89,7 +89,9 @@ struct SharedState {
   uint32_t tmem_base;
   int abort_flag;
   int total_tiles;
+  int total1;                            // EPI_FUSED_FWD: gate_up tiles (the down tiles follow)
   int tile_prefix[MOE_MAX_EXPERTS + 1];  // tiles before the i-th expert of ``order``
+  int tile_prefix2[MOE_MAX_EXPERTS + 1]; // EPI_FUSED_FWD: down tiles before expert e
   int poff[MOE_MAX_EXPERTS + 1];         // padded row offsets, by expert id
   int order[MOE_MAX_EXPERTS];            // expert ids in tile-list order
 };
@@ -98,6 +100,7 @@ struct Tile {
   int e, mb, nb, nk;
   int a_row;  // first row of A (M-grouped: token row; K-grouped: row of the M dimension)
   int k0;     // first K coordinate (K-grouped: the expert's first token row)
+  bool down;  // EPI_FUSED_FWD: a tile of the down GEMM
 };
 
 // The i-th tile of this CTA: tiles are dealt out in rounds of gridDim.x, in boustrophedon order
@@ -109,6 +112,25 @@ __device__ __forceinline__ int tile_of(int i) {
 }
 
 __device__ __forceinline__ void decode_tile(int t, const SharedState& s, const GemmArgs& g, bool mx, Tile& o) {
+  o.down = false;
+  if (g.mblock_done && t >= s.total1) {  // fused forward: a down tile (experts in id order)
+    const int t2 = t - s.total1;
+    int lo = 0, hi = g.E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s.tile_prefix2[mid] <= t2) lo = mid; else hi = mid;
+    }
+    const int e = lo, local = t2 - s.tile_prefix2[e];
+    const int mt = (s.poff[e + 1] - s.poff[e]) / BM;
+    o.down = true;
+    o.e = e;
+    o.nb = local / mt;
+    o.mb = local - o.nb * mt;
+    o.a_row = s.poff[e] + o.mb * BM;
+    o.k0 = 0;
+    o.nk = g.K2 / (mx ? 128 : 64);
+    return;
+  }
   int lo = 0, hi = g.E;  // largest i with prefix[i] <= t (experts without tiles are skipped)
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -302,6 +324,16 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       acc += g.kgrouped ? g.m_tiles * g.n_tiles : ((s.poff[e + 1] - s.poff[e]) / BM) * g.n_tiles;
     }
     s.tile_prefix[g.E] = acc;
+    s.total1 = acc;
+    if (EPI == EPI_FUSED_FWD) {  // the down tiles after all gate_up tiles
+      int acc2 = 0;
+      for (int e = 0; e < g.E; ++e) {
+        s.tile_prefix2[e] = acc2;
+        acc2 += ((s.poff[e + 1] - s.poff[e]) / BM) * g.n_tiles2;
+      }
+      s.tile_prefix2[g.E] = acc2;
+      acc += acc2;
+    }
     s.total_tiles = acc;
     s.abort_flag = 0;
     for (int i = 0; i < S::STAGES; ++i) {
@@ -320,6 +352,10 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
   if (warp == 0 && lane == 0) {
     ptx::prefetch_tmap(&g.tmap_a);
     ptx::prefetch_tmap(&g.tmap_b);
+    if (EPI == EPI_FUSED_FWD) {
+      ptx::prefetch_tmap(&g.tmap_a2);
+      ptx::prefetch_tmap(&g.tmap_b2);
+    }
     if (MX) {
       ptx::prefetch_tmap(&g.tmap_sfa);
       ptx::prefetch_tmap(&g.tmap_sfb);
@@ -351,6 +387,16 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       Tile tl;
       decode_tile(t, s, g, MX, tl);
       const int bk = MX ? 128 : 64;
+      if (EPI == EPI_FUSED_FWD && tl.down) {
+        // the tile's 128 rows of a are complete once every gate_up tile of its row block has released them
+        if (!ptx::wait_counter(g.mblock_done + tl.a_row / BM, g.n_tiles * S::EPI_WARPS, abort_flag, lim)) break;
+        ptx::fence_proxy_async_global();  // TMA reads of what other CTAs wrote with ordinary stores
+      }
+      const CUtensorMap* map_a = tl.down ? &g.tmap_a2 : &g.tmap_a;
+      const CUtensorMap* map_b = tl.down ? &g.tmap_b2 : &g.tmap_b;
+      const CUtensorMap* map_sfa = tl.down ? &g.tmap_sfa2 : &g.tmap_sfa;
+      const CUtensorMap* map_sfb = tl.down ? &g.tmap_sfb2 : &g.tmap_sfb;
+      const int64_t sfb_rows = tl.down ? g.sfb_expert_rows2 : g.sfb_expert_rows;
       for (int kb = 0; kb < tl.nk; ++kb) {
         if (g.stall_flag && !stalled && kb == min(2, tl.nk - 1)) {  // test hook: a wait that can only expire
           stalled = true;
@@ -360,22 +406,22 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         uint8_t* st = smem + stage * S::STAGE_BYTES;
         ptx::mbar_arrive_expect_tx(&s.full[stage], tx);
         const int kx = tl.k0 + kb * bk;
-        ptx::tma_load_2d(st, &g.tmap_a, kx, tl.a_row, &s.full[stage]);
-        if (!g.kgrouped && g.gate_up_half) {
+        ptx::tma_load_2d(st, map_a, kx, tl.a_row, &s.full[stage]);
+        if (!g.kgrouped && g.gate_up_half && !tl.down) {
           // bf16 gate_up: BN/2 gate rows then the matching BN/2 up rows of expert e
-          ptx::tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * (BN / 2), tl.e, &s.full[stage]);
-          ptx::tma_load_3d(st + S::OFF_B + S::B_BYTES / 2, &g.tmap_b, kx, g.gate_up_half + tl.nb * (BN / 2), tl.e,
+          ptx::tma_load_3d(st + S::OFF_B, map_b, kx, tl.nb * (BN / 2), tl.e, &s.full[stage]);
+          ptx::tma_load_3d(st + S::OFF_B + S::B_BYTES / 2, map_b, kx, g.gate_up_half + tl.nb * (BN / 2), tl.e,
                       &s.full[stage]);
         } else if (!g.kgrouped) {  // one box of BN rows
-          ptx::tma_load_3d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * BN, tl.e, &s.full[stage]);
+          ptx::tma_load_3d(st + S::OFF_B, map_b, kx, tl.nb * BN, tl.e, &s.full[stage]);
         } else {
-          ptx::tma_load_2d(st + S::OFF_B, &g.tmap_b, kx, tl.nb * BN, &s.full[stage]);
+          ptx::tma_load_2d(st + S::OFF_B, map_b, kx, tl.nb * BN, &s.full[stage]);
         }
         if (MX) {  // this step's scale tiles: one of A, BN/128 consecutive ones of B
           const int32_t kq = kx / 128;
-          const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * g.sfb_expert_rows;
-          ptx::tma_load_3d(st + S::OFF_SFA, &g.tmap_sfa, 0, kq, tl.a_row / 128, &s.full[stage]);
-          ptx::tma_load_3d(st + S::OFF_SFB, &g.tmap_sfb, 0, kq,
+          const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * sfb_rows;
+          ptx::tma_load_3d(st + S::OFF_SFA, map_sfa, 0, kq, tl.a_row / 128, &s.full[stage]);
+          ptx::tma_load_3d(st + S::OFF_SFB, map_sfb, 0, kq,
                       static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128), &s.full[stage]);
         }
         issued_mask |= 1u << stage;
@@ -504,7 +550,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       const uint32_t acc_par = static_cast<uint32_t>((S::NBUF == 2 ? (local >> 1) : local) & 1);
       ++local;
 
-      if (EPI == EPI_STORE) {
+      if (EPI == EPI_STORE || (EPI == EPI_FUSED_FWD && tl.down)) {
         // drain the accumulator into packed bf16, release it, then store
         if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
         ptx::tc_fence_after();
@@ -533,7 +579,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
 #pragma unroll
           for (int i = 0; i < CPT / 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
         }
-      } else if (EPI == EPI_SWIGLU) {
+      } else if (EPI == EPI_SWIGLU || EPI == EPI_FUSED_FWD) {
         // tile = BN/2 output columns; accumulator columns [0,BN/2) gate, [BN/2,BN) up
         constexpr int OPT = BN / 2 / NPART;  // output columns per thread
         constexpr int G = OPT / 32;          // groups of 32 output columns per thread
@@ -584,6 +630,15 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
 #pragma unroll
             for (int i = 0; i < 2; ++i) ptx::st_global_v8(dst + 16 * i, pack_bf16x8(gv + 16 * i), pack_bf16x8(gv + 16 * i + 8));
             if (ep.o_colT) colwise_bf16<S::PASS>(gv, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
+          }
+        }
+        if (EPI == EPI_FUSED_FWD) {
+          // this warp's share of the tile's rows of a (codes and scales) is written: release it to the
+          // down tiles of the row block (every lane's stores, then one GPU-scope fence and count)
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence();
+            atomicAdd(g.mblock_done + tl.a_row / BM, 1);
           }
         }
       } else {  // EPI_DSWIGLU: tile = BN f-columns of da; this thread owns BN/2 of them
@@ -733,7 +788,8 @@ cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
 }  // namespace
 
 int gemm_tile_n(int epi) {
-  return epi == EPI_STORE ? ShapeStore::BN : (epi == EPI_SWIGLU ? ShapeSwiglu::BN : ShapeDswiglu::BN);
+  return epi == EPI_STORE ? ShapeStore::BN
+                          : ((epi == EPI_SWIGLU || epi == EPI_FUSED_FWD) ? ShapeSwiglu::BN : ShapeDswiglu::BN);
 }
 
 int gemm_dswiglu_parts() { return ShapeDswiglu::EPI_WARPS / 4; }
@@ -742,11 +798,13 @@ cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_
   if (mx) {
     if (epi == EPI_STORE) return launch_t<true, EPI_STORE, ShapeStore>(args, num_sms, st);
     if (epi == EPI_SWIGLU) return launch_t<true, EPI_SWIGLU, ShapeSwiglu>(args, num_sms, st);
+    if (epi == EPI_FUSED_FWD) return launch_t<true, EPI_FUSED_FWD, ShapeSwiglu>(args, num_sms, st);
     if (args.epi.h_q) return launch_t<true, EPI_DSWIGLU, ShapeDswigluG>(args, num_sms, st);
     return launch_t<true, EPI_DSWIGLU, ShapeDswiglu>(args, num_sms, st);
   }
   if (epi == EPI_STORE) return launch_t<false, EPI_STORE, ShapeStore>(args, num_sms, st);
   if (epi == EPI_SWIGLU) return launch_t<false, EPI_SWIGLU, ShapeSwiglu>(args, num_sms, st);
+  if (epi == EPI_FUSED_FWD) return launch_t<false, EPI_FUSED_FWD, ShapeSwiglu>(args, num_sms, st);
   return launch_t<false, EPI_DSWIGLU, ShapeDswiglu>(args, num_sms, st);
 }
 

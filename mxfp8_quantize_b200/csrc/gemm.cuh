@@ -10,6 +10,8 @@ enum EpiKind : int {
   EPI_STORE = 0,    // fp32 accumulator -> bf16 rows
   EPI_SWIGLU = 1,   // gate/up accumulator -> a = silu(g)*u*p, requantised (ScaledSwiGLU)
   EPI_DSWIGLU = 2,  // da accumulator + saved h -> dh = [dg, du] requantised, dp partial sums
+  EPI_FUSED_FWD = 3,  // the whole forward in one launch: gate_up tiles (EPI_SWIGLU epilogue), then
+                      // down tiles (bf16 rows), each waiting for its rows of a
 };
 
 struct EpiArgs {
@@ -59,6 +61,17 @@ struct GemmArgs {
   int64_t sfb_kb4;
   int64_t sfb_expert_rows;  // rows of B per expert (M-grouped), for the scale tile index
   int a_e5m2;          // MXFP8: A's elements are E5M2 (B's stay E4M3)
+  // EPI_FUSED_FWD: the down GEMM that follows the gate_up tiles (A = a [rows, f], B = W2 [E, d, f]),
+  // its output rows go to epi.out / epi.ldo
+  CUtensorMap tmap_a2;
+  CUtensorMap tmap_b2;
+  CUtensorMap tmap_sfa2;
+  CUtensorMap tmap_sfb2;
+  int K2;              // the down GEMM's reduction length (f)
+  int n_tiles2;        // its output tiles per 128-row block (d / BN)
+  int64_t sfb_expert_rows2;
+  int* mblock_done;    // per 128-row block: epilogue-warp completions of its gate_up tiles (zeroed by the
+                       // caller before the launch); a down tile starts once all n_tiles x warps arrived
   int* status;
   // test hook: a device flag nothing sets; when non-null the producer of each CTA waits on it once,
   // for at most stall_limit cycles, after issuing the first stages of its first tile

@@ -77,6 +77,29 @@ __device__ __forceinline__ bool wait_flag(const int* flag, volatile int* abort_f
   }
 }
 
+// Bounded wait until a global counter reaches ``target`` (acquire at GPU scope).  Returns false on
+// abort or after ``limit_cycles`` SM clocks (then raising the abort flag itself).
+__device__ __forceinline__ bool wait_counter(const int* ctr, int target, volatile int* abort_flag,
+                                             long long limit_cycles) {
+  const long long t0 = clock64();
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit_cycles) {
+      *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(128);
+  }
+}
+// Order this thread's later asynchronous-proxy accesses (TMA loads) of global memory after what it
+// has observed through the generic proxy (data other threads wrote with ordinary stores).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- wide global stores
 // 32 bytes (lo then hi) to a 32-byte aligned global address with one 256-bit store: a warp of
 // these writes whole 32-byte sectors even when every lane targets a different row.

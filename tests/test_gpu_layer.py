@@ -347,3 +347,30 @@ def test_saved_h_mxfp8_layer():
     for name, got, ref in (("dx", bf16_np(dx), gr["dx"]), ("dw1", bf16_np(dw1), gr["dw_gate_up"]),
                            ("dw2", bf16_np(dw2), gr["dw_down"]), ("dp", dp.cpu().numpy(), gr["d_topk_prob"])):
         parity(f"small_saved_h_mxfp8.{name}", got, ref, TOL[precision])
+
+
+@pytest.mark.parametrize("precision", ["mxfp8", "bf16"])
+@pytest.mark.parametrize("T", [3, 1500])
+def test_fused_forward_matches_two_launches(precision, T):
+    """moe_ctx_set_fused_forward: the gate_up and down tiles in one persistent launch (down tiles
+    waiting on per-row-block completion counters) compute exactly what the two launches compute:
+    the same tiles with the same accumulation order, so every output of the forward and of the
+    backward that follows is bit-identical, and within tolerance of the oracle."""
+    cfg = workloads.scaled_config(workloads.CONFIGS["small_mxfp8"], precision=precision, T=T, seed=44)
+    inp = workloads.make_inputs(cfg, with_dy=True)
+    dev = {n: t.cuda() for n, t in inp.items()}
+    res = []
+    for fused in (False, True):
+        moe.set_fused_forward(0, fused)
+        try:
+            y, saved = moe.moe_grouped_mlp_fwd(dev["x"], dev["topk_idx"], dev["topk_prob"], dev["w_gate_up"],
+                                               dev["w_down"], precision=precision, training=True)
+            dx, dw1, dw2, dp = moe.moe_grouped_mlp_bwd(dev["dy"], saved, dev["w_gate_up"], dev["w_down"])
+            moe.get_status(0)
+        finally:
+            moe.set_fused_forward(0, False)
+        res.append([t.float().cpu() if t.dtype == torch.bfloat16 else t.cpu() for t in (y, dx, dw1, dw2, dp)])
+    for name, a, b in zip(("y", "dx", "dw_gate_up", "dw_down", "d_topk_prob"), *res):
+        assert torch.equal(a, b), name
+    ref = _oracle(inp, precision, backward=False)
+    parity(f"fused_forward_{precision}_T{T}.y", res[1][0].numpy(), ref["y"], TOL[precision])
