@@ -62,6 +62,7 @@ def kernel_work(cfg, name):
         "gemm_wgrad_down": 2.0 * Tk * d * f,
         "gemm_dgrad_gate_up": 2.0 * Tk * 2 * f * d,
         "gemm_wgrad_gate_up": 2.0 * Tk * 2 * f * d,
+        "gemm_fused_forward": 2.0 * Tk * d * 2 * f + 2.0 * Tk * f * d,
     }
     if name in gemm:
         return "tensor", gemm[name]
@@ -244,6 +245,7 @@ def torch_loop_context(cfg, device: int, steps: int = 5, warmup: int = 2):
     library path, not this build's kernels.  Returns TFLOP/s and ms per fwd+bwd step."""
     dev = torch.device("cuda", device)
     inp = workloads.make_inputs(cfg, with_dy=True)
+    moe.set_fused_forward(local_rank, args.fused_forward)
     x = inp["x"].to(dev)
     idx = inp["topk_idx"].to(dev).long()
     prob = inp["topk_prob"].to(dev).to(torch.bfloat16)
@@ -491,7 +493,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     tensor_peaks = {"matched_tflops": round(loop_tflops, 1), "matched_ms": round(loop_ms, 1),
                     "burst_tflops": round(peak_burst, 1), "nominal_rule_tflops": round(nominal_rule, 1)}
     return dict(ms=ms, kernels=kern, roofline=roofline, clocks=clk, e2e=e2e, launches=launches,
-                tensor_peaks=tensor_peaks, memory={"saved_h": args.saved_h, "saved_bytes": sz["saved"],
+                tensor_peaks=tensor_peaks, fused_forward=bool(args.fused_forward),
+                memory={"saved_h": args.saved_h, "saved_bytes": sz["saved"],
                                                    "fwd_workspace_bytes": sz["fwd_ws"], "bwd_workspace_bytes": sz["bwd_ws"]})
 
 
@@ -516,6 +519,7 @@ def main():
     ap.add_argument("--experts", type=int, default=None, help="override E (profiling cases)")
     ap.add_argument("--clocks-dir", default=tempfile.gettempdir(), help="where the nvidia-smi clock samples go")
     ap.add_argument("--peaks", action="store_true", help="measure the tensor-core peak loop (burst and sustained)")
+    ap.add_argument("--fused-forward", action="store_true", help="both forward GEMMs in one persistent launch")
     ap.add_argument("--saved-h", default="bf16", choices=["bf16", "mxfp8"],
                     help="format h is saved in for the backward (long-sequence memory mode)")
     ap.add_argument("--context-torch-loop", action="store_true",
@@ -577,6 +581,7 @@ def main():
             "tokens_per_s": round(world * cfg.T / (res["ms"] * 1e-3), 1),
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["launches"],
             "clocks": res["clocks"], "tensor_peaks": res["tensor_peaks"], "memory": res["memory"],
+            "fused_forward": res["fused_forward"],
             "kernels": res["kernels"]}
     if args.context_torch_loop and world == 1:
         line["context_torch_loop"] = torch_loop_context(workloads.scaled_config(cfg, precision="bf16"), local_rank)
