@@ -520,7 +520,7 @@ def main():
     ap.add_argument("--clocks-dir", default=tempfile.gettempdir(), help="where the nvidia-smi clock samples go")
     ap.add_argument("--peaks", action="store_true", help="measure the tensor-core peak loop (burst and sustained)")
     ap.add_argument("--fused-forward", action="store_true", help="both forward GEMMs in one persistent launch")
-    ap.add_argument("--saved-h", default="bf16", choices=["bf16", "mxfp8"],
+    ap.add_argument("--saved-h", default="bf16", choices=["bf16", "mxfp8", "recompute"],
                     help="format h is saved in for the backward (long-sequence memory mode)")
     ap.add_argument("--context-torch-loop", action="store_true",
                     help="also time a plain PyTorch per-expert loop (BF16, autograd) on the same workload shape")

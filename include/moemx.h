@@ -117,9 +117,16 @@ moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt);
  *                     2f (row-major [capacity, 2f/32]), quantised in the gate_up GEMM's epilogue with
  *                     the context's scale rule; the dSwiGLU epilogue reads g and u dequantised from
  *                     it.  About half the bytes; MXFP8 precision only (MOE_ERR_UNSUPPORTED for BF16).
- * moe_saved_size_ex gives the saved-buffer size for a mode. */
+ *   MOE_SAVED_H_RECOMPUTE no h at all: the forward keeps x's gate_up operand instead (MXFP8 row-wise
+ *                     codes and scales, or the BF16 gathered rows, [capacity, d]); the backward
+ *                     quantises W1 again (MXFP8), re-runs the gate_up GEMM with an epilogue that only
+ *                     writes h into its workspace (moe_bwd_workspace_size_ex), and goes on as with a
+ *                     saved bf16 h, giving the same results bit for bit.  Costs one more gate_up GEMM
+ *                     (and W1 quantisation) per backward.
+ * moe_saved_size_ex / moe_bwd_workspace_size_ex give the buffer sizes for a mode. */
 #define MOE_SAVED_H_BF16 0
 #define MOE_SAVED_H_MXFP8 1
+#define MOE_SAVED_H_RECOMPUTE 2
 moe_status_t moe_ctx_set_saved_h(moe_ctx_t ctx, int mode);
 
 /* Forward GEMMs in one launch (hyper.ai: gate-up projection, SwiGLU, routing-weight scaling and the
@@ -249,6 +256,7 @@ size_t moe_saved_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precisi
 size_t moe_saved_size_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int saved_h);
 size_t moe_fwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training);
 size_t moe_bwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec);
+size_t moe_bwd_workspace_size_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int saved_h);
 
 /* x bf16 [T, d]; topk_idx int32 [T, k]; topk_prob fp32 [T, k]; split_sizes int32 [E] or NULL
  * (checked against topk_idx on the device when given); y bf16 [T, d]. */
@@ -314,11 +322,12 @@ double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters)
  * a forward workspace (which = 1) or a backward workspace (which = 2) laid out for these
  * dimensions, given the buffer's base address ``base``; NULL for an unknown name.  Names:
  * saved: split_sizes poffsets sorted_to_src src_to_sorted prob_perm w1c_q w1c_s w2c_q w2c_s
- *        xT_q xT_s aT_q aT_s xT aT h (h_q h_s with moe_buffer_address_ex and MOE_SAVED_H_MXFP8)
+ *        xT_q xT_s aT_q aT_s xT aT h (with moe_buffer_address_ex: h_q h_s for MOE_SAVED_H_MXFP8,
+ *        xr_q xr_s xr for MOE_SAVED_H_RECOMPUTE)
  * forward workspace: w1_q w1_s w2_q w2_s x_q x_s a_q a_s x_perm a y_perm (+ the routing names
  *        when training == 0)
  * backward workspace: dy_q dy_s dyT_q dyT_s dh_q dh_s dhT_q dhT_s dy_perm dyT dh dhT w1T w2T
- *        dx_perm dp_part
+ *        dx_perm dp_part (+ hr w1r_q w1r_s for MOE_SAVED_H_RECOMPUTE)
  * Scales (*_s) are in the tensor-core tile layout described at mxfp8_quantize. */
 void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
                          int which, void* base, const char* name);

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(HERE, "libmoemx.so")
 MOE_ROW_ALIGN = 128
 MXFP8_ROWWISE, MXFP8_COLWISE_T, MXFP8_SF_MMA_LAYOUT, MXFP8_FLAG_SCALE_FLOOR, MXFP8_FLAG_E5M2 = 1, 2, 4, 8, 16
 GRAD_FORMATS = {"e4m3": 0, "e5m2": 1}
-SAVED_H = {"bf16": 0, "mxfp8": 1}
+SAVED_H = {"bf16": 0, "mxfp8": 1, "recompute": 2}
 SCALE_RULES = {"ceil": 0, "floor": 1}
 PRECISIONS = {"bf16": 0, "mxfp8": 1}
 STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "unsupported", 4: "cuda", 5: "device", 6: "timeout",
@@ -35,7 +35,7 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_get_status", "moe_ctx_set_d
            "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook", "moe_grouped_mlp_fwd_noalloc",
            "moe_ctx_set_test_stall", "moe_tensor_peak_loop", "moe_tensor_peak_flops", "moe_ctx_set_scale_rule",
            "moe_ctx_set_grad_format", "moe_ctx_set_saved_h", "moe_saved_size_ex", "moe_buffer_address_ex",
-           "moe_ctx_set_fused_forward"]
+           "moe_ctx_set_fused_forward", "moe_bwd_workspace_size_ex"]
 
 LAUNCH_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_ctx_set_saved_h": (c_int, [c_vp, c_int]),
         "moe_ctx_set_fused_forward": (c_int, [c_vp, c_int]),
         "moe_saved_size_ex": (c_size, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int]),
+        "moe_bwd_workspace_size_ex": (c_size, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int]),
         "moe_buffer_address_ex": (c_vp, [c_i64, c_int, c_int, c_i64, c_i64, c_int, c_int, c_int, c_int, c_vp,
                                          ctypes.c_char_p]),
         "moe_tensor_peak_loop": (c_int, [c_vp, c_int, c_i64, c_int, c_vp]),
@@ -294,7 +295,7 @@ def sizes(T: int, d: int, f: int, E: int, k: int, precision: str, training: bool
     p = PRECISIONS[precision]
     return dict(saved=int(L.moe_saved_size_ex(T, k, E, d, f, p, SAVED_H[saved_h])),
                 fwd_ws=int(L.moe_fwd_workspace_size(T, k, E, d, f, p, int(training))),
-                bwd_ws=int(L.moe_bwd_workspace_size(T, k, E, d, f, p)))
+                bwd_ws=int(L.moe_bwd_workspace_size_ex(T, k, E, d, f, p, SAVED_H[saved_h])))
 
 
 def buffer_view(buf: torch.Tensor, which: int, name: str, dims: tuple, training: bool, nbytes: int,
@@ -379,7 +380,7 @@ def moe_grouped_mlp_bwd(dy: torch.Tensor, saved: Saved, w_gate_up: Weights, w_do
     """Gradients (dx, dw_gate_up [E,2f,d], dw_down [E,d,f], d_topk_prob [T,k]) for upstream dy."""
     T, d, f, E, k, precision = saved.dims
     dev = _device_index(dy)
-    sz = sizes(T, d, f, E, k, precision, True)
+    sz = sizes(T, d, f, E, k, precision, True, saved.saved_h)
     if workspace is None:
         workspace = torch.empty(sz["bwd_ws"], dtype=torch.uint8, device=dy.device)
     if dx is None:

@@ -210,7 +210,9 @@ struct Saved {
   uint8_t *xT_q, *xT_s, *aT_q, *aT_s;      // MXFP8: token-axis quantised x and a, transposed
   bf16 *xT, *aT;                           // BF16: transposed copies
   bf16* h;                                 // [cap, 2f] gate/up pre-activations (bf16) ...
-  uint8_t *h_q, *h_s;                      // ... or as MXFP8: codes [cap, 2f], scales [cap, 2f/32]
+  uint8_t *h_q, *h_s;                      // ... or as MXFP8: codes [cap, 2f], scales [cap, 2f/32] ...
+  uint8_t *xr_q, *xr_s;                    // ... or not at all (recompute): x's gate_up operand instead,
+  bf16* xr;                                //     MXFP8 row-wise codes + scales, or the BF16 gathered rows
 };
 void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
   s.split = c.take<int32_t>(D.E * 4);
@@ -222,6 +224,8 @@ void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
   s.xT = s.aT = nullptr;
   s.h = nullptr;
   s.h_q = s.h_s = nullptr;
+  s.xr_q = s.xr_s = nullptr;
+  s.xr = nullptr;
   if (!full) return;  // inference: routing bookkeeping only
   if (D.mx) {
     s.w1c_q = c.take<uint8_t>(D.E * D.d * 2 * D.f);
@@ -239,6 +243,13 @@ void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
   if (D.saved_h == MOE_SAVED_H_MXFP8) {
     s.h_q = c.take<uint8_t>(D.cap * 2 * D.f);
     s.h_s = c.take<uint8_t>(D.cap * 2 * D.f / 32);
+  } else if (D.saved_h == MOE_SAVED_H_RECOMPUTE) {
+    if (D.mx) {
+      s.xr_q = c.take<uint8_t>(D.cap * D.d);
+      s.xr_s = c.take<uint8_t>(D.cap * D.d / 32);
+    } else {
+      s.xr = c.take<bf16>(D.cap * D.d * 2);
+    }
   } else {
     s.h = c.take<bf16>(D.cap * 2 * D.f * 2);
   }
@@ -276,6 +287,9 @@ struct BwdWs {
   bf16 *dy_perm, *dyT, *dh, *dhT, *w1T, *w2T;
   bf16* dx_perm;
   float* dp_part;
+  bf16* hr;               // recompute: h regenerated by the gate_up GEMM
+  uint8_t *w1r_q, *w1r_s;  // recompute, MXFP8: W1 quantised again (row-wise, gate/up interleaved)
+  bf16* w1r_copy;          // recompute, BF16: W1 gathered when the experts are not evenly spaced
 };
 void carve_bwd(Carve& c, const Dims& D, BwdWs& w) {
   std::memset(&w, 0, sizeof(w));
@@ -298,6 +312,15 @@ void carve_bwd(Carve& c, const Dims& D, BwdWs& w) {
   }
   w.dx_perm = c.take<bf16>(D.cap * D.d * 2);
   w.dp_part = c.take<float>(gemm_dswiglu_parts() * (D.f / gemm_tile_n(EPI_DSWIGLU)) * D.cap * 4);
+  if (D.saved_h == MOE_SAVED_H_RECOMPUTE) {
+    w.hr = c.take<bf16>(D.cap * 2 * D.f * 2);
+    if (D.mx) {
+      w.w1r_q = c.take<uint8_t>(D.E * 2 * D.f * D.d);
+      w.w1r_s = c.take<uint8_t>(D.E * 2 * D.f * D.d / 32);
+    } else {
+      w.w1r_copy = c.take<bf16>(D.E * 2 * D.f * D.d * 2);
+    }
+  }
 }
 
 int64_t capacity_rows(int64_t T, int k, int E) {
@@ -486,7 +509,7 @@ moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt) {
 }
 
 moe_status_t moe_ctx_set_saved_h(moe_ctx_t ctx, int mode) {
-  if (!ctx || (mode != MOE_SAVED_H_BF16 && mode != MOE_SAVED_H_MXFP8)) return MOE_ERR_INVALID_ARG;
+  if (!ctx || mode < MOE_SAVED_H_BF16 || mode > MOE_SAVED_H_RECOMPUTE) return MOE_ERR_INVALID_ARG;
   ctx->saved_h = mode;
   return MOE_OK;
 }
@@ -607,7 +630,9 @@ moe_status_t moe_unpermute(moe_ctx_t ctx, const void* y_perm, const int32_t* src
 
 size_t moe_saved_size_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int saved_h) {
   if (check_dims(T, d, f, E, k) != MOE_OK) return 0;
-  if (saved_h != MOE_SAVED_H_BF16 && (saved_h != MOE_SAVED_H_MXFP8 || prec != MOE_PREC_MXFP8)) return 0;
+  if (saved_h != MOE_SAVED_H_BF16 && saved_h != MOE_SAVED_H_RECOMPUTE &&
+      (saved_h != MOE_SAVED_H_MXFP8 || prec != MOE_PREC_MXFP8))
+    return 0;
   Dims D = make_dims(T, d, f, E, k, prec, saved_h);
   Carve c(nullptr);
   Saved s;
@@ -632,13 +657,18 @@ size_t moe_fwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe
   return c.off + 1024;
 }
 
-size_t moe_bwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec) {
+size_t moe_bwd_workspace_size_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int saved_h) {
   if (check_dims(T, d, f, E, k) != MOE_OK) return 0;
-  Dims D = make_dims(T, d, f, E, k, prec);
+  if (saved_h < MOE_SAVED_H_BF16 || saved_h > MOE_SAVED_H_RECOMPUTE) return 0;
+  Dims D = make_dims(T, d, f, E, k, prec, saved_h);
   Carve c(nullptr);
   BwdWs w;
   carve_bwd(c, D, w);
   return c.off + 1024;
+}
+
+size_t moe_bwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec) {
+  return moe_bwd_workspace_size_ex(T, k, E, d, f, prec, MOE_SAVED_H_BF16);
 }
 
 moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, const float* topk_prob,
@@ -672,6 +702,11 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
   } else {
     carve_saved(cw, D, s, false);
   }
+
+  // x's gate_up operand: in the workspace, or in the saved buffer when the backward recomputes h
+  uint8_t* x_q = s.xr_q ? s.xr_q : w.x_q;
+  uint8_t* x_s = s.xr_s ? s.xr_s : w.x_s;
+  bf16* x_perm = s.xr ? s.xr : w.x_perm;
 
   // 1. routing: counts, padded offsets, stable permutation, per-row probabilities
   MOE_LAUNCH(ctx, "route", st, launch_route(topk_idx, topk_prob, static_cast<int>(D.Tk), E, static_cast<int>(D.cap), split_sizes, s.split,
@@ -728,8 +763,8 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.mx = 1;
     xa.sf_mma = 1;
     xa.do_row = 1;
-    xa.q_row = w.x_q;
-    xa.s_row = w.x_s;
+    xa.q_row = x_q;
+    xa.s_row = x_s;
     xa.do_col = training;
     xa.q_colT = s.xT_q;
     xa.s_colT = s.xT_s;
@@ -775,7 +810,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     xa.cols = d;
     xa.mx = 0;
     xa.do_row = 1;
-    xa.o_row = w.x_perm;
+    xa.o_row = x_perm;
     xa.do_col = training;
     xa.o_colT = s.xT;
     if (!quant_store_maps(xa, static_cast<int>(1))) return MOE_ERR_CUDA;
@@ -787,7 +822,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     GemmArgs g = gemm_args(ctx);
     // MXFP8: the quantised copy is gate/up interleaved, two 128-row boxes per tile; BF16 reads the
     // unpermuted weights as a 128-row gate box plus the matching 128-row up box.
-    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.x_q) : w.x_perm, D.mx, d, D.cap,
+    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(x_q) : x_perm, D.mx, d, D.cap,
                            d * (D.mx ? 1 : 2)) &&
                     map_3d(&g.tmap_b, w1_base, D.mx, d, 2 * f, E, d * (D.mx ? 1 : 2), w1_stride,
                            D.mx ? gemm_tile_n(EPI_SWIGLU) : gemm_tile_n(EPI_SWIGLU) / 2);
@@ -798,7 +833,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     g.n_tiles = static_cast<int>(f / 128);
     g.gate_up_half = D.mx ? 0 : static_cast<int>(f);
     g.poffsets = s.poff;
-    g.sfa = w.x_s;
+    g.sfa = x_s;
     g.sfa_kb4 = d / 128;
     g.sfb = w.w1_s;
     g.sfb_kb4 = d / 128;
@@ -882,7 +917,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   const int saved_h = ctx->saved_h;
   if (saved_h == MOE_SAVED_H_MXFP8 && prec != MOE_PREC_MXFP8) return MOE_ERR_UNSUPPORTED;
   if (saved_bytes < moe_saved_size_ex(T, k, E, d, f, prec, saved_h)) return MOE_ERR_WORKSPACE;
-  if (workspace_bytes < moe_bwd_workspace_size(T, k, E, d, f, prec)) return MOE_ERR_WORKSPACE;
+  if (workspace_bytes < moe_bwd_workspace_size_ex(T, k, E, d, f, prec, saved_h)) return MOE_ERR_WORKSPACE;
 
   DeviceGuard guard(ctx->device);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -893,6 +928,72 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   BwdWs w;
   Carve cw(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(workspace), 1024)));
   carve_bwd(cw, D, w);
+
+  // 0. recompute mode: h again, from x's saved gate_up operand and W1 (quantised again for MXFP8),
+  //    through the gate_up GEMM with an epilogue that only writes h
+  bf16* h_src = s.h;
+  if (D.saved_h == MOE_SAVED_H_RECOMPUTE) {
+    const void* w1_base;
+    int64_t w1_stride;
+    if (D.mx) {
+      QuantArgs a = quant_args(ctx);
+      for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_gate_up[e];
+      a.src_ld = d;
+      a.rows = 2 * f;
+      a.cols = d;
+      a.mx = 1;
+      a.sf_mma = 1;
+      a.do_row = 1;
+      a.q_row = w.w1r_q;
+      a.s_row = w.w1r_s;
+      a.gate_up_half = f;
+      if (!quant_store_maps(a, static_cast<int>(E))) return MOE_ERR_CUDA;
+      MOE_LAUNCH(ctx, "requantize_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
+      w1_base = w.w1r_q;
+      w1_stride = 2 * f * d;
+    } else {
+      w1_stride = uniform_stride(w_gate_up, E, 2 * f * d * 2);
+      w1_base = w_gate_up[0];
+      if (!w1_stride) {
+        QuantArgs a = quant_args(ctx);
+        for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = w_gate_up[e];
+        a.src_ld = d;
+        a.rows = 2 * f;
+        a.cols = d;
+        a.mx = 0;
+        a.do_row = 1;
+        a.o_row = w.w1r_copy;
+        if (!quant_store_maps(a, static_cast<int>(E))) return MOE_ERR_CUDA;
+        MOE_LAUNCH(ctx, "gather_w_gate_up", st, launch_quant(a, E, ctx->num_sms, st));
+        w1_base = w.w1r_copy;
+        w1_stride = 2 * f * d * 2;
+      }
+    }
+    GemmArgs g = gemm_args(ctx);
+    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(s.xr_q) : s.xr, D.mx, d, D.cap,
+                           d * (D.mx ? 1 : 2)) &&
+                    map_3d(&g.tmap_b, w1_base, D.mx, d, 2 * f, E, d * (D.mx ? 1 : 2), w1_stride,
+                           D.mx ? gemm_tile_n(EPI_SWIGLU) : gemm_tile_n(EPI_SWIGLU) / 2);
+    if (!ok) return MOE_ERR_CUDA;
+    g.kgrouped = 0;
+    g.E = E;
+    g.K = static_cast<int>(d);
+    g.n_tiles = static_cast<int>(f / 128);
+    g.gate_up_half = D.mx ? 0 : static_cast<int>(f);
+    g.poffsets = s.poff;
+    g.sfa = s.xr_s;
+    g.sfa_kb4 = d / 128;
+    g.sfb = w.w1r_s;
+    g.sfb_kb4 = d / 128;
+    g.sfb_expert_rows = 2 * f;
+    if (D.mx && !sf_maps(g, D.cap, E * 2 * f, gemm_tile_n(EPI_SWIGLU))) return MOE_ERR_CUDA;
+    g.epi.f = f;
+    g.epi.cap = D.cap;
+    g.epi.p_perm = s.pperm;
+    g.epi.h = w.hr;  // no a outputs: the epilogue stops after saving h
+    MOE_LAUNCH(ctx, "gemm_recompute_h", st, launch_grouped_gemm(g, D.mx, EPI_SWIGLU, ctx->num_sms, st));
+    h_src = w.hr;
+  }
 
   // 1. dy gathered by expert: row-wise (K = d, dgrad of down) and token-axis transposed (wgrad of down)
   {
@@ -953,7 +1054,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     GemmArgs g = gemm_args(ctx);
     const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dy_q) : w.dy_perm, D.mx, d, D.cap, d * es) &&
                     map_3d(&g.tmap_b, w2c, D.mx, d, f, E, d * es, f * d * es, gemm_tile_n(EPI_DSWIGLU)) &&
-                    (s.h_q || map_2d(&g.tmap_h, s.h, false, 2 * f, D.cap, 2 * f * 2));  // bf16 boxes, 128 x 64
+                    (s.h_q || map_2d(&g.tmap_h, h_src, false, 2 * f, D.cap, 2 * f * 2));  // bf16 boxes, 128 x 64
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
@@ -970,7 +1071,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     ep.f = f;
     ep.cap = D.cap;
     ep.p_perm = s.pperm;
-    ep.h = s.h;      // bf16 h staged by TMA, or
+    ep.h = h_src;    // bf16 h (saved or recomputed) staged by TMA, or
     ep.h_q = s.h_q;  // MXFP8 h read by the epilogue (the kernel instance without h staging)
     ep.h_s = s.h_s;
     ep.dump = ctx->dbg_dh;
@@ -1101,7 +1202,8 @@ void* moe_buffer_address_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_p
                          {"src_to_sorted", s.src2s}, {"prob_perm", s.pperm}, {"w1c_q", s.w1c_q},
                          {"w1c_s", s.w1c_s}, {"w2c_q", s.w2c_q}, {"w2c_s", s.w2c_s}, {"xT_q", s.xT_q},
                          {"xT_s", s.xT_s}, {"aT_q", s.aT_q}, {"aT_s", s.aT_s}, {"xT", s.xT}, {"aT", s.aT},
-                         {"h", s.h},       {"h_q", s.h_q},     {"h_s", s.h_s}};
+                         {"h", s.h},       {"h_q", s.h_q},     {"h_s", s.h_s},   {"xr_q", s.xr_q},
+                         {"xr_s", s.xr_s}, {"xr", s.xr}};
     for (const Named& e : tab)
       if (!std::strcmp(e.n, name) && e.p) return e.p;
     if (which == 0) return nullptr;
@@ -1124,7 +1226,7 @@ void* moe_buffer_address_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_p
                          {"dh_q", w.dh_q},   {"dh_s", w.dh_s},     {"dhT_q", w.dhT_q}, {"dhT_s", w.dhT_s},
                          {"dy_perm", w.dy_perm}, {"dyT", w.dyT},   {"dh", w.dh},       {"dhT", w.dhT},
                          {"w1T", w.w1T},     {"w2T", w.w2T},       {"dx_perm", w.dx_perm},
-                         {"dp_part", w.dp_part}};
+                         {"dp_part", w.dp_part}, {"hr", w.hr},     {"w1r_q", w.w1r_q}, {"w1r_s", w.w1r_s}};
     for (const Named& e : tab)
       if (!std::strcmp(e.n, name) && e.p) return e.p;
   }

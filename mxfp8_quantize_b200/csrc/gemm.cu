@@ -612,6 +612,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
 #pragma unroll
             for (int i = 0; i < 2; ++i) ptx::st_global_v8(hu + 16 * i, pack_bf16x8(uv + 16 * i), pack_bf16x8(uv + 16 * i + 8));
           }
+          if (!ep.q_row && !ep.o_row) continue;  // h only (the backward recomputing h)
 #pragma unroll
           for (int i = 0; i < 32; ++i) gv[i] = gv[i] * sigmoid_f(gv[i]) * uv[i] * p;  // a, in place
           if (ep.dump) {

@@ -374,3 +374,35 @@ def test_fused_forward_matches_two_launches(precision, T):
         assert torch.equal(a, b), name
     ref = _oracle(inp, precision, backward=False)
     parity(f"fused_forward_{precision}_T{T}.y", res[1][0].numpy(), ref["y"], TOL[precision])
+
+
+@pytest.mark.parametrize("precision", ["mxfp8", "bf16"])
+def test_recompute_h_matches_saved_h(precision):
+    """MOE_SAVED_H_RECOMPUTE: the forward saves x's gate_up operand instead of h, and the backward
+    quantises W1 again and re-runs the gate_up GEMM to regenerate h.  Same kernels on the same
+    operands: every gradient is bit-identical to the saved-bf16-h backward, with a smaller saved
+    buffer; and the regenerated h equals the one the forward saved."""
+    cfg = workloads.scaled_config(workloads.CONFIGS["small_mxfp8"], precision=precision, T=1200, seed=45)
+    T, d, f, E, k = cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
+    inp = workloads.make_inputs(cfg, with_dy=True)
+    dev = {n: t.cuda() for n, t in inp.items()}
+    res, keep = [], {}
+    for mode in ("bf16", "recompute"):
+        bws = torch.zeros(moe.sizes(T, d, f, E, k, precision, True, mode)["bwd_ws"], dtype=torch.uint8, device="cuda")
+        y, saved = moe.moe_grouped_mlp_fwd(dev["x"], dev["topk_idx"], dev["topk_prob"], dev["w_gate_up"],
+                                           dev["w_down"], precision=precision, training=True, saved_h=mode)
+        dx, dw1, dw2, dp = moe.moe_grouped_mlp_bwd(dev["dy"], saved, dev["w_gate_up"], dev["w_down"], workspace=bws)
+        moe.get_status(0)
+        keep[mode] = (saved, bws)
+        res.append([t.float().cpu() if t.dtype == torch.bfloat16 else t.cpu() for t in (y, dx, dw1, dw2, dp)])
+    for name, a, b in zip(("y", "dx", "dw_gate_up", "dw_down", "d_topk_prob"), *res):
+        assert torch.equal(a, b), name
+    sz = {m: moe.sizes(T, d, f, E, k, precision, True, m)["saved"] for m in ("bf16", "recompute")}
+    assert sz["recompute"] < sz["bf16"]
+    cap = moe.capacity_rows(T, k, E)
+    dims = (T, d, f, E, k, precision)
+    h_saved = moe.buffer_view(keep["bf16"][0].buf, 0, "h", dims, True, cap * 2 * f, torch.bfloat16)
+    h_again = moe.buffer_view(keep["recompute"][1], 2, "hr", dims, True, cap * 2 * f, torch.bfloat16,
+                              saved_h="recompute")
+    Tp = int(moe.buffer_view(keep["bf16"][0].buf, 0, "poffsets", dims, True, E + 1, torch.int32)[E])
+    assert torch.equal(h_saved[: Tp * 2 * f], h_again[: Tp * 2 * f])
