@@ -245,7 +245,6 @@ def torch_loop_context(cfg, device: int, steps: int = 5, warmup: int = 2):
     library path, not this build's kernels.  Returns TFLOP/s and ms per fwd+bwd step."""
     dev = torch.device("cuda", device)
     inp = workloads.make_inputs(cfg, with_dy=True)
-    moe.set_fused_forward(local_rank, args.fused_forward)
     x = inp["x"].to(dev)
     idx = inp["topk_idx"].to(dev).long()
     prob = inp["topk_prob"].to(dev).to(torch.bfloat16)
@@ -303,6 +302,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     import mxfp8_quantize_b200 as moe
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    moe.set_fused_forward(local_rank, args.fused_forward)
     inp = workloads.make_inputs(cfg, with_dy=True)
     x = inp["x"].to(dev)
     idx = inp["topk_idx"].to(dev)
