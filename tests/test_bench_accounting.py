@@ -29,3 +29,18 @@ def test_weight_quantiser_bytes():
     assert abs(b - 3.82e9) < 0.01e9
     kind, b = bench.kernel_work(workloads.CONFIGS["mixtral_bf16"], "transpose_w_down")
     assert kind == "hbm" and b == cfg.E * cfg.d * cfg.f * 4  # bf16 in, bf16 transposed out
+
+
+def test_fused_forward_work_is_both_forward_gemms():
+    cfg = workloads.CONFIGS["mixtral_mxfp8"]
+    kind, w = bench.kernel_work(cfg, "gemm_fused_forward")
+    assert kind == "tensor"
+    assert w == bench.kernel_work(cfg, "gemm_gate_up_swiglu")[1] + bench.kernel_work(cfg, "gemm_down")[1]
+    assert w == cfg.flops_fwd()
+
+
+def test_oracle_sample_is_shared_by_both_cpu_legs():
+    """The cpu_baseline object and the --impl reference arm time the same bounded slice."""
+    import inspect
+    src = inspect.getsource(bench.main)
+    assert src.count("ORACLE_SAMPLE") >= 2
