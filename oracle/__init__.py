@@ -23,8 +23,9 @@ for biological foundation models" with Transformer Engine / BioNeMo):
 
 Modules:
   mx       E4M3 / E8M0 codec (round-up shared exponent, RNE, satfinite)
+  fp8      per-tensor FP8 codec (one fp32 scale per tensor, current scaling)
   routing  stable counting-sort permutation, padded expert segments
-  moe      per-expert-loop forward and backward (MXFP8 or BF16 operands)
+  moe      per-expert-loop forward and backward (MXFP8, per-tensor FP8 or BF16 operands)
 
 Parity unpinned: Transformer Engine's own numerics (its exact shared-exponent
 rule, gradient formats, where it applies the routing probability).  The pages

@@ -40,6 +40,13 @@ Precision modes and the readings they encode:
   MXFP8 instead of bf16 (``saved_h="mxfp8"``: E4M3, blocks of 32 along 2f,
   which never straddle the gate and up halves since f % 32 == 0); the
   backward then reads g and u dequantised from it.
+* "fp8": per-tensor FP8 with current scaling (``oracle.fp8``): every GEMM
+  operand of every expert is quantised as one tensor with its own fp32 scale;
+  E4M3 elements, E5M2 for the gradient operands dy and dh with
+  ``grad_format="e5m2"``.  a and dh are rounded to bf16 before they are
+  quantised (the tensor is materialised in 16 bits so that its maximum is
+  known before any of it is quantised).  Products as for mxfp8; h saved as
+  bf16.
 * "bf16": the same chain with bf16 GEMM operands (a, dh rounded to bf16) and
   fp32 products.
 * "fp64": no quantisation and no rounding anywhere (used to pin the algebra
@@ -49,7 +56,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from . import mx
+from . import fp8, mx
 from .routing import route
 
 
@@ -81,6 +88,7 @@ def gemm(A, B, precision: str, scale_rule: str = "ceil", a_fmt: str = "e4m3") ->
     mxfp8: A quantised in blocks of 32 along its axis 1 (K) with elements ``a_fmt``, B along its
            axis 0 (K) with E4M3 elements, both with the shared-exponent rule ``scale_rule``
            (oracle.mx).
+    fp8:   A and B each quantised as one tensor (oracle.fp8), A with elements ``a_fmt``, B E4M3.
     bf16:  both operands rounded to bf16.   fp64: used as given.
     The product is formed in fp64 (callers round it).
     """
@@ -89,6 +97,9 @@ def gemm(A, B, precision: str, scale_rule: str = "ceil", a_fmt: str = "e4m3") ->
     if precision == "mxfp8":
         A = mx.fake_quant(A, axis=1, rule=scale_rule, fmt=a_fmt)
         B = mx.fake_quant(B, axis=0, rule=scale_rule)
+    elif precision == "fp8":
+        A = fp8.fake_quant(A, a_fmt)
+        B = fp8.fake_quant(B)
     elif precision == "bf16":
         A = bf16_round(A).astype(np.float64)
         B = bf16_round(B).astype(np.float64)
@@ -124,7 +135,7 @@ def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: in
     MXFP8 shared-exponent rule of every quantisation (forward and backward); ``grad_format`` the
     element format of the gradient operands (dy, dh) of the four backward GEMMs; ``saved_h`` the
     format h is kept in for the backward ("bf16" or "mxfp8")."""
-    if saved_h not in ("bf16", "mxfp8"):
+    if saved_h not in ("bf16", "mxfp8") or (saved_h == "mxfp8" and precision != "mxfp8"):
         raise ValueError(saved_h)
     x = np.asarray(x, dtype=np.float64)
     T, d = x.shape
@@ -161,6 +172,8 @@ def forward(x, topk_idx, topk_prob, w_gate_up, w_down, precision: str, align: in
         a = silu(g) * u * pe[:, None]
         if precision != "fp64":
             a = f32(a)
+        if precision == "fp8":
+            a = bf16_round(a)
         ye = gemm(a, W2.T, precision, scale_rule)
         y_perm[lo:hi] = _round_out(ye, precision)
         h_all[lo:hi] = h
@@ -230,6 +243,8 @@ def backward(dy, state, w_gate_up, w_down):
         if precision != "fp64":
             dh = f32(dh)
             dp = f32(dp)
+        if precision == "fp8":
+            dh = bf16_round(dh)
 
         # gate_up projection: dgrad (K = 2f) and wgrad (K = tokens)
         dx_perm[lo:hi] = _round_out(gemm(dh, W1, precision, rule, gf), precision)

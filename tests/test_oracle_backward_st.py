@@ -85,6 +85,23 @@ def _fq_mx(v: torch.Tensor, axis: int, rule: str = "ceil") -> torch.Tensor:
     return q.movedim(-1, axis)
 
 
+def _fq_pt(v: torch.Tensor, fmt: str = "e4m3") -> torch.Tensor:
+    """Per-tensor FP8 fake quantisation: s = fp32(vmax / amax) (1 for an all-zero tensor, the
+    largest fp32 when the quotient overflows), elements by torch's own float8 conversion of the
+    fp32 product v * s, value code / s."""
+    vmax, dt = (448.0, torch.float8_e4m3fn) if fmt == "e4m3" else (57344.0, torch.float8_e5m2)
+    v32 = v.to(torch.float32)
+    amax = v32.abs().max()
+    if amax > 0:
+        s = torch.tensor(vmax, dtype=torch.float32) / amax
+        if torch.isinf(s):
+            s = torch.tensor(torch.finfo(torch.float32).max, dtype=torch.float32)
+    else:
+        s = torch.tensor(1.0, dtype=torch.float32)
+    q = (v32 * s).clamp(-vmax, vmax).to(dt).to(torch.float64)
+    return q / s.to(torch.float64)
+
+
 def _to_f32(v):
     return v.to(torch.float32).to(torch.float64)
 
@@ -99,11 +116,15 @@ ROUND = {"f32": _to_f32, "bf16": _to_bf16}
 def _operand(v, axis, mode):
     if mode == "bf16":
         return _to_bf16(v)
+    if mode.startswith("fp8"):  # one scale for the whole tensor: the axis does not matter
+        return _fq_pt(v)
     return _fq_mx(v, axis, "floor" if mode == "mxfp8-floor" else "ceil")
 
 
 def _grad_operand(v, axis, mode):
     """The gradient operand of a backward product (E5M2 elements in the gradient-format variant)."""
+    if mode == "fp8-e5m2grad":
+        return _fq_pt(v, "e5m2")
     return _fq_mx5(v, axis) if mode == "mxfp8-e5m2grad" else _operand(v, axis, mode)
 
 
@@ -128,16 +149,19 @@ class _QuantLinear(torch.autograd.Function):
 
 
 class _ScaledSwiGLU(torch.autograd.Function):
-    """a = silu(g) * u * p from fp32 h (result rounded to fp32).  Backward: autograd of the same
-    expression evaluated on h as saved in bf16; dh and dp rounded to fp32."""
+    """a = silu(g) * u * p from fp32 h (result rounded to fp32, then to bf16 in the per-tensor FP8
+    mode).  Backward: autograd of the same expression evaluated on h as saved in bf16; dh and dp
+    rounded to fp32 (dh then to bf16 in the per-tensor FP8 mode)."""
 
     @staticmethod
     def forward(ctx, h, p):
         ctx.save_for_backward(h, p)
         f = h.shape[1] // 2
-        return _to_f32(torch.nn.functional.silu(h[:, :f]) * h[:, f:] * p)
+        a = _to_f32(torch.nn.functional.silu(h[:, :f]) * h[:, f:] * p)
+        return _to_bf16(a) if _ScaledSwiGLU.act_bf16 else a
 
     saved_h = "bf16"   # format h is read back in for the backward ("mxfp8": E4M3 blocks of 32 along 2f)
+    act_bf16 = False   # a and dh materialised in bf16 before they are quantised (per-tensor FP8)
 
     @staticmethod
     def backward(ctx, da):
@@ -149,7 +173,8 @@ class _ScaledSwiGLU(torch.autograd.Function):
         with torch.enable_grad():
             a = torch.nn.functional.silu(hb[:, :f]) * hb[:, f:] * pp
             dh, dp = torch.autograd.grad(a, (hb, pp), da)
-        return _to_f32(dh), _to_f32(dp)
+        dh = _to_bf16(dh) if _ScaledSwiGLU.act_bf16 else _to_f32(dh)
+        return dh, _to_f32(dp)
 
 
 def _reference(x, idx, prob, w1, w2, dy, mode):
@@ -223,12 +248,15 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("mode", ["mxfp8", "bf16", "mxfp8-floor", "mxfp8-e5m2grad", "mxfp8-savedh"])
+@pytest.mark.parametrize("mode", ["mxfp8", "bf16", "mxfp8-floor", "mxfp8-e5m2grad", "mxfp8-savedh", "fp8",
+                                  "fp8-e5m2grad"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"T{s['T']}_E{s['E']}_k{s['k']}_{s['routing']}")
 def test_quantised_backward_matches_straight_through_autograd(shape, mode):
     """mxfp8-floor: the oracle's OCP floor shared-exponent variant, in every quantisation;
     mxfp8-e5m2grad: E5M2 elements for the gradient operand of every backward product;
-    mxfp8-savedh: h kept as MXFP8 for the backward (the long-sequence memory variant)."""
+    mxfp8-savedh: h kept as MXFP8 for the backward (the long-sequence memory variant);
+    fp8: per-tensor FP8 (one scale per expert operand, a and dh materialised in bf16);
+    fp8-e5m2grad: the same with E5M2 gradient operands."""
     inp = _inputs(**shape)
     args = [inp[n] for n in ("x", "topk_idx", "topk_prob", "w_gate_up", "w_down")]
     if mode == "mxfp8-floor":
@@ -237,15 +265,19 @@ def test_quantised_backward_matches_straight_through_autograd(shape, mode):
         y, st = moe.forward(*args, "mxfp8", grad_format="e5m2")
     elif mode == "mxfp8-savedh":
         y, st = moe.forward(*args, "mxfp8", saved_h="mxfp8")
+    elif mode == "fp8-e5m2grad":
+        y, st = moe.forward(*args, "fp8", grad_format="e5m2")
     else:
         y, st = moe.forward(*args, mode)
     got = moe.backward(inp["dy"], st, inp["w_gate_up"], inp["w_down"])
     got["y"] = y
     _ScaledSwiGLU.saved_h = "mxfp8" if mode == "mxfp8-savedh" else "bf16"
+    _ScaledSwiGLU.act_bf16 = mode.startswith("fp8")
     try:
         ref = _reference(*args, inp["dy"], "mxfp8" if mode == "mxfp8-savedh" else mode)
     finally:
         _ScaledSwiGLU.saved_h = "bf16"
+        _ScaledSwiGLU.act_bf16 = False
     got["dh_slot"] = got["dh_perm"][st["route"]["src_to_sorted"]]
     for name in ("y", "dx", "dw_gate_up", "dw_down", "d_topk_prob", "dh_slot"):
         r = ref[name].numpy()
