@@ -54,7 +54,8 @@ def kernel_work(cfg, name):
     """(kind, algorithmic amount per launch): FLOPs for GEMMs, bytes for the HBM-bound kernels."""
     Tk, T, d, f, E, k = cfg.Tk, cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
     mx = cfg.precision == "mxfp8"
-    q = 1.0 + 1.0 / 32  # bytes per quantised element (code + its share of a scale)
+    q8 = cfg.precision in ("mxfp8", "fp8")
+    q = (1.0 + 1.0 / 32) if mx else 1.0  # bytes per quantised element (code + its share of a scale)
     gemm = {
         "gemm_gate_up_swiglu": 2.0 * Tk * d * 2 * f,
         "gemm_down": 2.0 * Tk * f * d,
@@ -66,7 +67,7 @@ def kernel_work(cfg, name):
     }
     if name in gemm:
         return "tensor", gemm[name]
-    out_b = 2 * q if mx else 4.0  # row + column outputs per element
+    out_b = 2 * q if q8 else 4.0  # row + column outputs per element
     hbm = {
         "quantize_w_gate_up": E * 2 * f * d * (2 + out_b),
         "quantize_w_down": E * d * f * (2 + out_b),
@@ -79,6 +80,13 @@ def kernel_work(cfg, name):
         "unpermute_dx": Tk * d * 2 + T * d * 2 + Tk * 4,
         "route": Tk * 4 * 3,
         "dprob_reduce": Tk * 4 * 2,
+        # per-tensor FP8: the maxima (reads), and the quantisation of the bf16 a / dh rows both ways
+        "amax_w_gate_up": E * 2 * f * d * 2,
+        "amax_w_down": E * d * f * 2,
+        "amax_x": Tk * d * 2,
+        "amax_dy": Tk * d * 2,
+        "quantize_a": Tk * f * (2 + out_b),
+        "quantize_dh": Tk * 2 * f * (2 + out_b),
     }
     return "hbm", hbm.get(name, 0.0)
 
@@ -213,7 +221,7 @@ def measure_peaks(args):
     torch.cuda.set_device(dev)
     out = {}
     for name, prec, refresh in (("mxfp8", "mxfp8", False), ("mxfp8_scale_refresh", "mxfp8", True),
-                                ("bf16", "bf16", False)):
+                                ("fp8", "fp8", False), ("bf16", "bf16", False)):
         for regime, ms in (("burst", 100.0), ("sustained", 4000.0)):
             time.sleep(1.0)
             clk = ClockSampler(dev, args.clocks_dir)
@@ -385,11 +393,11 @@ def run_ours(args, cfg, rank, world, local_rank):
             per.setdefault(name, []).append(open_ev.pop(name).elapsed_time(ev))
     kern = {}
     peaks, peak_src = load_peaks()
-    mx = cfg.precision == "mxfp8"
+    q8 = cfg.precision in ("mxfp8", "fp8")
     # tensor peak: the peak loop measured live on this GPU (burst); the file's bf16 burst figure
-    # (times the nominal fp8/bf16 ratio of 2 for MXFP8) is reported beside it
+    # (times the nominal fp8/bf16 ratio of 2 for the 8-bit kinds) is reported beside it
     tensor_peak_tf = loop_tflops
-    nominal_rule = peaks["bf16_tflops"] * (2.0 if mx else 1.0)
+    nominal_rule = peaks["bf16_tflops"] * (2.0 if q8 else 1.0)
     mhz = clk.get("sm_mhz")
     for name, v in per.items():
         avg = float(np.mean(v))
@@ -421,14 +429,15 @@ def run_ours(args, cfg, rank, world, local_rank):
             h.update(open(os.path.join(ROOT, fn), "rb").read())
         if rec.get("sources") and h.hexdigest()[:12] == rec.get("sources_sha1"):
             traffic = rec.get(cfg.name, {}).get(dom)  # counters taken on this very kernel source
+    kind_name = {"mxfp8": "kind::mxf8f6f4 block-scaled", "fp8": "kind::f8f6f4"}.get(cfg.precision, "kind::f16")
     roofline = {"bound": kind, "kernel": dom, "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": unit,
                 "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_source": (f"measured live: tcgen05 {'kind::mxf8f6f4 block-scaled' if mx else 'kind::f16'} "
+                "peak_source": (f"measured live: tcgen05 {kind_name} "
                                 f"peak loop (operands resident in shared memory, one CTA per SM), run back to back "
                                 f"for {round(loop_ms)} ms (the length of the timed region) just before it; its 0.1 s "
                                 f"burst was {round(peak_burst, 1)} TFLOP/s (frac {round(achieved / peak_burst, 4)}); "
                                 f"{peak_src} bf16 burst {peaks['bf16_tflops']}"
-                                f"{' x 2 (nominal fp8/bf16 ratio)' if mx else ''} = {round(nominal_rule, 1)} TFLOP/s "
+                                f"{' x 2 (nominal fp8/bf16 ratio)' if q8 else ''} = {round(nominal_rule, 1)} TFLOP/s "
                                 f"(frac {round(achieved / nominal_rule, 4)})"
                                 if kind == "tensor" else f"{peak_src}: HBM copy {peaks['hbm_gbs']} GB/s")}
 
@@ -576,7 +585,9 @@ def main():
                "kind": "oracle", "sample": desc + f"; median of {len(ts)} runs of {float(np.median(ts)):.1f} s"}
     line = {"metric": METRIC, "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(res["ms"], 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "mxfp8-e4m3 (fp32 accumulate)" if cfg.precision == "mxfp8" else "bf16",
+            "vs_baseline": None, "dtype": {"mxfp8": "mxfp8-e4m3 (fp32 accumulate)",
+                                                      "fp8": "fp8-e4m3 per-tensor (fp32 accumulate)"}.get(cfg.precision,
+                                                                                                          "bf16"),
             "data": "synthetic", "config": config_desc(cfg),
             "tokens_per_s": round(world * cfg.T / (res["ms"] * 1e-3), 1),
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["launches"],

@@ -52,7 +52,10 @@ typedef enum {
   MOE_ERR_WORKSPACE = 7     /* a workspace / saved buffer is smaller than required        */
 } moe_status_t;
 
-typedef enum { MOE_PREC_BF16 = 0, MOE_PREC_MXFP8 = 1 } moe_precision_t;
+/* GEMM operand precision of the fused layer.  FP8 is per-tensor FP8 with current scaling (ai4snews
+ * paragraph 2: FP8 and MXFP8 training; MXFP8 being the format that adds a scale per block of 32,
+ * plain FP8 keeps one scale per tensor): see "Per-tensor FP8" at the fused layer below. */
+typedef enum { MOE_PREC_BF16 = 0, MOE_PREC_MXFP8 = 1, MOE_PREC_FP8 = 2 } moe_precision_t;
 
 /* flags of mxfp8_quantize */
 #define MXFP8_ROWWISE 1        /* blocks of 32 along each row                              */
@@ -60,6 +63,11 @@ typedef enum { MOE_PREC_BF16 = 0, MOE_PREC_MXFP8 = 1 } moe_precision_t;
 #define MXFP8_SF_MMA_LAYOUT 4  /* scales in the tensor-core tile layout instead of row-major */
 #define MXFP8_FLAG_SCALE_FLOOR 8 /* shared exponent by the OCP floor rule instead of round-up   */
 #define MXFP8_FLAG_E5M2 16       /* E5M2 elements (max 57344) instead of E4M3                   */
+
+/* flags of fp8_quantize */
+#define FP8_ROWWISE 1        /* codes in the source layout (required)                      */
+#define FP8_COLWISE_T 2      /* the same codes transposed as well                          */
+#define FP8_FLAG_E5M2 16     /* E5M2 elements (max 57344) instead of E4M3 (max 448)         */
 
 /* Element format of the gradient operands (dy, dh) of the backward GEMMs (moe_ctx_set_grad_format). */
 #define MOE_GRAD_E4M3 0
@@ -99,8 +107,10 @@ moe_status_t moe_ctx_set_debug_dump(moe_ctx_t ctx, float* a_f32, float* dh_f32);
  * MXFP8_SCALE_FLOOR.  Calls already enqueued are not affected. */
 moe_status_t moe_ctx_set_scale_rule(moe_ctx_t ctx, int rule);
 
-/* Element format of the MXFP8 gradient operands of the fused layer's backward with this context
- * (ai4snews paragraph 2: FP8 and MXFP8 training): MOE_GRAD_E4M3 (default) or MOE_GRAD_E5M2.
+/* Element format of the MXFP8 (or per-tensor FP8) gradient operands of the fused layer's backward
+ * with this context (ai4snews paragraph 2: FP8 and MXFP8 training): MOE_GRAD_E4M3 (default) or
+ * MOE_GRAD_E5M2.  Per-tensor FP8 takes it the same way: dy and dh get E5M2 codes with scales
+ * computed against 57344.
  * With E5M2, dy (quantised along d and along the tokens) and the requantised dh take E5M2
  * elements (round to nearest even, saturating at 57344) with the same E8M0 scales per 32 values,
  * the shared exponent computed against 57344 (round-up: the smallest e with amax <= 57344 * 2^e;
@@ -116,14 +126,16 @@ moe_status_t moe_ctx_set_grad_format(moe_ctx_t ctx, int fmt);
  *   MOE_SAVED_H_MXFP8 MXFP8 h: E4M3 codes [capacity, 2f] with one E8M0 scale per 32 values along
  *                     2f (row-major [capacity, 2f/32]), quantised in the gate_up GEMM's epilogue with
  *                     the context's scale rule; the dSwiGLU epilogue reads g and u dequantised from
- *                     it.  About half the bytes; MXFP8 precision only (MOE_ERR_UNSUPPORTED for BF16).
+ *                     it.  About half the bytes; MXFP8 precision only (MOE_ERR_UNSUPPORTED otherwise).
  *   MOE_SAVED_H_RECOMPUTE no h at all: the forward keeps x's gate_up operand instead (MXFP8 row-wise
  *                     codes and scales, or the BF16 gathered rows, [capacity, d]); the backward
  *                     quantises W1 again (MXFP8), re-runs the gate_up GEMM with an epilogue that only
  *                     writes h into its workspace (moe_bwd_workspace_size_ex), and goes on as with a
  *                     saved bf16 h, giving the same results bit for bit.  Costs one more gate_up GEMM
- *                     (and W1 quantisation) per backward.
- * moe_saved_size_ex / moe_bwd_workspace_size_ex give the buffer sizes for a mode. */
+ *                     (and W1 quantisation) per backward.  MXFP8 and BF16 only.
+ * Per-tensor FP8 saves h in bf16 only (MOE_ERR_UNSUPPORTED for the other two).
+ * moe_saved_size_ex / moe_bwd_workspace_size_ex give the buffer sizes for a mode (0 for an
+ * unsupported combination). */
 #define MOE_SAVED_H_BF16 0
 #define MOE_SAVED_H_MXFP8 1
 #define MOE_SAVED_H_RECOMPUTE 2
@@ -136,7 +148,8 @@ moe_status_t moe_ctx_set_saved_h(moe_ctx_t ctx, int mode);
  * 128-row block has written its rows of a, which the gate_up epilogues release through one
  * counter per row block in the forward workspace.  The kernel keeps one CTA on every SM for its
  * whole run and its CTAs wait on one another, so it needs the GPU to itself: kernels of other
- * streams that hold SMs meanwhile can make those waits expire.  Default off. */
+ * streams that hold SMs meanwhile can make those waits expire.  Default off.  Per-tensor FP8 keeps
+ * two launches whatever the setting: a is quantised only once its expert's maximum is complete. */
 moe_status_t moe_ctx_set_fused_forward(moe_ctx_t ctx, int on);
 
 /* Test hook for the bounded in-kernel waits (tests only).  With ``stall`` non-zero, every CTA of
@@ -196,6 +209,25 @@ moe_status_t mxfp8_dequantize(moe_ctx_t ctx, const uint8_t* q, const uint8_t* s,
                               int sf_mma_layout, float* out, void* stream);
 
 /* ---------------------------------------------------------------------------------------
+ * fp8_quantize: bf16 -> per-tensor FP8 with current scaling (ai4snews paragraph 2: FP8 and MXFP8
+ * training; plain FP8 has no block scales, so one scale serves the whole tensor).
+ *
+ * x        bf16 [batch, rows, cols], each batch one tensor
+ * flags    FP8_ROWWISE (required), optionally | FP8_COLWISE_T, | FP8_FLAG_E5M2
+ * q_row    uint8 [batch, rows, cols] codes
+ * q_colT   uint8 [batch, cols, rows] the same codes transposed (FP8_COLWISE_T)
+ * scale    fp32 [batch] out: the scale s of each tensor (also used as scratch during the call)
+ *
+ * s = vmax / amax rounded to nearest in fp32, amax the tensor's largest magnitude, vmax 448 (E4M3)
+ * or 57344 (E5M2); s = 1 for an all-zero tensor; the largest finite fp32 when the quotient
+ * overflows.  Code = E4M3 (E5M2) of the fp32 product v * s, rounded to nearest even, saturating;
+ * the value it stands for is code / s.
+ * Shapes: rows % 128 == 0, cols % 128 == 0 (MOE_ERR_SHAPE otherwise); batch <= MOE_MAX_EXPERTS
+ * (MOE_ERR_UNSUPPORTED); x, q_row, q_colT 16-byte aligned (MOE_ERR_INVALID_ARG). */
+moe_status_t fp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t rows, int64_t cols, int flags,
+                          uint8_t* q_row, uint8_t* q_colT, float* scale, void* stream);
+
+/* ---------------------------------------------------------------------------------------
  * Routing bookkeeping and token permutation (sitech.ge "Grouped experts instead of a Python
  * loop": GroupedLinear gathers each expert's tokens and takes per-expert counts).
  *
@@ -241,6 +273,15 @@ moe_status_t moe_unpermute(moe_ctx_t ctx, const void* y_perm, const int32_t* src
  * are quantised from the bf16 masters inside each call.  a is requantised straight from the
  * gate_up GEMM's epilogue into the down GEMM's operand; h never goes to memory except the bf16
  * copy saved for the backward when ``training`` is set.  Products accumulate in fp32.
+ *
+ * Per-tensor FP8 (MOE_PREC_FP8): every GEMM operand of every expert is one tensor with one scale
+ * (fp8_quantize's rule): W1_e, W2_e, expert e's rows of x, of a, of dy and of dh.  The weights and
+ * the gathered rows of x / dy are quantised after a pass that finds their maxima; a and dh leave
+ * their GEMM epilogues as bf16 rows together with their per-expert maxima and are quantised in a
+ * pass of their own.  One set of codes serves both GEMMs that read a tensor (the transposed copy
+ * holds the same codes).  The GEMMs run on the kind::f8f6f4 tensor-core instructions and multiply
+ * each expert's fp32 accumulator by 1/s_A * 1/s_B.  E4M3 elements; dy and dh take the context's
+ * gradient format.
  *
  * w_gate_up, w_down, dw_gate_up, dw_down are HOST arrays of E device pointers (each expert
  * keeps its own weight tensor, ai4snews paragraph 1).
@@ -307,8 +348,9 @@ moe_status_t moe_grouped_mlp_fwd_noalloc(const void* x, const int32_t* topk_idx,
  * MXFP8 GEMMs run on Blackwell's block-scaled tensor-core instructions (ai4snews, paragraph 2);
  * this measures what those instructions deliver on this GPU with nothing else in the way.
  * Enqueues one kernel: one CTA per SM, each issuing ``iters`` groups of four tcgen05 MMAs of
- * M = 128, N = 256 (K = 32 E4M3 with E8M0 scales per MMA for MXFP8, kind::mxf8f6f4; K = 16 bf16
- * for BF16, kind::f16) on operands resident in shared memory, into one TMEM accumulator.  It
+ * M = 128, N = 256 (K = 32 E4M3 with E8M0 scales per MMA for MXFP8, kind::mxf8f6f4; K = 32 E4M3
+ * for per-tensor FP8, kind::f8f6f4; K = 16 bf16 for BF16, kind::f16) on operands resident in
+ * shared memory, into one TMEM accumulator.  It
  * reads and writes no global memory except the context's status word.  ``scale_refresh``
  * (MXFP8 only) also copies the scale tiles shared memory -> TMEM before every group, as the
  * grouped GEMM mainloop does per 128-wide K step.  The caller times it (CUDA events on
@@ -323,11 +365,13 @@ double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters)
  * dimensions, given the buffer's base address ``base``; NULL for an unknown name.  Names:
  * saved: split_sizes poffsets sorted_to_src src_to_sorted prob_perm w1c_q w1c_s w2c_q w2c_s
  *        xT_q xT_s aT_q aT_s xT aT h (with moe_buffer_address_ex: h_q h_s for MOE_SAVED_H_MXFP8,
- *        xr_q xr_s xr for MOE_SAVED_H_RECOMPUTE)
+ *        xr_q xr_s xr for MOE_SAVED_H_RECOMPUTE); per-tensor FP8: pt_amax, the [4][E] maxima
+ *        (fp32) of x, W1, W2 and a
  * forward workspace: w1_q w1_s w2_q w2_s x_q x_s a_q a_s x_perm a y_perm (+ the routing names
- *        when training == 0)
+ *        when training == 0; per-tensor FP8 inference: pt_amax)
  * backward workspace: dy_q dy_s dyT_q dyT_s dh_q dh_s dhT_q dhT_s dy_perm dyT dh dhT w1T w2T
- *        dx_perm dp_part (+ hr w1r_q w1r_s for MOE_SAVED_H_RECOMPUTE)
+ *        dx_perm dp_part (+ hr w1r_q w1r_s for MOE_SAVED_H_RECOMPUTE; per-tensor FP8: pt_amax,
+ *        the [2][E] maxima of dy and dh)
  * Scales (*_s) are in the tensor-core tile layout described at mxfp8_quantize. */
 void* moe_buffer_address(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
                          int which, void* base, const char* name);

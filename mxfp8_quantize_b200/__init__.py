@@ -1,12 +1,13 @@
-"""Python binding of libmoemx: the grouped MoE expert MLP with MXFP8 / BF16 operands on B200.
+"""Python binding of libmoemx: the grouped MoE expert MLP with MXFP8 / per-tensor FP8 / BF16
+operands on B200.
 
 Argument marshalling only.  Every step of the computation runs in the CUDA kernels of
 ``libmoemx.so`` behind the C ABI declared in ``include/moemx.h``; PyTorch provides device
 memory (outputs, workspaces) and the current CUDA stream.  There is no CPU fallback: if the
 library is not built, or the device is not an sm_100 GPU, the calls raise.
 
-Names follow the C ABI: ``mxfp8_quantize``, ``mxfp8_dequantize``, ``moe_permute``,
-``moe_unpermute``, ``moe_grouped_mlp_fwd``, ``moe_grouped_mlp_bwd``.
+Names follow the C ABI: ``mxfp8_quantize``, ``mxfp8_dequantize``, ``fp8_quantize``,
+``moe_permute``, ``moe_unpermute``, ``moe_grouped_mlp_fwd``, ``moe_grouped_mlp_bwd``.
 """
 from __future__ import annotations
 
@@ -24,7 +25,8 @@ MXFP8_ROWWISE, MXFP8_COLWISE_T, MXFP8_SF_MMA_LAYOUT, MXFP8_FLAG_SCALE_FLOOR, MXF
 GRAD_FORMATS = {"e4m3": 0, "e5m2": 1}
 SAVED_H = {"bf16": 0, "mxfp8": 1, "recompute": 2}
 SCALE_RULES = {"ceil": 0, "floor": 1}
-PRECISIONS = {"bf16": 0, "mxfp8": 1}
+PRECISIONS = {"bf16": 0, "mxfp8": 1, "fp8": 2}
+FP8_ROWWISE, FP8_COLWISE_T, FP8_FLAG_E5M2 = 1, 2, 16
 STATUS = {0: "ok", 1: "invalid argument", 2: "shape", 3: "unsupported", 4: "cuda", 5: "device", 6: "timeout",
           7: "workspace"}
 
@@ -35,7 +37,7 @@ EXPORTS = ["moe_ctx_create", "moe_ctx_destroy", "moe_get_status", "moe_ctx_set_d
            "moe_grouped_mlp_bwd", "moe_buffer_address", "moe_ctx_set_launch_hook", "moe_grouped_mlp_fwd_noalloc",
            "moe_ctx_set_test_stall", "moe_tensor_peak_loop", "moe_tensor_peak_flops", "moe_ctx_set_scale_rule",
            "moe_ctx_set_grad_format", "moe_ctx_set_saved_h", "moe_saved_size_ex", "moe_buffer_address_ex",
-           "moe_ctx_set_fused_forward", "moe_bwd_workspace_size_ex"]
+           "moe_ctx_set_fused_forward", "moe_bwd_workspace_size_ex", "fp8_quantize"]
 
 LAUNCH_HOOK = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
@@ -79,6 +81,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_status_string": (ctypes.c_char_p, [c_int]),
         "mxfp8_quantize": (c_int, [c_vp, c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp, c_vp, c_vp, c_vp]),
         "mxfp8_dequantize": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_int, c_vp, c_vp]),
+        "fp8_quantize": (c_int, [c_vp, c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp, c_vp, c_vp]),
         "moe_capacity_rows": (c_i64, [c_i64, c_int, c_int]),
         "moe_permute": (c_int, [c_vp, c_vp, c_vp, c_vp, c_i64, c_int, c_int, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp,
                                 c_vp, c_vp, c_vp]),
@@ -222,6 +225,28 @@ def mxfp8_dequantize(q: torch.Tensor, s: torch.Tensor, mma_layout: bool = False)
     L = load_library()
     _check("mxfp8_dequantize", L.mxfp8_dequantize(context(dev), q.data_ptr(), s.data_ptr(), rows, cols,
                                                   int(mma_layout), out.data_ptr(), _stream(dev)))
+    return out
+
+
+def fp8_quantize(x: torch.Tensor, colwise: bool = False, fmt: str = "e4m3"):
+    """x bf16 [..., rows, cols], each [rows, cols] matrix one tensor -> dict(q_row, q_colT, scale):
+    per-tensor FP8 codes (uint8; q_colT transposed, None unless ``colwise``) and the fp32 scale of
+    each tensor."""
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() >= 2
+    dev = _device_index(x)
+    rows, cols = x.shape[-2], x.shape[-1]
+    lead = tuple(x.shape[:-2])
+    batch = 1
+    for s in lead:
+        batch *= s
+    flags = FP8_ROWWISE | (FP8_COLWISE_T if colwise else 0) | (FP8_FLAG_E5M2 if fmt == "e5m2" else 0)
+    out = dict(q_row=torch.empty(lead + (rows, cols), dtype=torch.uint8, device=x.device),
+               q_colT=torch.empty(lead + (cols, rows), dtype=torch.uint8, device=x.device) if colwise else None,
+               scale=torch.empty(lead if lead else (1,), dtype=torch.float32, device=x.device))
+    L = load_library()
+    _check("fp8_quantize", L.fp8_quantize(context(dev), x.data_ptr(), batch, rows, cols, flags,
+                                          out["q_row"].data_ptr(), _ptr(out["q_colT"]), out["scale"].data_ptr(),
+                                          _stream(dev)))
     return out
 
 

@@ -198,7 +198,9 @@ struct Carve {
 struct Dims {
   int64_t T, d, f, cap, Tk;
   int E, k;
-  bool mx;
+  bool mx;      // MXFP8
+  bool fp8;     // per-tensor FP8
+  bool q8;      // 8-bit GEMM operands (either of the two)
   int saved_h;  // MOE_SAVED_H_BF16 or MOE_SAVED_H_MXFP8
 };
 
@@ -213,6 +215,7 @@ struct Saved {
   uint8_t *h_q, *h_s;                      // ... or as MXFP8: codes [cap, 2f], scales [cap, 2f/32] ...
   uint8_t *xr_q, *xr_s;                    // ... or not at all (recompute): x's gate_up operand instead,
   bf16* xr;                                //     MXFP8 row-wise codes + scales, or the BF16 gathered rows
+  uint32_t* pt_amax;                       // per-tensor FP8: [4][E] tensor maxima (fp32 bits) of x, W1, W2, a
 };
 void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
   s.split = c.take<int32_t>(D.E * 4);
@@ -226,8 +229,15 @@ void carve_saved(Carve& c, const Dims& D, Saved& s, bool full = true) {
   s.h_q = s.h_s = nullptr;
   s.xr_q = s.xr_s = nullptr;
   s.xr = nullptr;
+  s.pt_amax = nullptr;
   if (!full) return;  // inference: routing bookkeeping only
-  if (D.mx) {
+  if (D.fp8) {  // per-tensor FP8: codes only (one quantisation serves both of a tensor's GEMMs)
+    s.w1c_q = c.take<uint8_t>(D.E * D.d * 2 * D.f);
+    s.w2c_q = c.take<uint8_t>(D.E * D.f * D.d);
+    s.xT_q = c.take<uint8_t>(D.d * D.cap);
+    s.aT_q = c.take<uint8_t>(D.f * D.cap);
+    s.pt_amax = c.take<uint32_t>(4 * D.E * 4);
+  } else if (D.mx) {
     s.w1c_q = c.take<uint8_t>(D.E * D.d * 2 * D.f);
     s.w1c_s = c.take<uint8_t>(D.E * D.d * 2 * D.f / 32);
     s.w2c_q = c.take<uint8_t>(D.E * D.f * D.d);
@@ -259,11 +269,19 @@ struct FwdWs {
   uint8_t *w1_q, *w1_s, *w2_q, *w2_s, *x_q, *x_s, *a_q, *a_s;
   bf16 *x_perm, *a, *w1_copy, *w2_copy;
   bf16* y_perm;
-  int* mblk;  // fused forward: completion counters per 128-row block
+  int* mblk;          // fused forward: completion counters per 128-row block
+  uint32_t* pt_amax;  // per-tensor FP8 inference: [4][E] tensor maxima of x, W1, W2, a
 };
 void carve_fwd(Carve& c, const Dims& D, FwdWs& w) {
   std::memset(&w, 0, sizeof(w));
-  if (D.mx) {
+  if (D.fp8) {  // codes of W1 [E, 2f, d], W2 [E, d, f], x [cap, d]; a in bf16 [cap, f] and its codes
+    w.w1_q = c.take<uint8_t>(D.E * 2 * D.f * D.d);
+    w.w2_q = c.take<uint8_t>(D.E * D.d * D.f);
+    w.x_q = c.take<uint8_t>(D.cap * D.d);
+    w.a = c.take<bf16>(D.cap * D.f * 2);
+    w.a_q = c.take<uint8_t>(D.cap * D.f);
+    w.pt_amax = c.take<uint32_t>(4 * D.E * 4);
+  } else if (D.mx) {
     w.w1_q = c.take<uint8_t>(D.E * 2 * D.f * D.d);
     w.w1_s = c.take<uint8_t>(D.E * 2 * D.f * D.d / 32);
     w.w2_q = c.take<uint8_t>(D.E * D.d * D.f);
@@ -283,6 +301,7 @@ void carve_fwd(Carve& c, const Dims& D, FwdWs& w) {
 }
 
 struct BwdWs {
+  uint32_t* pt_amax;  // per-tensor FP8: [2][E] tensor maxima (fp32 bits) of dy, dh
   uint8_t *dy_q, *dy_s, *dyT_q, *dyT_s, *dh_q, *dh_s, *dhT_q, *dhT_s;
   bf16 *dy_perm, *dyT, *dh, *dhT, *w1T, *w2T;
   bf16* dx_perm;
@@ -293,7 +312,14 @@ struct BwdWs {
 };
 void carve_bwd(Carve& c, const Dims& D, BwdWs& w) {
   std::memset(&w, 0, sizeof(w));
-  if (D.mx) {
+  if (D.fp8) {  // codes of dy both ways; dh in bf16 [cap, 2f] and its codes both ways
+    w.dy_q = c.take<uint8_t>(D.cap * D.d);
+    w.dyT_q = c.take<uint8_t>(D.d * D.cap);
+    w.dh = c.take<bf16>(D.cap * 2 * D.f * 2);
+    w.dh_q = c.take<uint8_t>(D.cap * 2 * D.f);
+    w.dhT_q = c.take<uint8_t>(2 * D.f * D.cap);
+    w.pt_amax = c.take<uint32_t>(2 * D.E * 4);
+  } else if (D.mx) {
     w.dy_q = c.take<uint8_t>(D.cap * D.d);
     w.dy_s = c.take<uint8_t>(D.cap * D.d / 32);
     w.dyT_q = c.take<uint8_t>(D.d * D.cap);
@@ -346,6 +372,8 @@ Dims make_dims(int64_t T, int64_t d, int64_t f, int E, int k, moe_precision_t pr
   D.Tk = T * k;
   D.cap = capacity_rows(T, k, E);
   D.mx = prec == MOE_PREC_MXFP8;
+  D.fp8 = prec == MOE_PREC_FP8;
+  D.q8 = D.mx || D.fp8;
   return D;
 }
 
@@ -412,6 +440,68 @@ GemmArgs gemm_args(moe_ctx_t ctx) {
     g.stall_limit = ctx->stall_limit;
   }
   return g;
+}
+
+// Per-tensor FP8 codes of E expert matrices [rows, cols] (bf16 at ptrs[e], rows contiguous): row-wise
+// into q_row [E, rows, cols] and, when q_colT is set, transposed into q_colT [E, cols, rows], each
+// expert with the scale of amax[e].  One launch over all experts when they are evenly spaced, else
+// one launch per expert.
+moe_status_t quant_experts_fp8(moe_ctx_t ctx, const char* name, const void* const* ptrs, int E, int64_t rows,
+                               int64_t cols, const uint32_t* amax, uint8_t* q_row, uint8_t* q_colT, cudaStream_t st) {
+  QuantArgs a = quant_args(ctx);
+  a.src_ld = cols;
+  a.rows = rows;
+  a.cols = cols;
+  a.mx = 1;
+  a.sf_mma = 1;
+  a.scale_floor = 0;
+  a.do_row = 1;
+  a.do_col = q_colT != nullptr;
+  if (uniform_stride(ptrs, E, rows * cols * 2)) {
+    for (int e = 0; e < E; ++e) a.src_ptrs.p[e] = ptrs[e];
+    a.pt_amax = amax;
+    a.q_row = q_row;
+    a.q_colT = q_colT;
+    if (!quant_store_maps(a, E)) return MOE_ERR_CUDA;
+    MOE_LAUNCH(ctx, name, st, launch_quant(a, E, ctx->num_sms, st));
+    return MOE_OK;
+  }
+  for (int e = 0; e < E; ++e) {
+    a.src = static_cast<const bf16*>(ptrs[e]);
+    a.pt_amax = amax + e;
+    a.q_row = q_row + e * rows * cols;
+    a.q_colT = q_colT ? q_colT + e * cols * rows : nullptr;
+    if (!quant_store_maps(a, 1)) return MOE_ERR_CUDA;
+    MOE_LAUNCH(ctx, name, st, launch_quant(a, 1, ctx->num_sms, st));
+  }
+  return MOE_OK;
+}
+
+// Per-tensor FP8 codes of one [cap, cols] bf16 tensor of expert segments (a, dh): row-wise into
+// q_row and, when q_colT is set, transposed into q_colT [cols, cap], each 128-row block with the scale
+// of its expert's amax.
+moe_status_t quant_segments_fp8(moe_ctx_t ctx, const char* name, const bf16* src, int64_t cap, int64_t cols,
+                                const int32_t* poff, int E, const uint32_t* amax, int e5m2, uint8_t* q_row,
+                                uint8_t* q_colT, cudaStream_t st) {
+  QuantArgs a = quant_args(ctx);
+  a.src = src;
+  a.src_ld = cols;
+  a.rows = cap;
+  a.cols = cols;
+  a.mx = 1;
+  a.sf_mma = 1;
+  a.scale_floor = 0;
+  a.e5m2 = e5m2;
+  a.do_row = 1;
+  a.q_row = q_row;
+  a.do_col = q_colT != nullptr;
+  a.q_colT = q_colT;
+  a.pt_amax = amax;
+  a.pt_poff = poff;
+  a.pt_E = E;
+  if (!quant_store_maps(a, 1)) return MOE_ERR_CUDA;
+  MOE_LAUNCH(ctx, name, st, launch_quant(a, 1, ctx->num_sms, st));
+  return MOE_OK;
 }
 
 }  // namespace
@@ -583,6 +673,47 @@ moe_status_t mxfp8_dequantize(moe_ctx_t ctx, const uint8_t* q, const uint8_t* s,
   return MOE_OK;
 }
 
+moe_status_t fp8_quantize(moe_ctx_t ctx, const void* x, int64_t batch, int64_t rows, int64_t cols, int flags,
+                          uint8_t* q_row, uint8_t* q_colT, float* scale, void* stream) {
+  if (!ctx || !x || !scale || batch <= 0 || rows <= 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+  const bool col = flags & FP8_COLWISE_T;
+  if ((flags & ~(FP8_ROWWISE | FP8_COLWISE_T | FP8_FLAG_E5M2)) || !(flags & FP8_ROWWISE) || !q_row ||
+      (col && !q_colT))
+    return MOE_ERR_INVALID_ARG;
+  if (rows % 128 || cols % 128) return MOE_ERR_SHAPE;
+  if (batch > MOE_MAX_EXPERTS || rows * cols >= (int64_t(1) << 40)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(q_row) || (col && !aligned16(q_colT))) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(ctx->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int e5m2 = (flags & FP8_FLAG_E5M2) ? 1 : 0;
+  uint32_t* amax = reinterpret_cast<uint32_t*>(scale);  // the maxima first; the scales replace them at the end
+  MOE_CUDA(cudaMemsetAsync(amax, 0, static_cast<size_t>(batch) * sizeof(uint32_t), st));
+  PtrArray none;
+  std::memset(&none, 0, sizeof(none));
+  MOE_LAUNCH(ctx, "fp8_amax", st,
+             launch_amax_batched(none, static_cast<const bf16*>(x), rows * cols, static_cast<int>(batch), rows, cols,
+                                 cols, amax, ctx->num_sms, st));
+  QuantArgs a = quant_args(ctx);
+  a.src = static_cast<const bf16*>(x);
+  a.src_batch_stride = rows * cols;
+  a.src_ld = cols;
+  a.rows = rows;
+  a.cols = cols;
+  a.mx = 1;
+  a.sf_mma = 1;
+  a.scale_floor = 0;
+  a.e5m2 = e5m2;
+  a.do_row = 1;
+  a.q_row = q_row;
+  a.do_col = col;
+  a.q_colT = q_colT;
+  a.pt_amax = amax;
+  if (!quant_store_maps(a, static_cast<int>(batch))) return MOE_ERR_CUDA;
+  MOE_LAUNCH(ctx, "fp8_quantize", st, launch_quant(a, static_cast<int>(batch), ctx->num_sms, st));
+  MOE_LAUNCH(ctx, "fp8_scales", st, launch_fp8_scales(amax, static_cast<int>(batch), e5m2, st));
+  return MOE_OK;
+}
+
 moe_status_t moe_permute(moe_ctx_t ctx, const void* x, const int32_t* topk_idx, const float* topk_prob, int64_t T,
                          int k, int E, int64_t d, const int32_t* split_sizes_in, int32_t* split_sizes,
                          int32_t* poffsets, int32_t* sorted_to_src, int32_t* src_to_sorted, float* prob_perm,
@@ -633,6 +764,7 @@ size_t moe_saved_size_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_prec
   if (saved_h != MOE_SAVED_H_BF16 && saved_h != MOE_SAVED_H_RECOMPUTE &&
       (saved_h != MOE_SAVED_H_MXFP8 || prec != MOE_PREC_MXFP8))
     return 0;
+  if (prec == MOE_PREC_FP8 && saved_h != MOE_SAVED_H_BF16) return 0;
   Dims D = make_dims(T, d, f, E, k, prec, saved_h);
   Carve c(nullptr);
   Saved s;
@@ -660,6 +792,7 @@ size_t moe_fwd_workspace_size(int64_t T, int k, int E, int64_t d, int64_t f, moe
 size_t moe_bwd_workspace_size_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int saved_h) {
   if (check_dims(T, d, f, E, k) != MOE_OK) return 0;
   if (saved_h < MOE_SAVED_H_BF16 || saved_h > MOE_SAVED_H_RECOMPUTE) return 0;
+  if (prec == MOE_PREC_FP8 && saved_h != MOE_SAVED_H_BF16) return 0;
   Dims D = make_dims(T, d, f, E, k, prec, saved_h);
   Carve c(nullptr);
   BwdWs w;
@@ -677,7 +810,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
                                  moe_precision_t prec, int training, void* y, void* saved, size_t saved_bytes,
                                  void* workspace, size_t workspace_bytes, void* stream) {
   if (!ctx || !x || !topk_idx || !topk_prob || !w_gate_up || !w_down || !y || !workspace) return MOE_ERR_INVALID_ARG;
-  if (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8 && prec != MOE_PREC_FP8) return MOE_ERR_INVALID_ARG;
   const moe_status_t dc = check_dims(T, d, f, E, k);
   if (dc != MOE_OK) return dc;
   if (training && !saved) return MOE_ERR_INVALID_ARG;
@@ -686,6 +819,7 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
   if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   const int saved_h = training ? ctx->saved_h : MOE_SAVED_H_BF16;
   if (saved_h == MOE_SAVED_H_MXFP8 && prec != MOE_PREC_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (prec == MOE_PREC_FP8 && saved_h != MOE_SAVED_H_BF16) return MOE_ERR_UNSUPPORTED;
   if (workspace_bytes < moe_fwd_workspace_size(T, k, E, d, f, prec, training)) return MOE_ERR_WORKSPACE;
   if (training && saved_bytes < moe_saved_size_ex(T, k, E, d, f, prec, saved_h)) return MOE_ERR_WORKSPACE;
 
@@ -708,6 +842,14 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
   uint8_t* x_s = s.xr_s ? s.xr_s : w.x_s;
   bf16* x_perm = s.xr ? s.xr : w.x_perm;
 
+  // per-tensor FP8: the maxima of x, W1, W2 and a (per expert), kept for the backward when training
+  uint32_t* amax = D.fp8 ? (training ? s.pt_amax : w.pt_amax) : nullptr;
+  uint32_t* amax_x = amax;
+  uint32_t* amax_w1 = amax ? amax + E : nullptr;
+  uint32_t* amax_w2 = amax ? amax + 2 * E : nullptr;
+  uint32_t* amax_a = amax ? amax + 3 * E : nullptr;
+  if (D.fp8) MOE_CUDA(cudaMemsetAsync(amax, 0, 4 * static_cast<size_t>(E) * sizeof(uint32_t), st));
+
   // 1. routing: counts, padded offsets, stable permutation, per-row probabilities
   MOE_LAUNCH(ctx, "route", st, launch_route(topk_idx, topk_prob, static_cast<int>(D.Tk), E, static_cast<int>(D.cap), split_sizes, s.split,
                         s.poff, s.s2src, s.src2s, s.pperm, ctx->d_status, st));
@@ -716,7 +858,48 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
   const void* w1_base;
   const void* w2_base;
   int64_t w1_stride, w2_stride;  // bytes between experts
-  if (D.mx) {
+  if (D.fp8) {
+    // per-tensor FP8 with current scaling: every expert's W1, W2 and rows of x get one scale from their
+    // own maximum, so the maxima come first; one quantisation serves both GEMMs of each tensor
+    PtrArray p1, p2;
+    for (int e = 0; e < E; ++e) {
+      p1.p[e] = w_gate_up[e];
+      p2.p[e] = w_down[e];
+    }
+    MOE_LAUNCH(ctx, "amax_w_gate_up", st, launch_amax_batched(p1, nullptr, 0, E, 2 * f, d, d, amax_w1, ctx->num_sms, st));
+    MOE_LAUNCH(ctx, "amax_w_down", st, launch_amax_batched(p2, nullptr, 0, E, d, f, f, amax_w2, ctx->num_sms, st));
+    MOE_LAUNCH(ctx, "amax_x", st,
+               launch_amax_routed(static_cast<const bf16*>(x), d, d, s.s2src, s.poff, D.cap, k, E, amax_x, ctx->num_sms, st));
+    moe_status_t r = quant_experts_fp8(ctx, "quantize_w_gate_up", w_gate_up, E, 2 * f, d, amax_w1, w.w1_q,
+                                       training ? s.w1c_q : nullptr, st);
+    if (r != MOE_OK) return r;
+    r = quant_experts_fp8(ctx, "quantize_w_down", w_down, E, d, f, amax_w2, w.w2_q, training ? s.w2c_q : nullptr, st);
+    if (r != MOE_OK) return r;
+    w1_base = w.w1_q;
+    w1_stride = 2 * f * d;
+    w2_base = w.w2_q;
+    w2_stride = d * f;
+    QuantArgs xa = quant_args(ctx);
+    xa.src = static_cast<const bf16*>(x);
+    xa.src_ld = d;
+    xa.sorted_to_src = s.s2src;
+    xa.src_rows = T;
+    xa.k = k;
+    xa.rows = D.cap;
+    xa.cols = d;
+    xa.mx = 1;
+    xa.sf_mma = 1;
+    xa.scale_floor = 0;
+    xa.do_row = 1;
+    xa.q_row = w.x_q;
+    xa.do_col = training;
+    xa.q_colT = s.xT_q;
+    xa.pt_amax = amax_x;
+    xa.pt_poff = s.poff;
+    xa.pt_E = E;
+    if (!quant_store_maps(xa, 1)) return MOE_ERR_CUDA;
+    MOE_LAUNCH(ctx, "permute_quantize_x", st, launch_quant(xa, 1, ctx->num_sms, st));
+  } else if (D.mx) {
     // 16-bit masters -> MXFP8 every step: row-wise (K = d / f of the forward GEMMs) and, for the
     // backward, down the columns (K = 2f / d of the dgrad GEMMs), from one read of each weight.
     QuantArgs a = quant_args(ctx);
@@ -822,9 +1005,9 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     GemmArgs g = gemm_args(ctx);
     // MXFP8: the quantised copy is gate/up interleaved, two 128-row boxes per tile; BF16 reads the
     // unpermuted weights as a 128-row gate box plus the matching 128-row up box.
-    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(x_q) : x_perm, D.mx, d, D.cap,
-                           d * (D.mx ? 1 : 2)) &&
-                    map_3d(&g.tmap_b, w1_base, D.mx, d, 2 * f, E, d * (D.mx ? 1 : 2), w1_stride,
+    const bool ok = map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(x_q) : x_perm, D.q8, d, D.cap,
+                           d * (D.q8 ? 1 : 2)) &&
+                    map_3d(&g.tmap_b, w1_base, D.q8, d, 2 * f, E, d * (D.q8 ? 1 : 2), w1_stride,
                            D.mx ? gemm_tile_n(EPI_SWIGLU) : gemm_tile_n(EPI_SWIGLU) / 2);
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
@@ -832,6 +1015,9 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     g.K = static_cast<int>(d);
     g.n_tiles = static_cast<int>(f / 128);
     g.gate_up_half = D.mx ? 0 : static_cast<int>(f);
+    g.fp8 = D.fp8;
+    g.pt_amax_a = amax_x;
+    g.pt_amax_b = amax_w1;
     g.poffsets = s.poff;
     g.sfa = x_s;
     g.sfa_kb4 = d / 128;
@@ -853,19 +1039,25 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       ep.q_colT = training ? s.aT_q : nullptr;
       ep.s_colT = training ? s.aT_s : nullptr;
     } else {
+      // BF16: a in bf16 both ways; per-tensor FP8: a in bf16 rows and its per-expert maximum, then
+      // quantised once its maximum is complete
       ep.o_row = w.a;
-      ep.o_colT = training ? s.aT : nullptr;
+      ep.o_colT = (training && !D.fp8) ? s.aT : nullptr;
+      ep.amax_out = D.fp8 ? amax_a : nullptr;
     }
     // 4. down GEMM: its own launch, or (fused forward) the tiles that follow in the same launch
     GemmArgs g2 = gemm_args(ctx);
-    const bool ok2 = map_2d(&g2.tmap_a, D.mx ? static_cast<const void*>(w.a_q) : w.a, D.mx, f, D.cap,
-                            f * (D.mx ? 1 : 2)) &&
-                     map_3d(&g2.tmap_b, w2_base, D.mx, f, d, E, f * (D.mx ? 1 : 2), w2_stride, gemm_tile_n(EPI_STORE));
+    const bool ok2 = map_2d(&g2.tmap_a, D.q8 ? static_cast<const void*>(w.a_q) : w.a, D.q8, f, D.cap,
+                            f * (D.q8 ? 1 : 2)) &&
+                     map_3d(&g2.tmap_b, w2_base, D.q8, f, d, E, f * (D.q8 ? 1 : 2), w2_stride, gemm_tile_n(EPI_STORE));
     if (!ok2) return MOE_ERR_CUDA;
     g2.kgrouped = 0;
     g2.E = E;
     g2.K = static_cast<int>(f);
     g2.n_tiles = static_cast<int>(d / 256);
+    g2.fp8 = D.fp8;
+    g2.pt_amax_a = amax_a;
+    g2.pt_amax_b = amax_w2;
     g2.poffsets = s.poff;
     g2.sfa = w.a_s;
     g2.sfa_kb4 = f / 128;
@@ -875,8 +1067,9 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     if (D.mx && !sf_maps(g2, D.cap, E * d, gemm_tile_n(EPI_STORE))) return MOE_ERR_CUDA;
     g2.epi.out = w.y_perm;
     g2.epi.ldo = d;
-    if (ctx->fused_fwd) {
+    if (ctx->fused_fwd && !D.fp8) {
       // one persistent launch: gate_up tiles, then down tiles that wait for their 128-row blocks of a
+      // (per-tensor FP8 cannot: a is quantised only once all of its expert's tiles are done)
       g.tmap_a2 = g2.tmap_a;
       g.tmap_b2 = g2.tmap_b;
       g.tmap_sfa2 = g2.tmap_sfa;
@@ -891,6 +1084,11 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
       MOE_LAUNCH(ctx, "gemm_fused_forward", st, launch_grouped_gemm(g, D.mx, EPI_FUSED_FWD, ctx->num_sms, st));
     } else {
       MOE_LAUNCH(ctx, "gemm_gate_up_swiglu", st, launch_grouped_gemm(g, D.mx, EPI_SWIGLU, ctx->num_sms, st));
+      if (D.fp8) {
+        const moe_status_t r = quant_segments_fp8(ctx, "quantize_a", w.a, D.cap, f, s.poff, E, amax_a, 0, w.a_q,
+                                                  training ? s.aT_q : nullptr, st);
+        if (r != MOE_OK) return r;
+      }
       MOE_LAUNCH(ctx, "gemm_down", st, launch_grouped_gemm(g2, D.mx, EPI_STORE, ctx->num_sms, st));
     }
   }
@@ -906,7 +1104,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
                                  void* stream) {
   if (!ctx || !dy || !saved || !w_gate_up || !w_down || !dx || !dw_gate_up || !dw_down || !d_topk_prob || !workspace)
     return MOE_ERR_INVALID_ARG;
-  if (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8 && prec != MOE_PREC_FP8) return MOE_ERR_INVALID_ARG;
   const moe_status_t dc = check_dims(T, d, f, E, k);
   if (dc != MOE_OK) return dc;
   for (int e = 0; e < E; ++e)
@@ -916,6 +1114,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   if (!aligned16(dy) || !aligned16(dx)) return MOE_ERR_INVALID_ARG;
   const int saved_h = ctx->saved_h;
   if (saved_h == MOE_SAVED_H_MXFP8 && prec != MOE_PREC_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (prec == MOE_PREC_FP8 && saved_h != MOE_SAVED_H_BF16) return MOE_ERR_UNSUPPORTED;
   if (saved_bytes < moe_saved_size_ex(T, k, E, d, f, prec, saved_h)) return MOE_ERR_WORKSPACE;
   if (workspace_bytes < moe_bwd_workspace_size_ex(T, k, E, d, f, prec, saved_h)) return MOE_ERR_WORKSPACE;
 
@@ -928,6 +1127,18 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   BwdWs w;
   Carve cw(reinterpret_cast<void*>(round_up(reinterpret_cast<uintptr_t>(workspace), 1024)));
   carve_bwd(cw, D, w);
+  // per-tensor FP8: the forward's maxima of x, W1, W2, a, and this pass's of dy and dh
+  const uint32_t* amax_x = s.pt_amax;
+  const uint32_t* amax_w1 = s.pt_amax ? s.pt_amax + E : nullptr;
+  const uint32_t* amax_w2 = s.pt_amax ? s.pt_amax + 2 * E : nullptr;
+  const uint32_t* amax_a = s.pt_amax ? s.pt_amax + 3 * E : nullptr;
+  uint32_t* amax_dy = w.pt_amax;
+  uint32_t* amax_dh = w.pt_amax ? w.pt_amax + E : nullptr;
+  if (D.fp8) {
+    MOE_CUDA(cudaMemsetAsync(w.pt_amax, 0, 2 * static_cast<size_t>(E) * sizeof(uint32_t), st));
+    MOE_LAUNCH(ctx, "amax_dy", st,
+               launch_amax_routed(static_cast<const bf16*>(dy), d, d, s.s2src, s.poff, D.cap, k, E, amax_dy, ctx->num_sms, st));
+  }
 
   // 0. recompute mode: h again, from x's saved gate_up operand and W1 (quantised again for MXFP8),
   //    through the gate_up GEMM with an epilogue that only writes h
@@ -1007,7 +1218,17 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     a.cols = d;
     a.do_row = 1;
     a.do_col = 1;
-    if (D.mx) {
+    if (D.fp8) {  // per-tensor FP8 with each expert's maximum
+      a.mx = 1;
+      a.sf_mma = 1;
+      a.scale_floor = 0;
+      a.e5m2 = ctx->grad_e5m2;
+      a.q_row = w.dy_q;
+      a.q_colT = w.dyT_q;
+      a.pt_amax = amax_dy;
+      a.pt_poff = s.poff;
+      a.pt_E = E;
+    } else if (D.mx) {
       a.mx = 1;
       a.sf_mma = 1;
       a.e5m2 = ctx->grad_e5m2;  // dy is a gradient operand
@@ -1024,7 +1245,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   }
   const void* w1c;  // B of dgrad of gate_up: [E, d, 2f]
   const void* w2c;  // B of dgrad of down:    [E, f, d]
-  if (D.mx) {
+  if (D.q8) {
     w1c = s.w1c_q;
     w2c = s.w2c_q;
   } else {
@@ -1048,18 +1269,21 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     w1c = w.w1T;
     w2c = w.w2T;
   }
-  const int es = D.mx ? 1 : 2;
+  const int es = D.q8 ? 1 : 2;
   // 2. dgrad of down + ScaledSwiGLU backward: dh = [dg, du] requantised both ways, dp partials
   {
     GemmArgs g = gemm_args(ctx);
-    const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dy_q) : w.dy_perm, D.mx, d, D.cap, d * es) &&
-                    map_3d(&g.tmap_b, w2c, D.mx, d, f, E, d * es, f * d * es, gemm_tile_n(EPI_DSWIGLU)) &&
+    const bool ok = map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(w.dy_q) : w.dy_perm, D.q8, d, D.cap, d * es) &&
+                    map_3d(&g.tmap_b, w2c, D.q8, d, f, E, d * es, f * d * es, gemm_tile_n(EPI_DSWIGLU)) &&
                     (s.h_q || map_2d(&g.tmap_h, h_src, false, 2 * f, D.cap, 2 * f * 2));  // bf16 boxes, 128 x 64
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
     g.K = static_cast<int>(d);
     g.n_tiles = static_cast<int>(f / gemm_tile_n(EPI_DSWIGLU));
+    g.fp8 = D.fp8;
+    g.pt_amax_a = amax_dy;
+    g.pt_amax_b = amax_w2;
     g.poffsets = s.poff;
     g.sfa = w.dy_s;
     g.sfa_kb4 = d / 128;
@@ -1084,23 +1308,34 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
       ep.q_colT = w.dhT_q;
       ep.s_colT = w.dhT_s;
     } else {
+      // BF16: dh in bf16 both ways; per-tensor FP8: dh in bf16 rows and its per-expert maximum, then
+      // quantised once its maximum is complete
       ep.o_row = w.dh;
-      ep.o_colT = w.dhT;
+      ep.o_colT = D.fp8 ? nullptr : w.dhT;
+      ep.amax_out = amax_dh;
     }
     MOE_LAUNCH(ctx, "gemm_dgrad_down_dswiglu", st, launch_grouped_gemm(g, D.mx, EPI_DSWIGLU, ctx->num_sms, st));
+    if (D.fp8) {
+      const moe_status_t r = quant_segments_fp8(ctx, "quantize_dh", w.dh, D.cap, 2 * f, s.poff, E, amax_dh,
+                                                ctx->grad_e5m2, w.dh_q, w.dhT_q, st);
+      if (r != MOE_OK) return r;
+    }
   }
   // 3. wgrad of down: dW2_e [d, f] = dy_e^T a_e (K = the expert's tokens)
   {
     GemmArgs g = gemm_args(ctx);
     const bool ok =
-        map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dyT_q) : w.dyT, D.mx, D.cap, d, D.cap * es) &&
-        map_2d(&g.tmap_b, D.mx ? static_cast<const void*>(s.aT_q) : s.aT, D.mx, D.cap, f, D.cap * es,
+        map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(w.dyT_q) : w.dyT, D.q8, D.cap, d, D.cap * es) &&
+        map_2d(&g.tmap_b, D.q8 ? static_cast<const void*>(s.aT_q) : s.aT, D.q8, D.cap, f, D.cap * es,
                gemm_tile_n(EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 1;
     g.E = E;
     g.m_tiles = static_cast<int>(d / 128);
     g.n_tiles = static_cast<int>(f / 256);
+    g.fp8 = D.fp8;
+    g.pt_amax_a = amax_dy;
+    g.pt_amax_b = amax_a;
     g.poffsets = s.poff;
     g.sfa = w.dyT_s;
     g.sfa_kb4 = D.cap / 128;
@@ -1116,13 +1351,16 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   {
     GemmArgs g = gemm_args(ctx);
     const bool ok =
-        map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dh_q) : w.dh, D.mx, 2 * f, D.cap, 2 * f * es) &&
-        map_3d(&g.tmap_b, w1c, D.mx, 2 * f, d, E, 2 * f * es, 2 * f * d * es, gemm_tile_n(EPI_STORE));
+        map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(w.dh_q) : w.dh, D.q8, 2 * f, D.cap, 2 * f * es) &&
+        map_3d(&g.tmap_b, w1c, D.q8, 2 * f, d, E, 2 * f * es, 2 * f * d * es, gemm_tile_n(EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
     g.K = static_cast<int>(2 * f);
     g.n_tiles = static_cast<int>(d / 256);
+    g.fp8 = D.fp8;
+    g.pt_amax_a = amax_dh;
+    g.pt_amax_b = amax_w1;
     g.poffsets = s.poff;
     g.sfa = w.dh_s;
     g.sfa_kb4 = 2 * f / 128;
@@ -1139,14 +1377,17 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
   {
     GemmArgs g = gemm_args(ctx);
     const bool ok =
-        map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(w.dhT_q) : w.dhT, D.mx, D.cap, 2 * f, D.cap * es) &&
-        map_2d(&g.tmap_b, D.mx ? static_cast<const void*>(s.xT_q) : s.xT, D.mx, D.cap, d, D.cap * es,
+        map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(w.dhT_q) : w.dhT, D.q8, D.cap, 2 * f, D.cap * es) &&
+        map_2d(&g.tmap_b, D.q8 ? static_cast<const void*>(s.xT_q) : s.xT, D.q8, D.cap, d, D.cap * es,
                gemm_tile_n(EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 1;
     g.E = E;
     g.m_tiles = static_cast<int>(2 * f / 128);
     g.n_tiles = static_cast<int>(d / 256);
+    g.fp8 = D.fp8;
+    g.pt_amax_a = amax_dh;
+    g.pt_amax_b = amax_x;
     g.poffsets = s.poff;
     g.sfa = w.dhT_s;
     g.sfa_kb4 = D.cap / 128;
@@ -1168,18 +1409,20 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
 
 moe_status_t moe_tensor_peak_loop(moe_ctx_t ctx, moe_precision_t prec, int64_t iters, int scale_refresh,
                                   void* stream) {
-  if (!ctx || iters <= 0 || iters > 1000000 || (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8))
+  if (!ctx || iters <= 0 || iters > 1000000 ||
+      (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8 && prec != MOE_PREC_FP8))
     return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(ctx->device);
   MOE_LAUNCH(ctx, "tensor_peak_loop", stream,
-             launch_tensor_peak(prec == MOE_PREC_MXFP8, iters, scale_refresh ? 1 : 0, ctx->num_sms, ctx->d_status,
+             launch_tensor_peak(static_cast<int>(prec), iters, scale_refresh ? 1 : 0, ctx->num_sms, ctx->d_status,
                                 static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 
 double moe_tensor_peak_flops(moe_ctx_t ctx, moe_precision_t prec, int64_t iters) {
   if (!ctx || iters <= 0) return 0.0;
-  return tensor_peak_flops(prec == MOE_PREC_MXFP8, ctx->num_sms, iters);
+  if (prec != MOE_PREC_BF16 && prec != MOE_PREC_MXFP8 && prec != MOE_PREC_FP8) return 0.0;
+  return tensor_peak_flops(static_cast<int>(prec), ctx->num_sms, iters);
 }
 
 void* moe_buffer_address_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_precision_t prec, int training,
@@ -1203,7 +1446,7 @@ void* moe_buffer_address_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_p
                          {"w1c_s", s.w1c_s}, {"w2c_q", s.w2c_q}, {"w2c_s", s.w2c_s}, {"xT_q", s.xT_q},
                          {"xT_s", s.xT_s}, {"aT_q", s.aT_q}, {"aT_s", s.aT_s}, {"xT", s.xT}, {"aT", s.aT},
                          {"h", s.h},       {"h_q", s.h_q},     {"h_s", s.h_s},   {"xr_q", s.xr_q},
-                         {"xr_s", s.xr_s}, {"xr", s.xr}};
+                         {"xr_s", s.xr_s}, {"xr", s.xr},   {"pt_amax", s.pt_amax}};
     for (const Named& e : tab)
       if (!std::strcmp(e.n, name) && e.p) return e.p;
     if (which == 0) return nullptr;
@@ -1214,7 +1457,7 @@ void* moe_buffer_address_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_p
     carve_fwd(c, D, w);
     const Named tab[] = {{"w1_q", w.w1_q}, {"w1_s", w.w1_s}, {"w2_q", w.w2_q}, {"w2_s", w.w2_s},
                          {"x_q", w.x_q},   {"x_s", w.x_s},   {"a_q", w.a_q},   {"a_s", w.a_s},
-                         {"x_perm", w.x_perm}, {"a", w.a}, {"y_perm", w.y_perm}};
+                         {"x_perm", w.x_perm}, {"a", w.a}, {"y_perm", w.y_perm}, {"pt_amax", w.pt_amax}};
     for (const Named& e : tab)
       if (!std::strcmp(e.n, name) && e.p) return e.p;
     return nullptr;
@@ -1226,7 +1469,8 @@ void* moe_buffer_address_ex(int64_t T, int k, int E, int64_t d, int64_t f, moe_p
                          {"dh_q", w.dh_q},   {"dh_s", w.dh_s},     {"dhT_q", w.dhT_q}, {"dhT_s", w.dhT_s},
                          {"dy_perm", w.dy_perm}, {"dyT", w.dyT},   {"dh", w.dh},       {"dhT", w.dhT},
                          {"w1T", w.w1T},     {"w2T", w.w2T},       {"dx_perm", w.dx_perm},
-                         {"dp_part", w.dp_part}, {"hr", w.hr},     {"w1r_q", w.w1r_q}, {"w1r_s", w.w1r_s}};
+                         {"dp_part", w.dp_part}, {"hr", w.hr},     {"w1r_q", w.w1r_q}, {"w1r_s", w.w1r_s},
+                         {"pt_amax", w.pt_amax}};
     for (const Named& e : tab)
       if (!std::strcmp(e.n, name) && e.p) return e.p;
   }

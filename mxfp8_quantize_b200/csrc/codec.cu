@@ -355,34 +355,49 @@ quant_tile_kernel(const __grid_constant__ QuantArgs a) {
 }
 
 // ------------------------------------------------------------------------------------------
-// The same MXFP8 quantisation (tensor-core scale layout, row-wise and optionally column-wise) for a uniformly
-// strided [batch, rows, cols] source whose rows and cols are multiples of 128, as a persistent
-// kernel: QW_CTAS_PER_SM CTAs per SM walk the 128 x 128 tiles (column tiles fastest); each source
-// tile arrives by a TMA tensor load into a QW_NIN-deep ring issued QW_NIN tiles ahead, and the
-// code tiles leave through TMA tensor stores, so the reads, math and writes of consecutive tiles
-// (and of the SM's other CTA) overlap.  Same arithmetic, bit for bit, as quant_tile_kernel.
+// The same MXFP8 quantisation (tensor-core scale layout, row-wise and optionally column-wise) for a
+// uniformly strided [batch, rows, cols] source whose rows and cols are multiples of 128, as a
+// persistent kernel: the CTAs walk the 128 x 128 tiles (column tiles fastest); each source tile
+// arrives by a TMA tensor load (or, for a gather, by tile::gather4 row fetches) into a QW_NIN-deep
+// ring issued QW_NIN tiles ahead.  Two ways out for the codes, chosen per use by measurement:
+//  * staged (weights, bf16 transposes): code tiles in 128B-swizzled shared memory leave through TMA
+//    tensor stores as whole 128-byte lines; two CTAs per SM;
+//  * direct (the x / dy gathers): codes leave straight from registers in whole sectors (8-byte row
+//    chunks, 16 threads per 128-byte row; 32-byte column runs), no output staging, three CTAs per
+//    SM.
+// Same arithmetic, bit for bit, as quant_tile_kernel.
 // ------------------------------------------------------------------------------------------
 namespace {
 constexpr int QW_NIN = 2;                           // source tiles in flight per CTA
-constexpr int QW_NOUT = 1;                          // code-tile buffers per CTA
-constexpr int QW_CTAS_PER_SM = 2;
 constexpr int QW_IN_BYTES = QT_ROWS * QT_COLS * 2;  // one bf16 source tile, rows of 256 bytes
-constexpr int QW_OUT_BYTES = 2 * QT_ROWS * QT_COLS;  // row-wise + column-wise code tiles
-constexpr int QW_SMEM = QW_NIN * QW_IN_BYTES + QW_NOUT * (QW_OUT_BYTES + 1024) + 1024;
+constexpr int QW_OUT_BYTES = 2 * QT_ROWS * QT_COLS;  // staged: row-wise + column-wise code tiles
 static_assert(QW_OUT_BYTES >= QT_ROWS * QT_COLS * 2, "an output buffer also holds one transposed bf16 tile");
+template <bool DIRECT>
+struct QwShape {
+  static constexpr int CTAS_PER_SM = DIRECT ? 3 : 2;
+  static constexpr int OUT_BYTES = DIRECT ? 0 : QW_OUT_BYTES;
+  static constexpr int SMEM = QW_NIN * QW_IN_BYTES + OUT_BYTES + 1024 + 1024;  // + 2 scale tiles, + alignment
+};
 }  // namespace
 
-__global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const __grid_constant__ QuantArgs a, int tiles) {
+template <bool DIRECT>
+__global__ void __launch_bounds__(256, QwShape<DIRECT>::CTAS_PER_SM)
+    quant_w_tma_kernel(const __grid_constant__ QuantArgs a, int tiles) {
   extern __shared__ uint8_t qw_raw[];
   uint8_t* sm = qw_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(qw_raw)) & 1023u)) & 1023u);
-  uint8_t* in_base = sm;                                   // QW_NIN source tiles
-  uint8_t* out_base = sm + QW_NIN * QW_IN_BYTES;           // QW_NOUT x [row codes 16 KB | column codes 16 KB]
-  uint8_t* atom_base = out_base + QW_NOUT * QW_OUT_BYTES;  // QW_NOUT x [row scale tile | column scale tile]
+  uint8_t* in_base = sm;                                        // QW_NIN source tiles
+  uint8_t* qrow = sm + QW_NIN * QW_IN_BYTES;                    // staged: row-wise code tile (16 KB)
+  uint8_t* qcol = qrow + QT_ROWS * QT_COLS;                     //         column-wise code tile (16 KB)
+  uint8_t* satom_row = qrow + QwShape<DIRECT>::OUT_BYTES;       // the tile's row-wise scale tile (512 B)
+  uint8_t* satom_col = satom_row + 512;                         // and its column-wise one
   __shared__ uint64_t full[QW_NIN];
   __shared__ int stop;
+  __shared__ float pt_sc[MOE_MAX_EXPERTS];       // per-tensor FP8: the scale of each tensor
+  __shared__ int32_t pt_off[MOE_MAX_EXPERTS + 1];  // ... and the expert segments' first rows
   const int tid = threadIdx.x;
   const int64_t R = a.rows, C = a.cols, KBr = C / 32, KBc = R / 32;
   const int CT = static_cast<int>(C / QT_COLS), RT = static_cast<int>(R / QT_ROWS);
+  const bool pt = a.pt_amax != nullptr;
   auto coords = [&](int t, int& b, int& rt, int& ct) {
     b = t / (RT * CT);
     const int rem = t - b * RT * CT;
@@ -422,6 +437,12 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
                      &full[slot]);
   };
   const bool issuer = a.tma_gather ? tid < 32 : tid == 0;
+  if (pt) {
+    const int n = a.pt_poff ? a.pt_E : tiles / (RT * CT);
+    for (int i = tid; i < n; i += blockDim.x) pt_sc[i] = fp8_tensor_scale(a.pt_amax[i], a.e5m2);
+    if (a.pt_poff)
+      for (int i = tid; i <= a.pt_E; i += blockDim.x) pt_off[i] = a.pt_poff[i];
+  }
   if (tid == 0) {
     for (int i = 0; i < QW_NIN; ++i) ptx::mbar_init(&full[i], 1);
     ptx::fence_mbar_init();
@@ -445,12 +466,14 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
     const int tn = blockIdx.x + QW_NIN * gridDim.x;
     if (a.tma_gather && tn < tiles) gather_rows(tn, y_next);
   }
+  // direct: 32-byte aligned column-wise output leaves in single 256-bit stores
+  const bool col32 = ((reinterpret_cast<uintptr_t>(a.mx ? static_cast<void*>(a.q_colT) : static_cast<void*>(a.o_colT)) &
+                       31u) == 0);
   int it = 0;
   for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
     const int slot = it % QW_NIN;
-    const int ob = it % QW_NOUT;
     if (tid == 0) {
-      // this tile's source has landed; the stores that last read output buffer ``ob`` are done
+      // this tile's source has landed (staged: and the stores that read the code tiles are done)
       volatile int* flag = &stop;  // raised by an expired wait
       bool ok = true;
       if (a.stall_flag && it == 0)  // test hook: a wait that can only expire, first source tiles in flight
@@ -461,7 +484,7 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         stop = 1;
         if (a.status) atomicOr(a.status, kStatusTimeout);
       }
-      asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(QW_NOUT - 1) : "memory");
+      if (!DIRECT) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     }
     __syncthreads();
     if (stop) break;
@@ -469,15 +492,23 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
     coords(t, b, rt, ct);
     const int64_t row0 = static_cast<int64_t>(rt) * QT_ROWS, col0 = static_cast<int64_t>(ct) * QT_COLS;
     const uint8_t* in = in_base + slot * QW_IN_BYTES;
-    uint8_t* qrow = out_base + ob * QW_OUT_BYTES;
-    uint8_t* qcol = qrow + QT_ROWS * QT_COLS;
-    uint8_t* satom_row = atom_base + ob * 1024;
-    uint8_t* satom_col = satom_row + 512;
+    float pts = 0.f;  // per-tensor FP8: the tile's tensor scale
+    if (pt) {
+      int e = b;
+      if (a.pt_poff) {  // the expert segment holding row0 (largest e with pt_off[e] <= row0)
+        int lo = 0, hi = a.pt_E;
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (pt_off[mid] <= row0) lo = mid; else hi = mid;
+        }
+        e = lo;
+      }
+      pts = pt_sc[e];
+    }
 
     if (!a.mx) {
       // bf16 transpose only: thread -> columns (2p, 2p+1) = rows of the transposed tile, source rows
-      // 32 rb .. +31; the transposed tile (32 KB: the whole output buffer, there are no row-wise
-      // codes) is two 64-column halves of 128-byte rows, 128B-swizzled
+      // 32 rb .. +31
       const int p = tid & 63, rb = tid >> 6;
       const uint32_t* words = reinterpret_cast<const uint32_t*>(in);  // 64 bf16 pairs per row
       uint32_t c0[16], c1[16];
@@ -487,20 +518,43 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         c0[i] = __byte_perm(w0, w1, 0x5410);  // low halves: column 2p
         c1[i] = __byte_perm(w0, w1, 0x7632);  // high halves: column 2p+1
       }
-      uint8_t* half = qrow + (rb >> 1) * (QT_ROWS * 128);
-      const int r0 = 2 * p, r1 = 2 * p + 1;
+      if (!DIRECT) {
+        // the transposed tile (32 KB: the whole output buffer) as two 64-column halves of 128-byte
+        // rows, 128B-swizzled
+        uint8_t* half = qrow + (rb >> 1) * (QT_ROWS * 128);
+        const int r0 = 2 * p, r1 = 2 * p + 1;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int chunk = (rb & 1) * 4 + j;
-        *reinterpret_cast<uint4*>(half + r0 * 128 + ((chunk ^ (r0 & 7)) << 4)) =
-            make_uint4(c0[4 * j], c0[4 * j + 1], c0[4 * j + 2], c0[4 * j + 3]);
-        *reinterpret_cast<uint4*>(half + r1 * 128 + ((chunk ^ (r1 & 7)) << 4)) =
-            make_uint4(c1[4 * j], c1[4 * j + 1], c1[4 * j + 2], c1[4 * j + 3]);
+        for (int j = 0; j < 4; ++j) {
+          const int chunk = (rb & 1) * 4 + j;
+          *reinterpret_cast<uint4*>(half + r0 * 128 + ((chunk ^ (r0 & 7)) << 4)) =
+              make_uint4(c0[4 * j], c0[4 * j + 1], c0[4 * j + 2], c0[4 * j + 3]);
+          *reinterpret_cast<uint4*>(half + r1 * 128 + ((chunk ^ (r1 & 7)) << 4)) =
+              make_uint4(c1[4 * j], c1[4 * j + 1], c1[4 * j + 2], c1[4 * j + 3]);
+        }
+      } else {
+        // columns 2p and 2p+1 of the source are rows of the transposed output: 64 bytes each
+        bf16* o0 = a.o_colT + (static_cast<int64_t>(b) * C + col0 + 2 * p) * R + row0 + rb * 32;
+        bf16* o1 = o0 + R;
+        if (col32) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            ptx::st_global_v8(o0 + 16 * j, make_uint4(c0[8 * j], c0[8 * j + 1], c0[8 * j + 2], c0[8 * j + 3]),
+                              make_uint4(c0[8 * j + 4], c0[8 * j + 5], c0[8 * j + 6], c0[8 * j + 7]));
+            ptx::st_global_v8(o1 + 16 * j, make_uint4(c1[8 * j], c1[8 * j + 1], c1[8 * j + 2], c1[8 * j + 3]),
+                              make_uint4(c1[8 * j + 4], c1[8 * j + 5], c1[8 * j + 6], c1[8 * j + 7]));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            reinterpret_cast<uint4*>(o0)[j] = make_uint4(c0[4 * j], c0[4 * j + 1], c0[4 * j + 2], c0[4 * j + 3]);
+            reinterpret_cast<uint4*>(o1)[j] = make_uint4(c1[4 * j], c1[4 * j + 1], c1[4 * j + 2], c1[4 * j + 3]);
+          }
+        }
       }
     } else {
       // ---- row-wise: thread -> 8-column chunk ``cchunk`` of rows tid/16 + 16 i
       const int cchunk = tid & 15;
-  #pragma unroll
+#pragma unroll
       for (int i = 0; i < QT_LOADS; ++i) {
         const int lr = (tid >> 4) + 16 * i;
         const uint4 v = *reinterpret_cast<const uint4*>(in + lr * 256 + cchunk * 16);
@@ -508,15 +562,19 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
         const uint32_t sb = e8m0_from_amax_bits(m, a.scale_floor, a.e5m2);
-        const float inv = e8m0_inv_scale(sb);
+        const float inv = pt ? pts : e8m0_inv_scale(sb);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
         uint32_t q[4];
-  #pragma unroll
+#pragma unroll
         for (int j = 0; j < 4; ++j)
           q[j] = fp8x2(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv, a.e5m2);
-        *reinterpret_cast<uint2*>(qrow + lr * 128 + (((cchunk >> 1) ^ (lr & 7)) << 4) + ((cchunk & 1) << 3)) =
-            make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
-        if ((cchunk & 3) == 0) satom_row[sf_mma_offset(lr, (cchunk >> 2) & 3, 4)] = static_cast<uint8_t>(sb);
+        const uint2 qq = make_uint2(q[0] | (q[1] << 16), q[2] | (q[3] << 16));
+        if (!DIRECT)
+          *reinterpret_cast<uint2*>(qrow + lr * 128 + (((cchunk >> 1) ^ (lr & 7)) << 4) + ((cchunk & 1) << 3)) = qq;
+        else
+          *reinterpret_cast<uint2*>(a.q_row + (static_cast<int64_t>(b) * R + dst_row(row0 + lr)) * C + col0 +
+                                    cchunk * 8) = qq;
+        if ((cchunk & 3) == 0 && !pt) satom_row[sf_mma_offset(lr, (cchunk >> 2) & 3, 4)] = static_cast<uint8_t>(sb);
       }
 
       // ---- column-wise: thread -> columns (2p, 2p+1), 32-row block rb
@@ -525,16 +583,16 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         const uint32_t* words = reinterpret_cast<const uint32_t*>(in);  // 64 bf16 pairs per row
         uint32_t wv[32];
         uint32_t m2 = 0;
-  #pragma unroll
+#pragma unroll
         for (int i = 0; i < 32; ++i) {
           wv[i] = words[(rb * 32 + i) * 64 + p];
           m2 = absmax_bf16x2(m2, wv[i]);
         }
         const uint32_t sb0 = e8m0_from_amax_bits(m2 << 16, a.scale_floor, a.e5m2);
         const uint32_t sb1 = e8m0_from_amax_bits(m2 & 0xFFFF0000u, a.scale_floor, a.e5m2);
-        const float inv0 = e8m0_inv_scale(sb0), inv1 = e8m0_inv_scale(sb1);
+        const float inv0 = pt ? pts : e8m0_inv_scale(sb0), inv1 = pt ? pts : e8m0_inv_scale(sb1);
         uint32_t q0[8], q1[8];
-  #pragma unroll
+#pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint32_t lo0 =
               fp8x2(__uint_as_float(wv[4 * i] << 16) * inv0, __uint_as_float(wv[4 * i + 1] << 16) * inv0, a.e5m2);
@@ -547,21 +605,38 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
           q0[i] = lo0 | (hi0 << 16);
           q1[i] = lo1 | (hi1 << 16);
         }
-        const int r0 = 2 * p, r1 = 2 * p + 1;  // rows of the transposed code tile
-        uint8_t* row0p = qcol + r0 * 128;
-        uint8_t* row1p = qcol + r1 * 128;
-        *reinterpret_cast<uint4*>(row0p + (((2 * rb) ^ (r0 & 7)) << 4)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
-        *reinterpret_cast<uint4*>(row0p + (((2 * rb + 1) ^ (r0 & 7)) << 4)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
-        *reinterpret_cast<uint4*>(row1p + (((2 * rb) ^ (r1 & 7)) << 4)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
-        *reinterpret_cast<uint4*>(row1p + (((2 * rb + 1) ^ (r1 & 7)) << 4)) = make_uint4(q1[4], q1[5], q1[6], q1[7]);
-        satom_col[sf_mma_offset(2 * p, rb, 4)] = static_cast<uint8_t>(sb0);
-        satom_col[sf_mma_offset(2 * p + 1, rb, 4)] = static_cast<uint8_t>(sb1);
+        if (!DIRECT) {
+          const int r0 = 2 * p, r1 = 2 * p + 1;  // rows of the transposed code tile
+          uint8_t* row0p = qcol + r0 * 128;
+          uint8_t* row1p = qcol + r1 * 128;
+          *reinterpret_cast<uint4*>(row0p + (((2 * rb) ^ (r0 & 7)) << 4)) = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+          *reinterpret_cast<uint4*>(row0p + (((2 * rb + 1) ^ (r0 & 7)) << 4)) = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+          *reinterpret_cast<uint4*>(row1p + (((2 * rb) ^ (r1 & 7)) << 4)) = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+          *reinterpret_cast<uint4*>(row1p + (((2 * rb + 1) ^ (r1 & 7)) << 4)) = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+        } else {
+          // columns 2p and 2p+1 are rows of the transposed codes: one 32-byte run each
+          uint8_t* c0p = a.q_colT + (static_cast<int64_t>(b) * C + col0 + 2 * p) * R + row0 + rb * 32;
+          uint8_t* c1p = c0p + R;
+          if (col32) {
+            ptx::st_global_v8(c0p, make_uint4(q0[0], q0[1], q0[2], q0[3]), make_uint4(q0[4], q0[5], q0[6], q0[7]));
+            ptx::st_global_v8(c1p, make_uint4(q1[0], q1[1], q1[2], q1[3]), make_uint4(q1[4], q1[5], q1[6], q1[7]));
+          } else {
+            reinterpret_cast<uint4*>(c0p)[0] = make_uint4(q0[0], q0[1], q0[2], q0[3]);
+            reinterpret_cast<uint4*>(c0p)[1] = make_uint4(q0[4], q0[5], q0[6], q0[7]);
+            reinterpret_cast<uint4*>(c1p)[0] = make_uint4(q1[0], q1[1], q1[2], q1[3]);
+            reinterpret_cast<uint4*>(c1p)[1] = make_uint4(q1[4], q1[5], q1[6], q1[7]);
+          }
+        }
+        if (!pt) {
+          satom_col[sf_mma_offset(2 * p, rb, 4)] = static_cast<uint8_t>(sb0);
+          satom_col[sf_mma_offset(2 * p + 1, rb, 4)] = static_cast<uint8_t>(sb1);
+        }
       }
     }
 
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // code tiles -> visible to the copy engine
-    __syncthreads();  // the source tile is consumed, the code tiles and scale tiles are complete
-    if (tid == 0) {
+    if (!DIRECT) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // code tiles -> the copy engine
+    __syncthreads();  // the source tile is consumed; code tiles (staged) and scale tiles are complete
+    if (!DIRECT && tid == 0) {
       if (a.mx) {
         asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
                          reinterpret_cast<uint64_t>(&a.tmap_qrow)),
@@ -592,17 +667,15 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         issued_last = tn;
         if (a.tma_gather && tn + static_cast<int>(gridDim.x) < tiles) gather_rows(tn + gridDim.x, y_next);
       }
-    } else if (a.mx && tid >= 32 && tid < 64) {  // warp 1: the two 512-byte scale tiles, 16 bytes per lane
+    } else if (a.mx && !pt && tid >= 32 && tid < 64) {  // warp 1: the two 512-byte scale tiles, 16 bytes per lane
       const int l = tid - 32;
-      {
-        uint8_t* sr = a.s_row + static_cast<int64_t>(b) * R * KBr;
-        reinterpret_cast<uint4*>(sr + ((dst_row(row0) / 128) * (KBr / 4) + col0 / 128) * 512)[l] =
-            reinterpret_cast<const uint4*>(satom_row)[l];
-        if (a.do_col) {
-          uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
-          reinterpret_cast<uint4*>(sc + ((col0 / 128) * (KBc / 4) + row0 / 128) * 512)[l] =
-              reinterpret_cast<const uint4*>(satom_col)[l];
-        }
+      uint8_t* sr = a.s_row + static_cast<int64_t>(b) * R * KBr;
+      reinterpret_cast<uint4*>(sr + ((dst_row(row0) / 128) * (KBr / 4) + col0 / 128) * 512)[l] =
+          reinterpret_cast<const uint4*>(satom_row)[l];
+      if (a.do_col) {
+        uint8_t* sc = a.s_colT + static_cast<int64_t>(b) * C * KBc;
+        reinterpret_cast<uint4*>(sc + ((col0 / 128) * (KBc / 4) + row0 / 128) * 512)[l] =
+            reinterpret_cast<const uint4*>(satom_col)[l];
       }
     }
   }
@@ -616,7 +689,7 @@ __global__ void __launch_bounds__(256, QW_CTAS_PER_SM) quant_w_tma_kernel(const 
         ptx::mbar_wait(&full[k % QW_NIN], static_cast<uint32_t>((k / QW_NIN) & 1), &never, kWaitLimitCycles);
       }
     }
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    if (!DIRECT) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
   }
 }
 
@@ -636,10 +709,7 @@ unpermute_kernel(const bf16* __restrict__ rows, const int32_t* __restrict__ src_
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int64_t r = src_to_sorted[t * k + j];
-      if (r < 0) continue;  // a slot the routing rejected (expert index out of range): contributes nothing
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(rows + r * d + c));
+    auto add = [&](const uint4& v, int j) {
       const bf16* h = reinterpret_cast<const bf16*>(&v);
       if (probs) {
         const float w = probs[t * k + j];
@@ -648,6 +718,20 @@ unpermute_kernel(const bf16* __restrict__ rows, const int32_t* __restrict__ src_
       } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = __fadd_rn(acc[q], __bfloat162float(h[q]));
+      }
+    };
+    if (k == 2) {  // top-2: both rows' loads in flight before either is used
+      const int64_t r0 = src_to_sorted[t * 2], r1 = src_to_sorted[t * 2 + 1];
+      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+      if (r0 >= 0) v0 = __ldg(reinterpret_cast<const uint4*>(rows + r0 * d + c));
+      if (r1 >= 0) v1 = __ldg(reinterpret_cast<const uint4*>(rows + r1 * d + c));
+      if (r0 >= 0) add(v0, 0);
+      if (r1 >= 0) add(v1, 1);
+    } else {
+      for (int j = 0; j < k; ++j) {
+        const int64_t r = src_to_sorted[t * k + j];
+        if (r < 0) continue;  // a slot the routing rejected (expert index out of range): contributes nothing
+        add(__ldg(reinterpret_cast<const uint4*>(rows + r * d + c)), j);
       }
     }
     uint4 o;
@@ -658,30 +742,41 @@ unpermute_kernel(const bf16* __restrict__ rows, const int32_t* __restrict__ src_
   }
 }
 
-// d_topk_prob[t][j] = sum over n-tiles (ascending) of the partial row sums of the ScaledSwiGLU
-// probability gradient at row(t, j).  Threads walk the rows (consecutive threads read consecutive
-// words of every partial) and write the sum to the row's slot; slots the routing rejected (no row)
-// get zero.
+// d_topk_prob[t][j] = the sum of the partial row sums of the ScaledSwiGLU probability gradient at
+// row(t, j), over all n-tiles.  Four consecutive threads share a row: thread q sums the q-th quarter
+// of the partials in ascending order (eight independent loads in flight; consecutive rows are
+// consecutive words of every partial), then the four quarter sums are added in order q = 0..3.  The
+// sum is written to the row's slot; slots the routing rejected (no row) get zero.
 __global__ void dprob_reduce_kernel(const float* __restrict__ part, int n_parts, int64_t part_stride,
                                     const int32_t* __restrict__ sorted_to_src, int64_t rows,
                                     const int32_t* __restrict__ src_to_sorted, int64_t Tk,
                                     float* __restrict__ d_prob) {
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  for (int64_t r = i0; r < rows; r += stride) {
-    const int32_t s = sorted_to_src[r];
-    if (s < 0) continue;  // padding row
+  const int lane = threadIdx.x & 31, q = lane & 3;
+  const int per = (n_parts + 3) / 4;
+  const int n0 = min(n_parts, q * per), n1 = min(n_parts, n0 + per);
+  // the loop bound is the same for the whole warp, so every lane reaches the shuffles below
+  for (int64_t wbase = i0 - lane; wbase < 4 * rows; wbase += stride) {
+    const int64_t r = (wbase + lane) / 4;
+    const int32_t s = r < rows ? sorted_to_src[r] : -1;
     float acc = 0.f;
-    int n = 0;
-    for (; n + 8 <= n_parts; n += 8) {  // eight independent loads in flight, summed in order
-      float v[8];
+    if (s >= 0) {
+      int n = n0;
+      for (; n + 8 <= n1; n += 8) {
+        float v[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = __ldg(part + (n + q) * part_stride + r);
+        for (int u = 0; u < 8; ++u) v[u] = __ldg(part + (n + u) * part_stride + r);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc = __fadd_rn(acc, v[q]);
+        for (int u = 0; u < 8; ++u) acc = __fadd_rn(acc, v[u]);
+      }
+      for (; n < n1; ++n) acc = __fadd_rn(acc, __ldg(part + n * part_stride + r));
     }
-    for (; n < n_parts; ++n) acc = __fadd_rn(acc, __ldg(part + n * part_stride + r));
-    d_prob[s] = acc;
+    // quarter sums in order 0..3 (the four lanes of a row are adjacent)
+    const float a1 = __shfl_down_sync(0xffffffffu, acc, 1, 4);
+    const float a2 = __shfl_down_sync(0xffffffffu, acc, 2, 4);
+    const float a3 = __shfl_down_sync(0xffffffffu, acc, 3, 4);
+    if (q == 0 && s >= 0) d_prob[s] = __fadd_rn(__fadd_rn(__fadd_rn(acc, a1), a2), a3);
   }
   for (int64_t s = i0; s < Tk; s += stride)
     if (src_to_sorted[s] < 0) d_prob[s] = 0.f;
@@ -718,14 +813,123 @@ cudaError_t launch_route(const int32_t* topk_idx, const float* topk_prob, int Tk
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------------------------
+// Per-tensor FP8 maxima: current scaling needs each tensor's largest magnitude before any of it is
+// quantised.  Magnitudes compare as bf16 bit patterns (bits & 0x7FFF grows with |x| for finite
+// values) and are kept as fp32 bits, so that atomicMax on unsigned words orders them.
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t absmax8_bf16(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+  return m;
+}
+
+// grid (row slices, batch): block x of batch b takes rows x, x + gridDim.x, ...
+__global__ void __launch_bounds__(256) amax_batched_kernel(const __grid_constant__ PtrArray ptrs, const bf16* src,
+                                                           int64_t batch_stride, int64_t rows, int64_t cols,
+                                                           int64_t ld, uint32_t* __restrict__ amax) {
+  __shared__ uint32_t wmax[8];
+  const int b = blockIdx.y;
+  const bf16* base = ptrs.p[b] ? static_cast<const bf16*>(ptrs.p[b]) : src + b * batch_stride;
+  const int64_t cv = cols / 8;
+  uint32_t m = 0;
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint4* row = reinterpret_cast<const uint4*>(base + r * ld);
+    for (int64_t c = threadIdx.x; c < cv; c += blockDim.x) m = max(m, absmax8_bf16(__ldcs(row + c)));
+  }
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < 8; ++w) m = max(m, wmax[w]);
+    if (m) atomicMax(amax + b, m << 16);
+  }
+}
+
+// One warp per row of the expert-sorted order (rows without a slot are skipped): the row reads token
+// sorted_to_src[r] / k and belongs to the expert whose padded segment poffsets[e] .. poffsets[e+1]
+// holds r; per-CTA maxima in shared memory first.
+__global__ void __launch_bounds__(256) amax_routed_kernel(const bf16* __restrict__ x, int64_t ld, int64_t d,
+                                                          const int32_t* __restrict__ sorted_to_src,
+                                                          const int32_t* __restrict__ poffsets, int64_t rows, int k,
+                                                          int E, uint32_t* __restrict__ amax) {
+  __shared__ uint32_t sm[MOE_MAX_EXPERTS];
+  __shared__ int32_t off[MOE_MAX_EXPERTS + 1];
+  for (int i = threadIdx.x; i < E; i += blockDim.x) sm[i] = 0;
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) off[i] = poffsets[i];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += nwarps) {
+    const int32_t slot = sorted_to_src[r];
+    if (slot < 0 || r >= off[E]) continue;  // padding row
+    int lo = 0, hi = E;                     // largest e with off[e] <= r
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid] <= r) lo = mid; else hi = mid;
+    }
+    const uint4* row = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(slot / k) * ld);
+    uint32_t m = 0;
+    for (int64_t c = lane; c < d / 8; c += 32) m = max(m, absmax8_bf16(row[c]));
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (lane == 0 && m) atomicMax(&sm[lo], m);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < E; i += blockDim.x)
+    if (sm[i]) atomicMax(amax + i, sm[i] << 16);
+}
+
+cudaError_t launch_amax_batched(const PtrArray& src_ptrs, const bf16* src, int64_t batch_stride, int batch,
+                                int64_t rows, int64_t cols, int64_t ld, uint32_t* amax, int num_sms,
+                                cudaStream_t st) {
+  if (batch <= 0 || rows <= 0 || cols <= 0) return cudaSuccess;
+  if (cols % 8 || ld % 8 || batch > 65535) return cudaErrorInvalidValue;
+  const int64_t per_batch = std::max<int64_t>(1, static_cast<int64_t>(num_sms) * 8 / batch);
+  dim3 grid(static_cast<unsigned>(std::min<int64_t>(rows, per_batch)), static_cast<unsigned>(batch));
+  amax_batched_kernel<<<grid, 256, 0, st>>>(src_ptrs, src, batch_stride, rows, cols, ld, amax);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax_routed(const bf16* x, int64_t ld, int64_t d, const int32_t* sorted_to_src,
+                               const int32_t* poffsets, int64_t rows, int k, int E, uint32_t* amax, int num_sms,
+                               cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  if (d % 8 || ld % 8 || E > MOE_MAX_EXPERTS) return cudaErrorInvalidValue;
+  const int64_t blocks = std::min<int64_t>(ceil_div(rows, 8), static_cast<int64_t>(num_sms) * 4);
+  amax_routed_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(x, ld, d, sorted_to_src, poffsets, rows, k, E,
+                                                                     amax);
+  return cudaGetLastError();
+}
+
+__global__ void fp8_scales_kernel(uint32_t* v, int n, int e5m2) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) v[i] = __float_as_uint(fp8_tensor_scale(v[i], e5m2));
+}
+
+cudaError_t launch_fp8_scales(uint32_t* amax_to_scale, int n, int e5m2, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  fp8_scales_kernel<<<(n + 255) / 256, 256, 0, st>>>(amax_to_scale, n, e5m2);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quant(const QuantArgs& a, int batch, int num_sms, cudaStream_t st) {
   if (a.rows == 0 || a.cols == 0 || batch == 0) return cudaSuccess;
-  if (a.tma_load && a.tma_store && (a.mx ? a.do_row : (a.do_col && !a.do_row))) {
+  const bool persistent = a.tma_load && a.tma_store && (a.mx ? a.do_row : (a.do_col && !a.do_row));
+  if (a.pt_amax && (!persistent || !a.mx || (a.pt_poff ? a.pt_E : batch) > MOE_MAX_EXPERTS))
+    return cudaErrorInvalidValue;  // per-tensor FP8 exists only in the TMA-fed kernel
+  if (persistent) {
     const int64_t tiles = (a.rows / QT_ROWS) * (a.cols / QT_COLS) * batch;
-    cudaError_t e = cudaFuncSetAttribute(quant_w_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QW_SMEM);
+    // direct stores for the gathers, staged TMA stores otherwise (measured: the gathers run 13% faster
+    // direct, the weight quantisation 10% faster staged)
+    auto kern = a.tma_gather ? quant_w_tma_kernel<true> : quant_w_tma_kernel<false>;
+    const int smem = a.tma_gather ? QwShape<true>::SMEM : QwShape<false>::SMEM;
+    const int per_sm = a.tma_gather ? QwShape<true>::CTAS_PER_SM : QwShape<false>::CTAS_PER_SM;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const int grid = static_cast<int>(std::min<int64_t>(tiles, static_cast<int64_t>(num_sms) * QW_CTAS_PER_SM));
-    quant_w_tma_kernel<<<grid, 256, QW_SMEM, st>>>(a, static_cast<int>(tiles));
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, static_cast<int64_t>(num_sms) * per_sm));
+    kern<<<grid, 256, smem, st>>>(a, static_cast<int>(tiles));
     return cudaGetLastError();
   }
   dim3 grid(static_cast<unsigned>(ceil_div(a.cols, QT_COLS)), static_cast<unsigned>(ceil_div(a.rows, QT_ROWS)),
@@ -752,7 +956,7 @@ cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_str
                                 int64_t rows, const int32_t* src_to_sorted, int64_t Tk, float* d_prob,
                                 cudaStream_t st) {
   if (Tk == 0) return cudaSuccess;
-  const int64_t blocks = std::min<int64_t>(ceil_div(std::max(rows, Tk), 256), 4096);
+  const int64_t blocks = std::min<int64_t>(ceil_div(std::max(4 * rows, Tk), 256), 4096);
   dprob_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(part, n_parts, part_stride, sorted_to_src, rows,
                                                                       src_to_sorted, Tk, d_prob);
   return cudaGetLastError();

@@ -45,6 +45,13 @@ struct QuantArgs {
   // src_rows, which the copy fills with zeros)
   int tma_gather;
   int64_t src_rows;
+  // per-tensor FP8 (with mx = 1: codes only, no scale bytes): a tile's codes are E4M3 / E5M2 of
+  // v * s with s = vmax / amax of its tensor (fp8_tensor_scale); amax as fp32 bits from
+  // pt_amax[b] for batch b, or, with pt_poff, from pt_amax[e] for the expert e whose padded rows
+  // pt_poff[e] .. pt_poff[e+1] hold the tile (one [rows, cols] source of expert segments)
+  const uint32_t* pt_amax;
+  const int32_t* pt_poff;
+  int pt_E;
   int* status;                 // device status word (a bounded wait that expired)
   const int* stall_flag;       // test hook: waited on once per CTA (TMA-fed kernel) for stall_limit cycles
   long long stall_limit;
@@ -59,6 +66,20 @@ cudaError_t launch_unpermute(const bf16* rows, const int32_t* src_to_sorted, con
 cudaError_t launch_dprob_reduce(const float* part, int n_parts, int64_t part_stride, const int32_t* sorted_to_src,
                                 int64_t rows, const int32_t* src_to_sorted, int64_t Tk, float* d_prob,
                                 cudaStream_t st);
+// Per-tensor maxima (fp32 bits, atomicMax into ``amax`` which the caller zeroes first):
+// amax[b] = max |x| over batch b of a [batch, rows, cols] bf16 source (per-batch pointers in
+// ``src_ptrs``, or ``src`` with ``batch_stride`` elements between batches; rows ``ld`` apart) ...
+cudaError_t launch_amax_batched(const PtrArray& src_ptrs, const bf16* src, int64_t batch_stride, int batch,
+                                int64_t rows, int64_t cols, int64_t ld, uint32_t* amax, int num_sms,
+                                cudaStream_t st);
+// ... and amax[e] = max |x[t]| over the tokens t routed to expert e: the rows r of the expert-sorted
+// order (``rows`` of them) with a slot sorted_to_src[r] >= 0 read token sorted_to_src[r] / k and
+// belong to the expert e with poffsets[e] <= r < poffsets[e+1]; x is [T, d] with rows ``ld`` apart.
+cudaError_t launch_amax_routed(const bf16* x, int64_t ld, int64_t d, const int32_t* sorted_to_src,
+                               const int32_t* poffsets, int64_t rows, int k, int E, uint32_t* amax, int num_sms,
+                               cudaStream_t st);
+// In place: the fp32 bits of each of n tensor maxima become that tensor's per-tensor FP8 scale.
+cudaError_t launch_fp8_scales(uint32_t* amax_to_scale, int n, int e5m2, cudaStream_t st);
 cudaError_t launch_dequant(const uint8_t* q, const uint8_t* s, int64_t R, int64_t C, int sf_mma, float* out,
                            int num_sms, cudaStream_t st);
 

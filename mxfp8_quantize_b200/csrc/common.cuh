@@ -46,6 +46,15 @@ __device__ __forceinline__ uint32_t fp8x2(float lo, float hi, int e5m2) {
   return static_cast<uint32_t>(
       __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, e5m2 ? __NV_E5M2 : __NV_E4M3));
 }
+// Per-tensor FP8 scale (current scaling): s = vmax / amax rounded to nearest in fp32 (vmax 448 for
+// E4M3, 57344 for E5M2); 1 for an all-zero tensor; the largest finite fp32 when the quotient
+// overflows.  ``amax_bits``: the fp32 bits of the tensor's largest magnitude.
+__device__ __forceinline__ float fp8_tensor_scale(uint32_t amax_bits, int e5m2) {
+  const float amax = __uint_as_float(amax_bits);
+  if (!(amax > 0.f)) return 1.f;
+  const float s = __fdiv_rn(e5m2 ? 57344.f : 448.f, amax);
+  return isinf(s) ? __uint_as_float(0x7F7FFFFFu) : s;
+}
 // 2^-(byte-127) as an fp32 (byte <= 253 for every finite input).
 __device__ __forceinline__ float e8m0_inv_scale(uint32_t byte) {
   return __uint_as_float((254u - byte) << 23);

@@ -193,6 +193,14 @@ __device__ __forceinline__ void e4m3x8_to_float(uint32_t lo, uint32_t hi, float 
       o[4 * k + 2 * h + 1] = v.y * scale;
     }
 }
+// Largest magnitude of eight packed bf16 values, as bf16 bits (bits & 0x7FFF grows with |x|).
+__device__ __forceinline__ uint32_t absmax_bf16x8_bits(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+  return m;
+}
 // 2^(byte - 127) as an fp32 (byte 0: 2^-127, a subnormal).
 __device__ __forceinline__ float e8m0_scale(uint32_t byte) {
   return byte ? __uint_as_float(byte << 23) : __uint_as_float(0x00400000u);
@@ -299,6 +307,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const bool K128 = MX || g.fp8;  // 8-bit operands: 128 K elements per 128-byte stage row
 
   // ---- set-up: tile prefix over experts, barriers, TMEM
   if (threadIdx.x == 0) {
@@ -385,8 +394,8 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     const uint32_t tx = S::A_BYTES + S::B_BYTES + (MX ? 512 + S::SFB_BYTES : 0);
     for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
       Tile tl;
-      decode_tile(t, s, g, MX, tl);
-      const int bk = MX ? 128 : 64;
+      decode_tile(t, s, g, K128, tl);
+      const int bk = K128 ? 128 : 64;
       if (EPI == EPI_FUSED_FWD && tl.down) {
         // the tile's 128 rows of a are complete once every gate_up tile of its row block has released them
         if (!ptx::wait_counter(g.mblock_done + tl.a_row / BM, g.n_tiles * S::EPI_WARPS, abort_flag, lim)) break;
@@ -473,7 +482,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     const uint32_t a_fmt = ptx::idesc_a_format(g.a_e5m2 ? ptx::kFmtE5M2 : ptx::kFmtE4M3);  // A's element format
     for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
       Tile tl;
-      decode_tile(t, s, g, MX, tl);
+      decode_tile(t, s, g, K128, tl);
       if (tl.nk == 0) continue;
       const int buf = S::NBUF == 2 ? (local & 1) : 0;
       const uint32_t acc_par = static_cast<uint32_t>((S::NBUF == 2 ? (local >> 1) : local) & 1);
@@ -500,6 +509,10 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           for (int k = 0; k < 4; ++k)
             ptx::tc_mma_mxf8(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(BM, BN, k, k) | a_fmt, sfa_t,
                              sfb_t, (kb | k) != 0);
+        } else if (g.fp8) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            ptx::tc_mma_f8(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_f8(BM, BN) | a_fmt, (kb | k) != 0);
         } else {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
@@ -530,11 +543,30 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
                                                 (warp - S::LEAD) * S::STAGING_PER_WARP);
     const EpiArgs& ep = g.epi;
     int local = 0;
+    // per-tensor FP8: this warp's largest magnitude written for expert amax_e so far (bf16 bits),
+    // added to ep.amax_out[amax_e] when the expert changes and at the end
+    uint32_t amax_run = 0;
+    int amax_e = -1;
+    auto amax_flush = [&]() {
+      if (MX || !ep.amax_out || amax_e < 0) return;
+      const unsigned mask = __activemask();
+      const uint32_t m = __reduce_max_sync(mask, amax_run);
+      if (lane == __ffs(mask) - 1 && m) atomicMax(ep.amax_out + amax_e, m << 16);
+    };
     for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
       Tile tl;
-      decode_tile(t, s, g, MX, tl);
+      decode_tile(t, s, g, K128, tl);
       const int64_t row_w = tl.a_row + 32 * q;  // first row of this warp
       const int64_t row = row_w + lane;
+      // per-tensor FP8: the accumulator times 1/s_a * 1/s_b of the tile's expert
+      float fac = 1.f;
+      if (!MX && g.pt_amax_a)
+        fac = __frcp_rn(fp8_tensor_scale(g.pt_amax_a[tl.e], g.a_e5m2)) * __frcp_rn(fp8_tensor_scale(g.pt_amax_b[tl.e], 0));
+      if (!MX && ep.amax_out && tl.e != amax_e) {
+        amax_flush();
+        amax_e = tl.e;
+        amax_run = 0;
+      }
       if (tl.nk == 0) {
         // K-grouped expert without tokens: its weight gradient is zero
         if (EPI == EPI_STORE) {
@@ -562,7 +594,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           float v[32];
           load_acc32(t_lane + CPT * ch + 32 * cc, v);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[16 * cc + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          for (int i = 0; i < 16; ++i) pk[16 * cc + i] = pack_bf16x2(v[2 * i] * fac, v[2 * i + 1] * fac);
         }
         ptx::tc_fence_before();
         __syncwarp();
@@ -594,6 +626,13 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           float gv[32], uv[32];
           load_acc32(t_lane + OPT * ch + 32 * cc, gv);
           load_acc32(t_lane + BN / 2 + OPT * ch + 32 * cc, uv);
+          if (!MX) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              gv[i] *= fac;
+              uv[i] *= fac;
+            }
+          }
           if (cc == G - 1) {
             ptx::tc_fence_before();
             __syncwarp();
@@ -629,7 +668,11 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           } else {
             bf16* dst = ep.o_row + row * f + j;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) ptx::st_global_v8(dst + 16 * i, pack_bf16x8(gv + 16 * i), pack_bf16x8(gv + 16 * i + 8));
+            for (int i = 0; i < 2; ++i) {
+              const uint4 lo = pack_bf16x8(gv + 16 * i), hi = pack_bf16x8(gv + 16 * i + 8);
+              ptx::st_global_v8(dst + 16 * i, lo, hi);
+              if (ep.amax_out) amax_run = max(amax_run, max(absmax_bf16x8_bits(lo), absmax_bf16x8_bits(hi)));
+            }
             if (ep.o_colT) colwise_bf16<S::PASS>(gv, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
           }
         }
@@ -703,6 +746,10 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           const int64_t j = j0 + 32 * cc;
           float da[32];
           load_acc32(t_lane + CPT * ch + 32 * cc, da);
+          if (!MX) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) da[i] *= fac;
+          }
           if (cc == G - 1) {
             ptx::tc_fence_before();
             __syncwarp();
@@ -757,16 +804,24 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             bf16* d1 = d0 + f;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-              ptx::st_global_v8(d0 + 16 * i, pack_bf16x8(dg + 16 * i), pack_bf16x8(dg + 16 * i + 8));
-              ptx::st_global_v8(d1 + 16 * i, pack_bf16x8(du + 16 * i), pack_bf16x8(du + 16 * i + 8));
+              const uint4 g0 = pack_bf16x8(dg + 16 * i), g1 = pack_bf16x8(dg + 16 * i + 8);
+              const uint4 u0 = pack_bf16x8(du + 16 * i), u1 = pack_bf16x8(du + 16 * i + 8);
+              ptx::st_global_v8(d0 + 16 * i, g0, g1);
+              ptx::st_global_v8(d1 + 16 * i, u0, u1);
+              if (ep.amax_out)
+                amax_run = max(amax_run, max(max(absmax_bf16x8_bits(g0), absmax_bf16x8_bits(g1)),
+                                             max(absmax_bf16x8_bits(u0), absmax_bf16x8_bits(u1))));
             }
-            colwise_bf16<S::PASS>(dg, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
-            colwise_bf16<S::PASS>(du, stage_buf, ep.o_colT + (f + j) * ep.cap + row_w, ep.cap);
+            if (ep.o_colT) {
+              colwise_bf16<S::PASS>(dg, stage_buf, ep.o_colT + j * ep.cap + row_w, ep.cap);
+              colwise_bf16<S::PASS>(du, stage_buf, ep.o_colT + (f + j) * ep.cap + row_w, ep.cap);
+            }
           }
         }
         ep.dp_part[(static_cast<int64_t>(tl.nb) * NPART + ch) * ep.cap + row] = dp;
       }
     }
+    amax_flush();
   }
 
   __syncthreads();

@@ -36,6 +36,8 @@ struct EpiArgs {
   int scale_floor;    // MXFP8 shared exponent of the requantisations: 0 round-up rule, 1 OCP floor rule
   int grad_e5m2;      // DSWIGLU: dh requantised with E5M2 elements (gradient-format variant)
   float* dp_part;     // DSWIGLU: [parts * n_tiles, cap] partial sums of the probability gradient
+  uint32_t* amax_out; // per-tensor FP8 (bf16 o_row outputs): per expert, the largest magnitude written,
+                      // as fp32 bits (atomicMax; the caller zeroes it)
 };
 
 struct GemmArgs {
@@ -60,7 +62,13 @@ struct GemmArgs {
   const uint8_t* sfb;
   int64_t sfb_kb4;
   int64_t sfb_expert_rows;  // rows of B per expert (M-grouped), for the scale tile index
-  int a_e5m2;          // MXFP8: A's elements are E5M2 (B's stay E4M3)
+  int a_e5m2;          // MXFP8 / FP8: A's elements are E5M2 (B's stay E4M3)
+  // per-tensor FP8 (with mx = false): 8-bit operands without block scales, kind::f8f6f4 MMAs over
+  // 128-element K steps; the epilogue multiplies the accumulator of expert e by
+  // 1/s_a(e) * 1/s_b(e), s = fp8_tensor_scale of pt_amax_a[e] (A's format) and pt_amax_b[e] (E4M3)
+  int fp8;
+  const uint32_t* pt_amax_a;
+  const uint32_t* pt_amax_b;
   // EPI_FUSED_FWD: the down GEMM that follows the gate_up tiles (A = a [rows, f], B = W2 [E, d, f]),
   // its output rows go to epi.out / epi.ldo
   CUtensorMap tmap_a2;
@@ -85,13 +93,14 @@ int gemm_tile_n(int epi);
 // Partial sums of the probability gradient the dSwiGLU epilogue writes per output tile and row.
 int gemm_dswiglu_parts();
 
-// Launch one grouped GEMM.  ``mx``: MXFP8 (kind::mxf8f6f4) or BF16 (kind::f16).
+// Launch one grouped GEMM.  ``mx``: MXFP8 (kind::mxf8f6f4); otherwise BF16 (kind::f16), or per-tensor
+// FP8 (kind::f8f6f4) when args.fp8 is set.
 cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st);
 
 // Tensor-core peak loop (peak.cu): one CTA per SM issuing iters x 4 MMAs of 128 x 256 on operands
-// resident in shared memory; its FLOPs per launch.
-cudaError_t launch_tensor_peak(bool mx, long long iters, int scale_refresh, int num_sms, int* status,
+// resident in shared memory (kind 0 BF16, 1 MXFP8, 2 per-tensor FP8); its FLOPs per launch.
+cudaError_t launch_tensor_peak(int kind, long long iters, int scale_refresh, int num_sms, int* status,
                                cudaStream_t st);
-double tensor_peak_flops(bool mx, int num_sms, long long iters);
+double tensor_peak_flops(int kind, int num_sms, long long iters);
 
 }  // namespace moemx

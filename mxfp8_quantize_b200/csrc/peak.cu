@@ -1,8 +1,8 @@
-// Tensor-core peak loop: the dense rate of this GPU's tcgen05 tensor cores for the two operand
+// Tensor-core peak loop: the dense rate of this GPU's tcgen05 tensor cores for the three operand
 // kinds the grouped GEMMs use (block-scaled MXFP8, kind::mxf8f6f4 with one E8M0 scale per 32 K;
-// and BF16, kind::f16), measured with every operand resident in shared memory so that no memory
-// traffic bounds it.  It is the denominator of the GEMMs' roofline fractions (ai4snews,
-// paragraph 2: MXFP8 runs on Blackwell's tensor-core instructions).
+// per-tensor FP8, kind::f8f6f4; and BF16, kind::f16), measured with every operand resident in
+// shared memory so that no memory traffic bounds it.  It is the denominator of the GEMMs' roofline
+// fractions (ai4snews, paragraph 2: MXFP8 runs on Blackwell's tensor-core instructions).
 //
 // One CTA per SM.  Warp 2 allocates all 512 TMEM columns; one thread of warp 1 issues ``iters``
 // groups of four M=128, N=256 MMAs (K = 4 x 32 E4M3 or 4 x 16 bf16: one 128-byte K step, the
@@ -25,8 +25,10 @@ constexpr long long PK_MAX_ITERS = 1000000;  // one launch stays well inside the
 constexpr uint32_t PK_SF_COL = 256;  // TMEM columns after the 128 x 256 fp32 accumulator
 }  // namespace
 
-template <bool MX>
+// KIND: 0 BF16, 1 MXFP8, 2 per-tensor FP8
+template <int KIND>
 __global__ void __launch_bounds__(128, 1) tensor_peak_kernel(long long iters, int scale_refresh, int* status) {
+  constexpr bool MX = KIND == 1, Q8 = KIND != 0;
   extern __shared__ uint8_t pk_raw[];
   uint8_t* smem = pk_raw + ((1024u - (ptx::smem_u32(pk_raw) & 1023u)) & 1023u);
   __shared__ uint64_t done;
@@ -41,7 +43,7 @@ __global__ void __launch_bounds__(128, 1) tensor_peak_kernel(long long iters, in
     h ^= h >> 15;
     h *= 2246822519u;
     h ^= h >> 13;
-    w[i] = MX ? (h & 0xF7F7F7F7u) : ((h & 0x807F807Fu) | 0x3F003F00u);
+    w[i] = Q8 ? (h & 0xF7F7F7F7u) : ((h & 0x807F807Fu) | 0x3F003F00u);
   }
   for (int i = tid; i < PK_SF / 4; i += blockDim.x) w[(PK_A + PK_B) / 4 + i] = 0x7F7F7F7Fu;
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor-core reads
@@ -83,6 +85,10 @@ __global__ void __launch_bounds__(128, 1) tensor_peak_kernel(long long iters, in
         for (int k = 0; k < 4; ++k)
           ptx::tc_mma_mxf8(tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(128, 256, k, k), sfa, sfa + 4,
                            (it | k) != 0);
+      } else if (Q8) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          ptx::tc_mma_f8(tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_f8(128, 256), (it | k) != 0);
       } else {
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -100,14 +106,14 @@ __global__ void __launch_bounds__(128, 1) tensor_peak_kernel(long long iters, in
   }
 }
 
-double tensor_peak_flops(bool mx, int num_sms, long long iters) {
-  return static_cast<double>(num_sms) * static_cast<double>(iters) * 4.0 * 2.0 * 128.0 * 256.0 * (mx ? 32.0 : 16.0);
+double tensor_peak_flops(int kind, int num_sms, long long iters) {
+  return static_cast<double>(num_sms) * static_cast<double>(iters) * 4.0 * 2.0 * 128.0 * 256.0 * (kind ? 32.0 : 16.0);
 }
 
-cudaError_t launch_tensor_peak(bool mx, long long iters, int scale_refresh, int num_sms, int* status,
+cudaError_t launch_tensor_peak(int kind, long long iters, int scale_refresh, int num_sms, int* status,
                                cudaStream_t st) {
-  if (iters > PK_MAX_ITERS) return cudaErrorInvalidValue;
-  auto kern = mx ? tensor_peak_kernel<true> : tensor_peak_kernel<false>;
+  if (iters > PK_MAX_ITERS || kind < 0 || kind > 2) return cudaErrorInvalidValue;
+  auto kern = kind == 1 ? tensor_peak_kernel<1> : (kind == 2 ? tensor_peak_kernel<2> : tensor_peak_kernel<0>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PK_SMEM);
   if (e != cudaSuccess) return e;
   kern<<<num_sms, 128, PK_SMEM, st>>>(iters, scale_refresh, status);

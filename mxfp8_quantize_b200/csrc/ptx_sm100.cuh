@@ -191,6 +191,18 @@ __device__ __forceinline__ void tc_mma_mxf8(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T with 8-bit float inputs (per-tensor FP8: no block scales; the
+// tensor scales are applied to D afterwards), fp32 accumulate.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Each thread of the warp reads 32 consecutive 32-bit TMEM columns of its own lane.
 __device__ __forceinline__ void tmem_ld_32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -228,11 +240,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16(uint32_t M, uint32_t N) {
          | ((N >> 3) << 17)   // N / 8
          | ((M >> 4) << 24);  // M / 16
 }
-// Element formats of kind::mxf8f6f4 operands (instruction descriptor fields at bits 7-9 for A and
-// 10-12 for B); A and B may differ.
+// Element formats of kind::mxf8f6f4 / kind::f8f6f4 operands (instruction descriptor fields at bits
+// 7-9 for A and 10-12 for B); A and B may differ.
 constexpr uint32_t kFmtE4M3 = 0;
 constexpr uint32_t kFmtE5M2 = 1;
 __host__ __device__ constexpr uint32_t idesc_a_format(uint32_t fmt) { return (fmt & 7u) << 7; }
+// Instruction descriptor, kind::f8f6f4 with E4M3 A/B, fp32 D, both operands K-major (the same
+// field layout as kind::f16); OR in idesc_a_format for an A operand of another format.
+__host__ __device__ constexpr uint32_t idesc_f8(uint32_t M, uint32_t N) {
+  return (1u << 4)            // D format f32
+         | (0u << 7)          // A E4M3
+         | (0u << 10)         // B E4M3
+         | ((N >> 3) << 17)   // N / 8
+         | ((M >> 4) << 24);  // M / 16
+}
 // Instruction descriptor, kind::mxf8f6f4 with E4M3 A/B, E8M0 scales, K-major; the scale-factor
 // ids select which byte of each 32-bit TMEM scale cell an MMA reads.  OR in idesc_a_format for an
 // A operand of another format.

@@ -37,7 +37,7 @@ class MoEConfig:
     f: int          # expert ffn size (gate and up are f wide each)
     E: int          # experts
     k: int          # experts per token
-    precision: str  # "bf16" or "mxfp8"
+    precision: str  # "bf16", "mxfp8" or "fp8" (per-tensor)
     backward: bool  # whether the workload includes the backward pass
     w_std: Optional[float]  # None -> 1/sqrt(fan_in)
     routing: str    # "uniform" | "zipf" | "dirichlet"
@@ -67,6 +67,8 @@ CONFIGS = {
     "mixtral_bf16": MoEConfig("mixtral_bf16", 8192, 4096, 14336, 8, 2, "bf16", True, 0.02, "uniform", 2),
     # Same layer, MXFP8 forward+backward, weights quantised every step.
     "mixtral_mxfp8": MoEConfig("mixtral_mxfp8", 8192, 4096, 14336, 8, 2, "mxfp8", True, 0.02, "uniform", 3),
+    # Same layer with per-tensor FP8 operands (one scale per expert operand, current scaling).
+    "mixtral_fp8": MoEConfig("mixtral_fp8", 8192, 4096, 14336, 8, 2, "fp8", True, 0.02, "uniform", 3),
     # Long-sequence genomics-style layer: one sequence of 32768 tokens, Dirichlet-skewed routing.
     "longseq_mxfp8": MoEConfig("longseq_mxfp8", 32768, 4096, 14336, 8, 2, "mxfp8", True, 0.02, "dirichlet", 4),
 }

@@ -21,7 +21,7 @@ def lib():
 def test_header_declarations_are_exported(lib):
     header = open(os.path.join(ROOT, "include", "moemx.h")).read()
     names = set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(\w+)\s*\(", header, flags=re.M))
-    names = {n for n in names if n.startswith(("moe_", "mxfp8_"))}
+    names = {n for n in names if n.startswith(("moe_", "mxfp8_", "fp8_"))}
     assert names == set(moe.EXPORTS)
     for n in names:
         assert hasattr(lib, n), n
