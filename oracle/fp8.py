@@ -46,13 +46,18 @@ def amax(v) -> np.float32:
     return np.float32(np.max(np.abs(v))) if v.size else np.float32(0)
 
 
+def encode(v, s, fmt: str = "e4m3") -> np.ndarray:
+    """Codes of the values v (fp32-representable) under the tensor scale s (fp32)."""
+    v = np.asarray(v, dtype=np.float32)
+    prod = (v * np.float32(s)).astype(np.float32)          # fp32 product, rounded to nearest
+    enc = mx.e4m3_encode if fmt == "e4m3" else mx.e5m2_encode
+    return enc(prod.astype(np.float64))
+
+
 def quantize(v, fmt: str = "e4m3"):
     """Codes (uint8, the shape of v) and the fp32 scale of the tensor v."""
-    v = np.asarray(v, dtype=np.float32)
     s = scale(amax(v), fmt)
-    prod = (v * s).astype(np.float32)                      # fp32 product, rounded to nearest
-    enc = mx.e4m3_encode if fmt == "e4m3" else mx.e5m2_encode
-    return enc(prod.astype(np.float64)), np.float32(s)
+    return encode(v, s, fmt), np.float32(s)
 
 
 def dequantize(codes, s, fmt: str = "e4m3") -> np.ndarray:
