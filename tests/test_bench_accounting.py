@@ -44,3 +44,17 @@ def test_oracle_sample_is_shared_by_both_cpu_legs():
     import inspect
     src = inspect.getsource(bench.main)
     assert src.count("ORACLE_SAMPLE") >= 2
+
+
+def test_fp8_kernel_bytes():
+    """Per-tensor FP8: codes without scale bytes, the maxima passes read their tensor once, and the
+    quantisation of the bf16 a / dh rows reads them and writes codes both ways."""
+    cfg = workloads.CONFIGS["mixtral_fp8"]
+    n = cfg.E * 2 * cfg.f * cfg.d
+    assert bench.kernel_work(cfg, "quantize_w_gate_up") == ("hbm", n * 2 + 2 * n)
+    assert bench.kernel_work(cfg, "amax_w_gate_up") == ("hbm", n * 2)
+    assert bench.kernel_work(cfg, "amax_w_down") == ("hbm", cfg.E * cfg.d * cfg.f * 2)
+    assert bench.kernel_work(cfg, "quantize_a") == ("hbm", cfg.Tk * cfg.f * 4)
+    assert bench.kernel_work(cfg, "quantize_dh") == ("hbm", cfg.Tk * 2 * cfg.f * 4)
+    total = sum(bench.kernel_work(cfg, g)[1] for g in GEMMS)
+    assert total == 18.0 * cfg.Tk * cfg.d * cfg.f
