@@ -62,3 +62,32 @@ def test_product_path_has_no_cpu_fallback():
     assert "oracle" not in src.replace("oracle_", "")
     for f in os.listdir(os.path.join(ROOT, "mxfp8_quantize_b200", "csrc")):
         assert "oracle" not in open(os.path.join(ROOT, "mxfp8_quantize_b200", "csrc", f)).read()
+
+
+def test_fp8_sizes_and_layout(lib):
+    """Per-tensor FP8 (precision 2): codes without scale bytes, so its buffers are smaller than
+    MXFP8's; it saves h in bf16 only; the maxima have names in the saved buffer, the inference
+    workspace and the backward workspace, and every named part lies inside its buffer."""
+    T, d, f, E, k = 4096, 1024, 2048, 8, 2
+    mx, f8 = moe.sizes(T, d, f, E, k, "mxfp8", True), moe.sizes(T, d, f, E, k, "fp8", True)
+    assert 0 < f8["saved"] < mx["saved"]
+    assert f8["fwd_ws"] > 0 and f8["bwd_ws"] > 0
+    assert moe.sizes(T, d, f, E, k, "fp8", True, "mxfp8")["saved"] == 0
+    assert moe.sizes(T, d, f, E, k, "fp8", True, "recompute")["saved"] == 0
+    base = 1 << 40
+    for which, training, name, limit in ((0, 1, b"pt_amax", f8["saved"]),
+                                         (1, 0, b"pt_amax", moe.sizes(T, d, f, E, k, "fp8", False)["fwd_ws"]),
+                                         (2, 1, b"pt_amax", f8["bwd_ws"]),
+                                         (1, 1, b"a", f8["fwd_ws"]), (2, 1, b"dh", f8["bwd_ws"])):
+        p = lib.moe_buffer_address_ex(T, k, E, d, f, 2, training, 0, which, base, name)
+        assert p and (p - base) % 1024 == 0 and p - base < limit, (which, name)
+    # MXFP8-only parts do not exist in the FP8 layout
+    assert lib.moe_buffer_address_ex(T, k, E, d, f, 2, 1, 0, 1, base, b"w1_s") is None
+    assert lib.moe_buffer_address_ex(T, k, E, d, f, 2, 1, 0, 0, base, b"xT_s") is None
+
+
+def test_fp8_quantize_argument_checks(lib):
+    """Refused on the host before anything is enqueued: no context, no row-wise flag, an unknown
+    flag, rows or cols not multiples of 128."""
+    assert lib.fp8_quantize(None, None, 1, 128, 128, 1, None, None, None, None) == 1
+    assert lib.moe_tensor_peak_flops(None, 2, 10) == 0.0
