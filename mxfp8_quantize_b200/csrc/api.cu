@@ -1049,7 +1049,8 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     GemmArgs g2 = gemm_args(ctx);
     const bool ok2 = map_2d(&g2.tmap_a, D.q8 ? static_cast<const void*>(w.a_q) : w.a, D.q8, f, D.cap,
                             f * (D.q8 ? 1 : 2)) &&
-                     map_3d(&g2.tmap_b, w2_base, D.q8, f, d, E, f * (D.q8 ? 1 : 2), w2_stride, gemm_tile_n(EPI_STORE));
+                     map_3d(&g2.tmap_b, w2_base, D.q8, f, d, E, f * (D.q8 ? 1 : 2), w2_stride,
+                            ctx->fused_fwd ? gemm_tile_n(EPI_STORE) : gemm_b_box_rows(D.mx, EPI_STORE));
     if (!ok2) return MOE_ERR_CUDA;
     g2.kgrouped = 0;
     g2.E = E;
@@ -1327,7 +1328,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     const bool ok =
         map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(w.dyT_q) : w.dyT, D.q8, D.cap, d, D.cap * es) &&
         map_2d(&g.tmap_b, D.q8 ? static_cast<const void*>(s.aT_q) : s.aT, D.q8, D.cap, f, D.cap * es,
-               gemm_tile_n(EPI_STORE));
+               gemm_b_box_rows(D.mx, EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 1;
     g.E = E;
@@ -1352,7 +1353,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     GemmArgs g = gemm_args(ctx);
     const bool ok =
         map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(w.dh_q) : w.dh, D.q8, 2 * f, D.cap, 2 * f * es) &&
-        map_3d(&g.tmap_b, w1c, D.q8, 2 * f, d, E, 2 * f * es, 2 * f * d * es, gemm_tile_n(EPI_STORE));
+        map_3d(&g.tmap_b, w1c, D.q8, 2 * f, d, E, 2 * f * es, 2 * f * d * es, gemm_b_box_rows(D.mx, EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
@@ -1379,7 +1380,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     const bool ok =
         map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(w.dhT_q) : w.dhT, D.q8, D.cap, 2 * f, D.cap * es) &&
         map_2d(&g.tmap_b, D.q8 ? static_cast<const void*>(s.xT_q) : s.xT, D.q8, D.cap, d, D.cap * es,
-               gemm_tile_n(EPI_STORE));
+               gemm_b_box_rows(D.mx, EPI_STORE));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 1;
     g.E = E;

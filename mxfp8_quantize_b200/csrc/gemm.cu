@@ -27,6 +27,7 @@
 // Every wait is bounded: on expiry the kernel records MOE_ERR_TIMEOUT and all roles stop; copies
 // and MMAs already issued are waited for before TMEM is freed.
 #include <cuda_fp16.h>
+#include <algorithm>
 #include <cuda_fp8.h>
 
 #include "gemm.cuh"
@@ -43,8 +44,13 @@ constexpr uint32_t TMEM_COLS = 512;
 //   split the tile's columns); PASS columns per pass of the column-wise transpose buffer.
 //   LEAD warps before the epilogue warps: 4 (producer, MMA issuer, TMEM allocator, idle) or 2 (the
 //   producer's warp also allocates TMEM), the latter leaving more registers per thread.
-template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_, bool HTILE_ = false, int LEAD_ = 4>
+//   PAIR: two CTAs of a cluster compute one 256 x BN tile with tcgen05 cta_group::2 MMAs; each CTA
+//   loads its 128 rows of A, half of the tile's B rows and all of the tile's B scales, and keeps its
+//   128 rows of the accumulator (MXFP8 store and SwiGLU epilogues).
+template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_, bool HTILE_ = false, int LEAD_ = 4,
+          bool PAIR_ = false>
 struct Shape {
+  static constexpr bool PAIR = PAIR_;
   static constexpr int BN = BN_;
   static constexpr int NBUF = NBUF_;
   static constexpr int STAGES = STAGES_;
@@ -55,7 +61,7 @@ struct Shape {
   static constexpr int PASS = PASS_;
   static constexpr int PITCH = PASS + 1;  // odd pitch: conflict-free row writes and column reads
   static constexpr int A_BYTES = BM * 128;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = (PAIR ? BN / 2 : BN) * 128;  // this CTA's B rows
   static constexpr int SFB_BYTES = (BN / 128) * 512;
   static constexpr int OFF_B = A_BYTES;
   static constexpr int OFF_SFA = A_BYTES + B_BYTES;
@@ -72,8 +78,12 @@ struct Shape {
   static_assert(NBUF * BN + STAGES * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
   static_assert(SMEM_DYN + 6144 <= 232448, "shared memory budget");  // + the static SharedState
   static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0 && (LEAD == 4 || LEAD == 2), "thread layout");
+  static_assert(!PAIR || (NBUF == 1 && !HTILE && LEAD == 4), "pair instances: one accumulator, no h tile");
 };
 using ShapeStore = Shape<256, 1, 4, false, 8, 16>;    // plain bf16-store epilogues
+// MXFP8 store GEMMs on CTA pairs: 256 x 256 tiles, each CTA streaming 128 rows of A and 128 of B per
+// stage (two thirds of the single-CTA bytes per MMA), six stages deep
+using ShapeStorePair = Shape<256, 1, 6, false, 8, 16, false, 4, true>;
 using ShapeSwiglu = Shape<256, 1, 4, true, 16, 8>;    // gate_up + ScaledSwiGLU: one 32-column group per thread
 using ShapeDswiglu = Shape<128, 2, 4, true, 8, 16, true>;  // dgrad of down + dSwiGLU: epilogue overlaps the next tile
 using ShapeDswigluG = Shape<128, 2, 4, true, 8, 16, false>;  // ... reading the saved h from global memory (MXFP8 h)
@@ -98,21 +108,23 @@ struct SharedState {
 
 struct Tile {
   int e, mb, nb, nk;
-  int a_row;  // first row of A (M-grouped: token row; K-grouped: row of the M dimension)
+  int a_row;  // first row of A (M-grouped: token row; K-grouped: row of the M dimension); for a CTA
+              // pair the first row of the pair's 256-row tile
   int k0;     // first K coordinate (K-grouped: the expert's first token row)
   bool down;  // EPI_FUSED_FWD: a tile of the down GEMM
+  bool hi_ok; // CTA pair: the tile's second 128 rows exist (an expert may end after the first half)
 };
 
-// The i-th tile of this CTA: tiles are dealt out in rounds of gridDim.x, in boustrophedon order
-// (even rounds to CTAs 0, 1, ..., odd rounds in reverse), so that with the tile list sorted from
-// the most to the least work every CTA gets a similar total.
-__device__ __forceinline__ int tile_of(int i) {
-  const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
-  return i * G + ((i & 1) ? G - 1 - b : b);
-}
+// The i-th tile of this CTA (or CTA pair): tiles are dealt out in rounds of G workers, in
+// boustrophedon order (even rounds to workers 0, 1, ..., odd rounds in reverse), so that with the
+// tile list sorted from the most to the least work every worker gets a similar total.
+__device__ __forceinline__ int tile_of(int i, int G, int b) { return i * G + ((i & 1) ? G - 1 - b : b); }
 
-__device__ __forceinline__ void decode_tile(int t, const SharedState& s, const GemmArgs& g, bool mx, Tile& o) {
+// Rows of A per tile: 128, or 256 for a CTA pair.
+__device__ __forceinline__ void decode_tile(int t, const SharedState& s, const GemmArgs& g, bool mx, Tile& o,
+                                            int rows = BM) {
   o.down = false;
+  o.hi_ok = true;
   if (g.mblock_done && t >= s.total1) {  // fused forward: a down tile (experts in id order)
     const int t2 = t - s.total1;
     int lo = 0, hi = g.E;
@@ -142,16 +154,17 @@ __device__ __forceinline__ void decode_tile(int t, const SharedState& s, const G
   const int bk = mx ? 128 : 64;  // K elements per stage (128 bytes)
   o.e = e;
   if (!g.kgrouped) {
-    const int mt = P / BM;
+    const int mt = (P + rows - 1) / rows;
     o.nb = local / mt;
     o.mb = local - o.nb * mt;
-    o.a_row = s.poff[e] + o.mb * BM;
+    o.a_row = s.poff[e] + o.mb * rows;
+    o.hi_ok = o.mb * rows + BM < P;
     o.k0 = 0;
     o.nk = g.K / bk;
   } else {
     o.mb = local / g.n_tiles;
     o.nb = local - o.mb * g.n_tiles;
-    o.a_row = o.mb * BM;
+    o.a_row = o.mb * rows;
     o.k0 = s.poff[e];
     o.nk = P / bk;
   }
@@ -308,6 +321,11 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const bool K128 = MX || g.fp8;  // 8-bit operands: 128 K elements per 128-byte stage row
+  // CTA pair: this CTA's rank (rank 0 issues the MMAs), the tile walkers are the pairs
+  const uint32_t rank = S::PAIR ? ptx::cluster_ctarank() : 0u;
+  const int NW = S::PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int WID = S::PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  constexpr int TILE_ROWS = S::PAIR ? 2 * BM : BM;
 
   // ---- set-up: tile prefix over experts, barriers, TMEM
   if (threadIdx.x == 0) {
@@ -330,7 +348,8 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     for (int i = 0; i < g.E; ++i) {
       const int e = s.order[i];
       s.tile_prefix[i] = acc;
-      acc += g.kgrouped ? g.m_tiles * g.n_tiles : ((s.poff[e + 1] - s.poff[e]) / BM) * g.n_tiles;
+      acc += g.kgrouped ? (g.m_tiles * BM / TILE_ROWS) * g.n_tiles
+                        : ((s.poff[e + 1] - s.poff[e] + TILE_ROWS - 1) / TILE_ROWS) * g.n_tiles;
     }
     s.tile_prefix[g.E] = acc;
     s.total1 = acc;
@@ -351,7 +370,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     }
     for (int i = 0; i < S::NBUF; ++i) {
       ptx::mbar_init(&s.acc_full[i], 1);
-      ptx::mbar_init(&s.acc_empty[i], S::EPI_WARPS);
+      ptx::mbar_init(&s.acc_empty[i], S::EPI_WARPS * (S::PAIR ? 2 : 1));  // pair: both CTAs' epilogues
     }
     ptx::mbar_init(&s.drain, 1);
     ptx::mbar_init(&s.h_full, 1);
@@ -372,11 +391,19 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     if (S::HTILE) ptx::prefetch_tmap(&g.tmap_h);
   }
   if (warp == S::ALLOC_WARP) {
-    ptx::tmem_alloc(&s.tmem_base, TMEM_COLS);
-    ptx::tmem_relinquish();
+    if (S::PAIR) {
+      ptx::tmem_alloc_pair(&s.tmem_base, TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(&s.tmem_base, TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  if (S::PAIR)
+    ptx::cluster_sync();  // both CTAs' barriers initialised before any load or commit reaches them
+  else
+    __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const int total = s.total_tiles;
@@ -391,10 +418,11 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     uint32_t h_count = 0;
     bool h_issued = false;
     bool stalled = false;
-    const uint32_t tx = S::A_BYTES + S::B_BYTES + (MX ? 512 + S::SFB_BYTES : 0);
-    for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
+    // bytes per stage; for a CTA pair rank 0's barrier counts both CTAs' loads
+    const uint32_t tx = (S::A_BYTES + S::B_BYTES + (MX ? 512 + S::SFB_BYTES : 0)) * (S::PAIR ? 2 : 1);
+    for (int i = 0, t = tile_of(0, NW, WID); t < total && !*abort_flag; t = tile_of(++i, NW, WID)) {
       Tile tl;
-      decode_tile(t, s, g, K128, tl);
+      decode_tile(t, s, g, K128, tl, TILE_ROWS);
       const int bk = K128 ? 128 : 64;
       if (EPI == EPI_FUSED_FWD && tl.down) {
         // the tile's 128 rows of a are complete once every gate_up tile of its row block has released them
@@ -413,8 +441,27 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         }
         if (!ptx::mbar_wait(&s.empty[stage], phase ^ 1, abort_flag, lim)) break;
         uint8_t* st = smem + stage * S::STAGE_BYTES;
-        ptx::mbar_arrive_expect_tx(&s.full[stage], tx);
         const int kx = tl.k0 + kb * bk;
+        if (S::PAIR) {
+          // this CTA's 128 rows of A and half of the tile's B rows, all of its B scales; completion
+          // counted on rank 0's barrier, which expects both CTAs' bytes
+          if (rank == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], tx);
+          const int32_t arow = tl.a_row + static_cast<int32_t>(rank) * BM;
+          const int32_t brow = tl.nb * BN + static_cast<int32_t>(rank) * (BN / 2);
+          ptx::tma_load_2d_pair(st, map_a, kx, arow, &s.full[stage]);
+          if (!g.kgrouped)
+            ptx::tma_load_3d_pair(st + S::OFF_B, map_b, kx, brow, tl.e, &s.full[stage]);
+          else
+            ptx::tma_load_2d_pair(st + S::OFF_B, map_b, kx, brow, &s.full[stage]);
+          if (MX) {
+            const int32_t kq = kx / 128;
+            const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * sfb_rows;
+            ptx::tma_load_3d_pair(st + S::OFF_SFA, map_sfa, 0, kq, arow / 128, &s.full[stage]);
+            ptx::tma_load_3d_pair(st + S::OFF_SFB, map_sfb, 0, kq,
+                                  static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128), &s.full[stage]);
+          }
+        } else {
+        ptx::mbar_arrive_expect_tx(&s.full[stage], tx);
         ptx::tma_load_2d(st, map_a, kx, tl.a_row, &s.full[stage]);
         if (!g.kgrouped && g.gate_up_half && !tl.down) {
           // bf16 gate_up: BN/2 gate rows then the matching BN/2 up rows of expert e
@@ -432,6 +479,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           ptx::tma_load_3d(st + S::OFF_SFA, map_sfa, 0, kq, tl.a_row / 128, &s.full[stage]);
           ptx::tma_load_3d(st + S::OFF_SFB, map_sfb, 0, kq,
                       static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128), &s.full[stage]);
+        }
         }
         issued_mask |= 1u << stage;
         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -460,12 +508,18 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       volatile int never = 0;
       ptx::mbar_wait(&s.h_full, (h_count - 1) & 1, &never, lim);
     }
-    // wait for the loads still in flight (only possible after an abort)
+    // wait for the loads still in flight (only possible after an abort; a pair's rank 1 has no
+    // barrier of its own to wait on: rank 0's waits and the final cluster barrier cover it)
     for (int i = 0; i < S::STAGES; ++i)
-      if (issued_mask & (1u << i)) {
+      if ((!S::PAIR || rank == 0) && (issued_mask & (1u << i))) {
         volatile int never = 0;
         ptx::mbar_wait(&s.full[i], (last_parity >> i) & 1u, &never, lim);
       }
+  } else if (S::PAIR && rank != 0 && warp == 1 && lane == 0) {
+    // pair rank 1: rank 0 issues the MMAs for both CTAs; its final commit arrives here once they have
+    // all completed, before this CTA's TMEM is freed
+    volatile int never = 0;
+    ptx::mbar_wait(&s.drain, 0, &never, lim);
   } else if (warp == 1 && lane == 0) {
     // ================= MMA issuer
     int stage = 0;
@@ -480,9 +534,9 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
     const uint64_t sfadesc0 = ptx::smem_desc(smem0 + S::OFF_SFA, 0, 128, ptx::kSwizzleNone);
     const uint64_t sfbdesc0 = ptx::smem_desc(smem0 + S::OFF_SFB, 0, 128, ptx::kSwizzleNone);
     const uint32_t a_fmt = ptx::idesc_a_format(g.a_e5m2 ? ptx::kFmtE5M2 : ptx::kFmtE4M3);  // A's element format
-    for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
+    for (int i = 0, t = tile_of(0, NW, WID); t < total && !*abort_flag; t = tile_of(++i, NW, WID)) {
       Tile tl;
-      decode_tile(t, s, g, K128, tl);
+      decode_tile(t, s, g, K128, tl, TILE_ROWS);
       if (tl.nk == 0) continue;
       const int buf = S::NBUF == 2 ? (local & 1) : 0;
       const uint32_t acc_par = static_cast<uint32_t>((S::NBUF == 2 ? (local >> 1) : local) & 1);
@@ -499,7 +553,18 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         const uint64_t soff = static_cast<uint64_t>(stage * (S::STAGE_BYTES >> 4));
         const uint64_t adesc = adesc0 + soff;
         const uint64_t bdesc = bdesc0 + soff;
-        if (MX) {
+        if (S::PAIR) {
+          // both CTAs' scale tiles into their own TMEM, then M = 256 MMAs over both CTAs' operands
+          const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * stage;
+          const uint32_t sfb_t = sfa_t + 4;
+          ptx::tc_cp_32x128b_warpx4_pair(sfa_t, sfadesc0 + soff);
+#pragma unroll
+          for (int i = 0; i < BN / 128; ++i) ptx::tc_cp_32x128b_warpx4_pair(sfb_t + 4 * i, sfbdesc0 + soff + 32 * i);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            ptx::tc_mma_mxf8_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(2 * BM, BN, k, k) | a_fmt,
+                                  sfa_t, sfb_t, (kb | k) != 0);
+        } else if (MX) {
           const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * stage;
           const uint32_t sfb_t = sfa_t + 4;
           ptx::tc_cp_32x128b_warpx4(sfa_t, sfadesc0 + soff);
@@ -518,7 +583,10 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           for (int k = 0; k < 4; ++k)
             ptx::tc_mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_bf16(BM, BN), (kb | k) != 0);
         }
-        ptx::tc_commit(&s.empty[stage]);
+        if (S::PAIR)
+          ptx::tc_commit_pair(&s.empty[stage]);  // frees the stage in both CTAs
+        else
+          ptx::tc_commit(&s.empty[stage]);
         issued_any = true;
         if (++stage == S::STAGES) {
           stage = 0;
@@ -526,10 +594,17 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         }
       }
       if (!ok) break;
-      ptx::tc_commit(&s.acc_full[buf]);
+      if (S::PAIR)
+        ptx::tc_commit_pair(&s.acc_full[buf]);  // both CTAs' epilogues
+      else
+        ptx::tc_commit(&s.acc_full[buf]);
       ++local;
     }
-    if (issued_any) {  // all MMAs of this CTA complete before TMEM can be released
+    if (S::PAIR) {  // always, so that rank 1's wait for it ends
+      ptx::tc_commit_pair(&s.drain);
+      volatile int never = 0;
+      ptx::mbar_wait(&s.drain, 0, &never, lim);
+    } else if (issued_any) {  // all MMAs of this CTA complete before TMEM can be released
       ptx::tc_commit(&s.drain);
       volatile int never = 0;
       ptx::mbar_wait(&s.drain, 0, &never, lim);
@@ -543,6 +618,14 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
                                                 (warp - S::LEAD) * S::STAGING_PER_WARP);
     const EpiArgs& ep = g.epi;
     int local = 0;
+    // hand the accumulator back to the MMA issuer (a pair's issuer is rank 0: its barrier counts the
+    // epilogue warps of both CTAs)
+    auto release_acc = [&](int b) {
+      if (S::PAIR)
+        ptx::mbar_arrive_leader(&s.acc_empty[b]);
+      else
+        ptx::mbar_arrive(&s.acc_empty[b]);
+    };
     // per-tensor FP8: this warp's largest magnitude written for expert amax_e so far (bf16 bits),
     // added to ep.amax_out[amax_e] when the expert changes and at the end
     uint32_t amax_run = 0;
@@ -553,10 +636,10 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       const uint32_t m = __reduce_max_sync(mask, amax_run);
       if (lane == __ffs(mask) - 1 && m) atomicMax(ep.amax_out + amax_e, m << 16);
     };
-    for (int i = 0, t = tile_of(0); t < total && !*abort_flag; t = tile_of(++i)) {
+    for (int i = 0, t = tile_of(0, NW, WID); t < total && !*abort_flag; t = tile_of(++i, NW, WID)) {
       Tile tl;
-      decode_tile(t, s, g, K128, tl);
-      const int64_t row_w = tl.a_row + 32 * q;  // first row of this warp
+      decode_tile(t, s, g, K128, tl, TILE_ROWS);
+      const int64_t row_w = tl.a_row + (S::PAIR ? static_cast<int>(rank) * BM : 0) + 32 * q;  // first row of this warp
       const int64_t row = row_w + lane;
       // per-tensor FP8: the accumulator times 1/s_a * 1/s_b of the tile's expert
       float fac = 1.f;
@@ -598,7 +681,8 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         }
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
+        if (lane == 0) release_acc(buf);
+        if (S::PAIR && rank != 0 && !tl.hi_ok) continue;  // the expert ends in the pair tile's first half
         bf16* out = g.kgrouped ? static_cast<bf16*>(const_cast<void*>(ep.out_ptrs.p[tl.e])) : ep.out;
         bf16* orow = out + row * ep.ldo + static_cast<int64_t>(tl.nb) * BN + CPT * ch;
         if ((reinterpret_cast<uintptr_t>(out) & 31u) == 0 && (ep.ldo & 15) == 0) {  // whole 32-byte sectors
@@ -636,7 +720,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           if (cc == G - 1) {
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
+            if (lane == 0) release_acc(buf);
           }
           if (ep.h_q) {  // saved as MXFP8: 32 codes and one scale per 32 gate (and up) values
             const uint32_t sbg = quant32_store(gv, ep.h_q + row * 2 * f + j, ep.scale_floor, 0);
@@ -753,7 +837,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           if (cc == G - 1) {
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&s.acc_empty[buf]);
+            if (lane == 0) release_acc(buf);
           }
           float dg[32], du[32];
 #pragma unroll
@@ -826,9 +910,13 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
 
   __syncthreads();
   if (threadIdx.x == 0 && s.abort_flag) atomicOr(g.status, kStatusTimeout);
+  if (S::PAIR) ptx::cluster_sync();  // no arrival from the other CTA can still be on its way here
   if (warp == S::ALLOC_WARP) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, TMEM_COLS);
+    if (S::PAIR)
+      ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
+    else
+      ptx::tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -838,10 +926,34 @@ cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
   auto kern = grouped_gemm_kernel<MX, EPI, S>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_DYN);
   if (e != cudaSuccess) return e;
+  if (S::PAIR) {
+    // clusters of two CTAs, as many pairs as can be resident at once (one CTA per SM)
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+    cfg.blockDim = dim3(S::NUM_THREADS);
+    cfg.dynamicSmemBytes = S::SMEM_DYN;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min(clusters, num_sms / 2)));
+    return cudaLaunchKernelEx(&cfg, kern, args);
+  }
   kern<<<num_sms, S::NUM_THREADS, S::SMEM_DYN, st>>>(args);
   return cudaGetLastError();
 }
 }  // namespace
+
+// Rows of B one CTA loads per stage (its tensor-map box): the tile's N, or half of it for CTA pairs.
+int gemm_b_box_rows(bool mx, int epi) { return (mx && epi == EPI_STORE) ? ShapeStorePair::BN / 2 : gemm_tile_n(epi); }
 
 int gemm_tile_n(int epi) {
   return epi == EPI_STORE ? ShapeStore::BN
@@ -852,7 +964,7 @@ int gemm_dswiglu_parts() { return ShapeDswiglu::EPI_WARPS / 4; }
 
 cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_sms, cudaStream_t st) {
   if (mx) {
-    if (epi == EPI_STORE) return launch_t<true, EPI_STORE, ShapeStore>(args, num_sms, st);
+    if (epi == EPI_STORE) return launch_t<true, EPI_STORE, ShapeStorePair>(args, num_sms, st);
     if (epi == EPI_SWIGLU) return launch_t<true, EPI_SWIGLU, ShapeSwiglu>(args, num_sms, st);
     if (epi == EPI_FUSED_FWD) return launch_t<true, EPI_FUSED_FWD, ShapeSwiglu>(args, num_sms, st);
     if (args.epi.h_q) return launch_t<true, EPI_DSWIGLU, ShapeDswigluG>(args, num_sms, st);

@@ -90,6 +90,9 @@ struct GemmArgs {
 
 // Output tile width (N) of the kernel used for an epilogue kind.
 int gemm_tile_n(int epi);
+// Rows of B per tensor-map box of the kernel used for an epilogue kind (half the tile's N for the
+// CTA-pair instances).
+int gemm_b_box_rows(bool mx, int epi);
 // Partial sums of the probability gradient the dSwiGLU epilogue writes per output tile and row.
 int gemm_dswiglu_parts();
 
