@@ -1008,7 +1008,8 @@ moe_status_t moe_grouped_mlp_fwd(moe_ctx_t ctx, const void* x, const int32_t* to
     const bool ok = map_2d(&g.tmap_a, D.q8 ? static_cast<const void*>(x_q) : x_perm, D.q8, d, D.cap,
                            d * (D.q8 ? 1 : 2)) &&
                     map_3d(&g.tmap_b, w1_base, D.q8, d, 2 * f, E, d * (D.q8 ? 1 : 2), w1_stride,
-                           D.mx ? gemm_tile_n(EPI_SWIGLU) : gemm_tile_n(EPI_SWIGLU) / 2);
+                           !D.mx ? gemm_tile_n(EPI_SWIGLU) / 2
+                                 : (ctx->fused_fwd ? gemm_tile_n(EPI_SWIGLU) : gemm_b_box_rows(true, EPI_SWIGLU)));
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;
@@ -1185,7 +1186,7 @@ moe_status_t moe_grouped_mlp_bwd(moe_ctx_t ctx, const void* dy, const void* save
     const bool ok = map_2d(&g.tmap_a, D.mx ? static_cast<const void*>(s.xr_q) : s.xr, D.mx, d, D.cap,
                            d * (D.mx ? 1 : 2)) &&
                     map_3d(&g.tmap_b, w1_base, D.mx, d, 2 * f, E, d * (D.mx ? 1 : 2), w1_stride,
-                           D.mx ? gemm_tile_n(EPI_SWIGLU) : gemm_tile_n(EPI_SWIGLU) / 2);
+                           D.mx ? gemm_b_box_rows(true, EPI_SWIGLU) : gemm_tile_n(EPI_SWIGLU) / 2);
     if (!ok) return MOE_ERR_CUDA;
     g.kgrouped = 0;
     g.E = E;

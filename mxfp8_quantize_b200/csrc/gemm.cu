@@ -47,10 +47,13 @@ constexpr uint32_t TMEM_COLS = 512;
 //   PAIR: two CTAs of a cluster compute one 256 x BN tile with tcgen05 cta_group::2 MMAs; each CTA
 //   loads its 128 rows of A, half of the tile's B rows and all of the tile's B scales, and keeps its
 //   128 rows of the accumulator (MXFP8 store and SwiGLU epilogues).
+//   KSUB: 128-byte K blocks per pipeline stage (more than one halves the barrier round trips per
+//   MMA; CTA-pair instances only).
 template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_, bool HTILE_ = false, int LEAD_ = 4,
-          bool PAIR_ = false>
+          bool PAIR_ = false, int KSUB_ = 1>
 struct Shape {
   static constexpr bool PAIR = PAIR_;
+  static constexpr int KSUB = KSUB_;
   static constexpr int BN = BN_;
   static constexpr int NBUF = NBUF_;
   static constexpr int STAGES = STAGES_;
@@ -66,7 +69,8 @@ struct Shape {
   static constexpr int OFF_B = A_BYTES;
   static constexpr int OFF_SFA = A_BYTES + B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + 512;
-  static constexpr int STAGE_BYTES = (OFF_SFB + SFB_BYTES + 1023) / 1024 * 1024;
+  static constexpr int BLOCK_BYTES = (OFF_SFB + SFB_BYTES + 1023) / 1024 * 1024;  // one K block
+  static constexpr int STAGE_BYTES = KSUB * BLOCK_BYTES;
   static constexpr int SF_COLS = 4 + 4 * (BN / 128);
   static constexpr uint32_t SF_TMEM_COL = NBUF * BN;
   static constexpr int STAGING_PER_WARP = STAGING_ ? (32 * PITCH * 4 + 15) / 16 * 16 : 0;
@@ -75,7 +79,8 @@ struct Shape {
   static constexpr int OFF_H = STAGES * STAGE_BYTES;
   static constexpr int OFF_STAGING = OFF_H + H_BYTES;
   static constexpr int SMEM_DYN = OFF_STAGING + EPI_WARPS * STAGING_PER_WARP + 1024;
-  static_assert(NBUF * BN + STAGES * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(NBUF * BN + STAGES * KSUB * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
+  static_assert(KSUB == 1 || PAIR, "several K blocks per stage: CTA-pair instances only");
   static_assert(SMEM_DYN + 6144 <= 232448, "shared memory budget");  // + the static SharedState
   static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0 && (LEAD == 4 || LEAD == 2), "thread layout");
   static_assert(!PAIR || (NBUF == 1 && !HTILE && LEAD == 4), "pair instances: one accumulator, no h tile");
@@ -83,7 +88,10 @@ struct Shape {
 using ShapeStore = Shape<256, 1, 4, false, 8, 16>;    // plain bf16-store epilogues
 // MXFP8 store GEMMs on CTA pairs: 256 x 256 tiles, each CTA streaming 128 rows of A and 128 of B per
 // stage (two thirds of the single-CTA bytes per MMA), six stages deep
-using ShapeStorePair = Shape<256, 1, 6, false, 8, 16, false, 4, true>;
+// (stages of two 128-byte K blocks each: one barrier round trip per two blocks)
+using ShapeStorePair = Shape<256, 1, 3, false, 8, 16, false, 4, true, 2>;
+// (the gate_up + ScaledSwiGLU kernel stays on single CTAs: on pairs each tile waits for the slower
+// of two heavy epilogues, and it measured 5% slower)
 using ShapeSwiglu = Shape<256, 1, 4, true, 16, 8>;    // gate_up + ScaledSwiGLU: one 32-column group per thread
 using ShapeDswiglu = Shape<128, 2, 4, true, 8, 16, true>;  // dgrad of down + dSwiGLU: epilogue overlaps the next tile
 using ShapeDswigluG = Shape<128, 2, 4, true, 8, 16, false>;  // ... reading the saved h from global memory (MXFP8 h)
@@ -434,8 +442,8 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       const CUtensorMap* map_sfa = tl.down ? &g.tmap_sfa2 : &g.tmap_sfa;
       const CUtensorMap* map_sfb = tl.down ? &g.tmap_sfb2 : &g.tmap_sfb;
       const int64_t sfb_rows = tl.down ? g.sfb_expert_rows2 : g.sfb_expert_rows;
-      for (int kb = 0; kb < tl.nk; ++kb) {
-        if (g.stall_flag && !stalled && kb == min(2, tl.nk - 1)) {  // test hook: a wait that can only expire
+      for (int kb = 0; kb < tl.nk; kb += S::KSUB) {
+        if (g.stall_flag && !stalled && kb + S::KSUB > min(2, tl.nk - 1)) {  // test hook: a wait that can only expire
           stalled = true;
           if (!ptx::wait_flag(g.stall_flag, abort_flag, g.stall_limit)) break;
         }
@@ -443,22 +451,28 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         uint8_t* st = smem + stage * S::STAGE_BYTES;
         const int kx = tl.k0 + kb * bk;
         if (S::PAIR) {
-          // this CTA's 128 rows of A and half of the tile's B rows, all of its B scales; completion
-          // counted on rank 0's barrier, which expects both CTAs' bytes
-          if (rank == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], tx);
+          // this CTA's 128 rows of A and half of the tile's B rows, all of its B scales, for the stage's
+          // K blocks; completion counted on rank 0's barrier, which expects both CTAs' bytes
+          const int nsub = min(S::KSUB, tl.nk - kb);
+          if (rank == 0) ptx::mbar_arrive_expect_tx(&s.full[stage], tx * nsub);
           const int32_t arow = tl.a_row + static_cast<int32_t>(rank) * BM;
           const int32_t brow = tl.nb * BN + static_cast<int32_t>(rank) * (BN / 2);
-          ptx::tma_load_2d_pair(st, map_a, kx, arow, &s.full[stage]);
-          if (!g.kgrouped)
-            ptx::tma_load_3d_pair(st + S::OFF_B, map_b, kx, brow, tl.e, &s.full[stage]);
-          else
-            ptx::tma_load_2d_pair(st + S::OFF_B, map_b, kx, brow, &s.full[stage]);
-          if (MX) {
-            const int32_t kq = kx / 128;
-            const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * sfb_rows;
-            ptx::tma_load_3d_pair(st + S::OFF_SFA, map_sfa, 0, kq, arow / 128, &s.full[stage]);
-            ptx::tma_load_3d_pair(st + S::OFF_SFB, map_sfb, 0, kq,
-                                  static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128), &s.full[stage]);
+          for (int j = 0; j < nsub; ++j) {
+            uint8_t* blk = st + j * S::BLOCK_BYTES;
+            const int kxj = kx + j * bk;
+            ptx::tma_load_2d_pair(blk, map_a, kxj, arow, &s.full[stage]);
+            if (!g.kgrouped)
+              ptx::tma_load_3d_pair(blk + S::OFF_B, map_b, kxj, brow, tl.e, &s.full[stage]);
+            else
+              ptx::tma_load_2d_pair(blk + S::OFF_B, map_b, kxj, brow, &s.full[stage]);
+            if (MX) {
+              const int32_t kq = kxj / 128;
+              const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * sfb_rows;
+              ptx::tma_load_3d_pair(blk + S::OFF_SFA, map_sfa, 0, kq, arow / 128, &s.full[stage]);
+              ptx::tma_load_3d_pair(blk + S::OFF_SFB, map_sfb, 0, kq,
+                                    static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128),
+                                    &s.full[stage]);
+            }
           }
         } else {
         ptx::mbar_arrive_expect_tx(&s.full[stage], tx);
@@ -544,7 +558,7 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
       ptx::tc_fence_after();
       const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * BN);
       bool ok = true;
-      for (int kb = 0; kb < tl.nk; ++kb) {
+      for (int kb = 0; kb < tl.nk; kb += S::KSUB) {
         if (!ptx::mbar_wait(&s.full[stage], phase, abort_flag, lim)) {
           ok = false;
           break;
@@ -554,16 +568,21 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         const uint64_t adesc = adesc0 + soff;
         const uint64_t bdesc = bdesc0 + soff;
         if (S::PAIR) {
-          // both CTAs' scale tiles into their own TMEM, then M = 256 MMAs over both CTAs' operands
-          const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * stage;
-          const uint32_t sfb_t = sfa_t + 4;
-          ptx::tc_cp_32x128b_warpx4_pair(sfa_t, sfadesc0 + soff);
+          // per K block of the stage: both CTAs' scale tiles into their own TMEM, then M = 256 MMAs
+          // over both CTAs' operands
+          const int nsub = min(S::KSUB, tl.nk - kb);
+          for (int j = 0; j < nsub; ++j) {
+            const uint64_t boff = soff + static_cast<uint64_t>(j * (S::BLOCK_BYTES >> 4));
+            const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * (stage * S::KSUB + j);
+            const uint32_t sfb_t = sfa_t + 4;
+            ptx::tc_cp_32x128b_warpx4_pair(sfa_t, sfadesc0 + boff);
 #pragma unroll
-          for (int i = 0; i < BN / 128; ++i) ptx::tc_cp_32x128b_warpx4_pair(sfb_t + 4 * i, sfbdesc0 + soff + 32 * i);
+            for (int i = 0; i < BN / 128; ++i) ptx::tc_cp_32x128b_warpx4_pair(sfb_t + 4 * i, sfbdesc0 + boff + 32 * i);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ptx::tc_mma_mxf8_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(2 * BM, BN, k, k) | a_fmt,
-                                  sfa_t, sfb_t, (kb | k) != 0);
+            for (int k = 0; k < 4; ++k)
+              ptx::tc_mma_mxf8_pair(d_tmem, adesc0 + boff + 2 * k, bdesc0 + boff + 2 * k,
+                                    ptx::idesc_mxf8(2 * BM, BN, k, k) | a_fmt, sfa_t, sfb_t, ((kb + j) | k) != 0);
+          }
         } else if (MX) {
           const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * stage;
           const uint32_t sfb_t = sfa_t + 4;
@@ -699,9 +718,16 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
         // tile = BN/2 output columns; accumulator columns [0,BN/2) gate, [BN/2,BN) up
         constexpr int OPT = BN / 2 / NPART;  // output columns per thread
         constexpr int G = OPT / 32;          // groups of 32 output columns per thread
+        if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
+        if (S::PAIR && rank != 0 && !tl.hi_ok) {  // the expert ends in the pair tile's first half
+          ptx::tc_fence_after();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) release_acc(buf);
+          continue;
+        }
         const float p = ep.p_perm[row];
         const int64_t f = ep.f;
-        if (!ptx::mbar_wait(&s.acc_full[buf], acc_par, abort_flag, lim)) break;
         ptx::tc_fence_after();
         const uint32_t t_lane = tmem + static_cast<uint32_t>(buf * BN) + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
@@ -953,7 +979,10 @@ cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
 }  // namespace
 
 // Rows of B one CTA loads per stage (its tensor-map box): the tile's N, or half of it for CTA pairs.
-int gemm_b_box_rows(bool mx, int epi) { return (mx && epi == EPI_STORE) ? ShapeStorePair::BN / 2 : gemm_tile_n(epi); }
+int gemm_b_box_rows(bool mx, int epi) {
+  if (mx && epi == EPI_STORE) return ShapeStorePair::BN / 2;
+  return gemm_tile_n(epi);
+}
 
 int gemm_tile_n(int epi) {
   return epi == EPI_STORE ? ShapeStore::BN
