@@ -48,7 +48,7 @@ constexpr uint32_t TMEM_COLS = 512;
 //   loads its 128 rows of A, half of the tile's B rows and all of the tile's B scales, and keeps its
 //   128 rows of the accumulator (MXFP8 store and SwiGLU epilogues).
 //   KSUB: 128-byte K blocks per pipeline stage (more than one halves the barrier round trips per
-//   MMA; CTA-pair instances only).
+//   MMA).
 template <int BN_, int NBUF_, int STAGES_, bool STAGING_, int EPI_WARPS_, int PASS_, bool HTILE_ = false, int LEAD_ = 4,
           bool PAIR_ = false, int KSUB_ = 1>
 struct Shape {
@@ -80,7 +80,6 @@ struct Shape {
   static constexpr int OFF_STAGING = OFF_H + H_BYTES;
   static constexpr int SMEM_DYN = OFF_STAGING + EPI_WARPS * STAGING_PER_WARP + 1024;
   static_assert(NBUF * BN + STAGES * KSUB * SF_COLS <= (int)TMEM_COLS, "TMEM budget");
-  static_assert(KSUB == 1 || PAIR, "several K blocks per stage: CTA-pair instances only");
   static_assert(SMEM_DYN + 6144 <= 232448, "shared memory budget");  // + the static SharedState
   static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0 && (LEAD == 4 || LEAD == 2), "thread layout");
   static_assert(!PAIR || (NBUF == 1 && !HTILE && LEAD == 4), "pair instances: one accumulator, no h tile");
@@ -93,7 +92,9 @@ using ShapeStorePair = Shape<256, 1, 3, false, 8, 16, false, 4, true, 2>;
 // (the gate_up + ScaledSwiGLU kernel stays on single CTAs: on pairs each tile waits for the slower
 // of two heavy epilogues, and it measured 5% slower)
 using ShapeSwiglu = Shape<256, 1, 4, true, 16, 8>;    // gate_up + ScaledSwiGLU: one 32-column group per thread
-using ShapeDswiglu = Shape<128, 2, 4, true, 8, 16, true>;  // dgrad of down + dSwiGLU: epilogue overlaps the next tile
+// dgrad of down + dSwiGLU: two accumulators, so the epilogue overlaps the next tile; stages of two K
+// blocks (one barrier round trip per two blocks)
+using ShapeDswiglu = Shape<128, 2, 2, true, 8, 16, true, 4, false, 2>;
 using ShapeDswigluG = Shape<128, 2, 4, true, 8, 16, false>;  // ... reading the saved h from global memory (MXFP8 h)
 
 struct SharedState {
@@ -475,25 +476,30 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             }
           }
         } else {
-        ptx::mbar_arrive_expect_tx(&s.full[stage], tx);
-        ptx::tma_load_2d(st, map_a, kx, tl.a_row, &s.full[stage]);
-        if (!g.kgrouped && g.gate_up_half && !tl.down) {
-          // bf16 gate_up: BN/2 gate rows then the matching BN/2 up rows of expert e
-          ptx::tma_load_3d(st + S::OFF_B, map_b, kx, tl.nb * (BN / 2), tl.e, &s.full[stage]);
-          ptx::tma_load_3d(st + S::OFF_B + S::B_BYTES / 2, map_b, kx, g.gate_up_half + tl.nb * (BN / 2), tl.e,
-                      &s.full[stage]);
-        } else if (!g.kgrouped) {  // one box of BN rows
-          ptx::tma_load_3d(st + S::OFF_B, map_b, kx, tl.nb * BN, tl.e, &s.full[stage]);
-        } else {
-          ptx::tma_load_2d(st + S::OFF_B, map_b, kx, tl.nb * BN, &s.full[stage]);
-        }
-        if (MX) {  // this step's scale tiles: one of A, BN/128 consecutive ones of B
-          const int32_t kq = kx / 128;
-          const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * sfb_rows;
-          ptx::tma_load_3d(st + S::OFF_SFA, map_sfa, 0, kq, tl.a_row / 128, &s.full[stage]);
-          ptx::tma_load_3d(st + S::OFF_SFB, map_sfb, 0, kq,
-                      static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128), &s.full[stage]);
-        }
+          const int nsub = min(S::KSUB, tl.nk - kb);
+          ptx::mbar_arrive_expect_tx(&s.full[stage], tx * nsub);
+          for (int j = 0; j < nsub; ++j) {
+            uint8_t* blk = st + j * S::BLOCK_BYTES;
+            const int kxj = kx + j * bk;
+            ptx::tma_load_2d(blk, map_a, kxj, tl.a_row, &s.full[stage]);
+            if (!g.kgrouped && g.gate_up_half && !tl.down) {
+              // bf16 gate_up: BN/2 gate rows then the matching BN/2 up rows of expert e
+              ptx::tma_load_3d(blk + S::OFF_B, map_b, kxj, tl.nb * (BN / 2), tl.e, &s.full[stage]);
+              ptx::tma_load_3d(blk + S::OFF_B + S::B_BYTES / 2, map_b, kxj, g.gate_up_half + tl.nb * (BN / 2), tl.e,
+                               &s.full[stage]);
+            } else if (!g.kgrouped) {  // one box of BN rows
+              ptx::tma_load_3d(blk + S::OFF_B, map_b, kxj, tl.nb * BN, tl.e, &s.full[stage]);
+            } else {
+              ptx::tma_load_2d(blk + S::OFF_B, map_b, kxj, tl.nb * BN, &s.full[stage]);
+            }
+            if (MX) {  // this block's scale tiles: one of A, BN/128 consecutive ones of B
+              const int32_t kq = kxj / 128;
+              const int64_t eb = g.kgrouped ? 0 : static_cast<int64_t>(tl.e) * sfb_rows;
+              ptx::tma_load_3d(blk + S::OFF_SFA, map_sfa, 0, kq, tl.a_row / 128, &s.full[stage]);
+              ptx::tma_load_3d(blk + S::OFF_SFB, map_sfb, 0, kq,
+                               static_cast<int32_t>((eb + static_cast<int64_t>(tl.nb) * BN) / 128), &s.full[stage]);
+            }
+          }
         }
         issued_mask |= 1u << stage;
         last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -583,24 +589,33 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
               ptx::tc_mma_mxf8_pair(d_tmem, adesc0 + boff + 2 * k, bdesc0 + boff + 2 * k,
                                     ptx::idesc_mxf8(2 * BM, BN, k, k) | a_fmt, sfa_t, sfb_t, ((kb + j) | k) != 0);
           }
-        } else if (MX) {
-          const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * stage;
-          const uint32_t sfb_t = sfa_t + 4;
-          ptx::tc_cp_32x128b_warpx4(sfa_t, sfadesc0 + soff);
-#pragma unroll
-          for (int i = 0; i < BN / 128; ++i) ptx::tc_cp_32x128b_warpx4(sfb_t + 4 * i, sfbdesc0 + soff + 32 * i);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ptx::tc_mma_mxf8(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_mxf8(BM, BN, k, k) | a_fmt, sfa_t,
-                             sfb_t, (kb | k) != 0);
-        } else if (g.fp8) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ptx::tc_mma_f8(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_f8(BM, BN) | a_fmt, (kb | k) != 0);
         } else {
+          const int nsub = min(S::KSUB, tl.nk - kb);
+          for (int j = 0; j < nsub; ++j) {
+            const uint64_t boff = static_cast<uint64_t>(j * (S::BLOCK_BYTES >> 4));
+            const uint32_t acc = ((kb + j) != 0) ? 1u : 0u;  // the tile's first block overwrites D
+            if (MX) {
+              const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * (stage * S::KSUB + j);
+              const uint32_t sfb_t = sfa_t + 4;
+              ptx::tc_cp_32x128b_warpx4(sfa_t, sfadesc0 + soff + boff);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ptx::tc_mma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, ptx::idesc_bf16(BM, BN), (kb | k) != 0);
+              for (int i = 0; i < BN / 128; ++i)
+                ptx::tc_cp_32x128b_warpx4(sfb_t + 4 * i, sfbdesc0 + soff + boff + 32 * i);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                ptx::tc_mma_mxf8(d_tmem, adesc + boff + 2 * k, bdesc + boff + 2 * k,
+                                 ptx::idesc_mxf8(BM, BN, k, k) | a_fmt, sfa_t, sfb_t, acc | k);
+            } else if (g.fp8) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                ptx::tc_mma_f8(d_tmem, adesc + boff + 2 * k, bdesc + boff + 2 * k, ptx::idesc_f8(BM, BN) | a_fmt,
+                               acc | k);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                ptx::tc_mma_bf16(d_tmem, adesc + boff + 2 * k, bdesc + boff + 2 * k, ptx::idesc_bf16(BM, BN), acc | k);
+            }
+          }
         }
         if (S::PAIR)
           ptx::tc_commit_pair(&s.empty[stage]);  // frees the stage in both CTAs
