@@ -579,15 +579,29 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
           const int nsub = min(S::KSUB, tl.nk - kb);
           for (int j = 0; j < nsub; ++j) {
             const uint64_t boff = soff + static_cast<uint64_t>(j * (S::BLOCK_BYTES >> 4));
-            const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * (stage * S::KSUB + j);
-            const uint32_t sfb_t = sfa_t + 4;
-            ptx::tc_cp_32x128b_warpx4_pair(sfa_t, sfadesc0 + boff);
+            const uint32_t acc = ((kb + j) != 0) ? 1u : 0u;  // the tile's first block overwrites D
+            if (MX) {
+              const uint32_t sfa_t = tmem + S::SF_TMEM_COL + S::SF_COLS * (stage * S::KSUB + j);
+              const uint32_t sfb_t = sfa_t + 4;
+              ptx::tc_cp_32x128b_warpx4_pair(sfa_t, sfadesc0 + boff);
 #pragma unroll
-            for (int i = 0; i < BN / 128; ++i) ptx::tc_cp_32x128b_warpx4_pair(sfb_t + 4 * i, sfbdesc0 + boff + 32 * i);
+              for (int i = 0; i < BN / 128; ++i)
+                ptx::tc_cp_32x128b_warpx4_pair(sfb_t + 4 * i, sfbdesc0 + boff + 32 * i);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              ptx::tc_mma_mxf8_pair(d_tmem, adesc0 + boff + 2 * k, bdesc0 + boff + 2 * k,
-                                    ptx::idesc_mxf8(2 * BM, BN, k, k) | a_fmt, sfa_t, sfb_t, ((kb + j) | k) != 0);
+              for (int k = 0; k < 4; ++k)
+                ptx::tc_mma_mxf8_pair(d_tmem, adesc0 + boff + 2 * k, bdesc0 + boff + 2 * k,
+                                      ptx::idesc_mxf8(2 * BM, BN, k, k) | a_fmt, sfa_t, sfb_t, acc | k);
+            } else if (g.fp8) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                ptx::tc_mma_f8_pair(d_tmem, adesc0 + boff + 2 * k, bdesc0 + boff + 2 * k,
+                                    ptx::idesc_f8(2 * BM, BN) | a_fmt, acc | k);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                ptx::tc_mma_bf16_pair(d_tmem, adesc0 + boff + 2 * k, bdesc0 + boff + 2 * k, ptx::idesc_bf16(2 * BM, BN),
+                                      acc | k);
+            }
           }
         } else {
           const int nsub = min(S::KSUB, tl.nk - kb);
@@ -995,7 +1009,7 @@ cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
 
 // Rows of B one CTA loads per stage (its tensor-map box): the tile's N, or half of it for CTA pairs.
 int gemm_b_box_rows(bool mx, int epi) {
-  if (mx && epi == EPI_STORE) return ShapeStorePair::BN / 2;
+  if (epi == EPI_STORE) return ShapeStorePair::BN / 2;
   return gemm_tile_n(epi);
 }
 
@@ -1014,7 +1028,7 @@ cudaError_t launch_grouped_gemm(const GemmArgs& args, bool mx, int epi, int num_
     if (args.epi.h_q) return launch_t<true, EPI_DSWIGLU, ShapeDswigluG>(args, num_sms, st);
     return launch_t<true, EPI_DSWIGLU, ShapeDswiglu>(args, num_sms, st);
   }
-  if (epi == EPI_STORE) return launch_t<false, EPI_STORE, ShapeStore>(args, num_sms, st);
+  if (epi == EPI_STORE) return launch_t<false, EPI_STORE, ShapeStorePair>(args, num_sms, st);
   if (epi == EPI_SWIGLU) return launch_t<false, EPI_SWIGLU, ShapeSwiglu>(args, num_sms, st);
   if (epi == EPI_FUSED_FWD) return launch_t<false, EPI_FUSED_FWD, ShapeSwiglu>(args, num_sms, st);
   return launch_t<false, EPI_DSWIGLU, ShapeDswiglu>(args, num_sms, st);
