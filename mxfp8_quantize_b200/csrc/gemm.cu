@@ -84,10 +84,9 @@ struct Shape {
   static_assert(EPI_WARPS % 4 == 0 && 32 % PASS == 0 && (LEAD == 4 || LEAD == 2), "thread layout");
   static_assert(!PAIR || (NBUF == 1 && !HTILE && LEAD == 4), "pair instances: one accumulator, no h tile");
 };
-using ShapeStore = Shape<256, 1, 4, false, 8, 16>;    // plain bf16-store epilogues
-// MXFP8 store GEMMs on CTA pairs: 256 x 256 tiles, each CTA streaming 128 rows of A and 128 of B per
-// stage (two thirds of the single-CTA bytes per MMA), six stages deep
-// (stages of two 128-byte K blocks each: one barrier round trip per two blocks)
+// the store GEMMs (all precisions) on CTA pairs: 256 x 256 tiles, each CTA streaming 128 rows of A
+// and 128 of B per K block (two thirds of the single-CTA bytes per MMA), three stages of two K
+// blocks (one barrier round trip per two blocks)
 using ShapeStorePair = Shape<256, 1, 3, false, 8, 16, false, 4, true, 2>;
 // (the gate_up + ScaledSwiGLU kernel stays on single CTAs: on pairs each tile waits for the slower
 // of two heavy epilogues, and it measured 5% slower)
@@ -995,10 +994,18 @@ cudaError_t launch_t(const GemmArgs& args, int num_sms, cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+    // the occupancy query once per device (a host call of some microseconds)
+    static int resident[64] = {};
+    int dev = 0;
+    e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    int clusters = (dev >= 0 && dev < 64) ? resident[dev] : 0;
+    if (clusters < 1) {
+      e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+      if (e != cudaSuccess) return e;
+      if (clusters < 1) return cudaErrorInvalidConfiguration;
+      if (dev >= 0 && dev < 64) resident[dev] = clusters;
+    }
     cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min(clusters, num_sms / 2)));
     return cudaLaunchKernelEx(&cfg, kern, args);
   }
@@ -1014,7 +1021,7 @@ int gemm_b_box_rows(bool mx, int epi) {
 }
 
 int gemm_tile_n(int epi) {
-  return epi == EPI_STORE ? ShapeStore::BN
+  return epi == EPI_STORE ? ShapeStorePair::BN
                           : ((epi == EPI_SWIGLU || epi == EPI_FUSED_FWD) ? ShapeSwiglu::BN : ShapeDswiglu::BN);
 }
 
