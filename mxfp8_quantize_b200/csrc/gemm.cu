@@ -28,6 +28,7 @@
 // and MMAs already issued are waited for before TMEM is freed.
 #include <cuda_fp16.h>
 #include <algorithm>
+#include <type_traits>
 #include <cuda_fp8.h>
 
 #include "gemm.cuh"
@@ -929,14 +930,23 @@ __global__ void __launch_bounds__(S::NUM_THREADS, 1) grouped_gemm_kernel(const _
             }
           }
           if (MX) {
-            uint32_t sb = quant32_store(dg, ep.q_row + row * f2 + j, ep.scale_floor, ep.grad_e5m2);
-            ep.s_row[sf_mma_offset(row, j / 32, f2 / 32)] = static_cast<uint8_t>(sb);
-            sb = quant32_store(du, ep.q_row + row * f2 + f + j, ep.scale_floor, ep.grad_e5m2);
-            ep.s_row[sf_mma_offset(row, (f + j) / 32, f2 / 32)] = static_cast<uint8_t>(sb);
-            colwise_mx<S::PASS>(dg, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
-                                ep.cap / 32, ep.scale_floor, ep.grad_e5m2);
-            colwise_mx<S::PASS>(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j,
-                                row_w / 32, ep.cap / 32, ep.scale_floor, ep.grad_e5m2);
+            // the gradient's element format as a constant inside each branch: one conversion
+            // instruction per pair of values instead of both formats' and a select
+            auto requant = [&](auto e5) {
+              constexpr int E5 = decltype(e5)::value;
+              uint32_t sb = quant32_store(dg, ep.q_row + row * f2 + j, ep.scale_floor, E5);
+              ep.s_row[sf_mma_offset(row, j / 32, f2 / 32)] = static_cast<uint8_t>(sb);
+              sb = quant32_store(du, ep.q_row + row * f2 + f + j, ep.scale_floor, E5);
+              ep.s_row[sf_mma_offset(row, (f + j) / 32, f2 / 32)] = static_cast<uint8_t>(sb);
+              colwise_mx<S::PASS>(dg, stage_buf, ep.q_colT + j * ep.cap + row_w, ep.cap, ep.s_colT, j, row_w / 32,
+                                  ep.cap / 32, ep.scale_floor, E5);
+              colwise_mx<S::PASS>(du, stage_buf, ep.q_colT + (f + j) * ep.cap + row_w, ep.cap, ep.s_colT, f + j,
+                                  row_w / 32, ep.cap / 32, ep.scale_floor, E5);
+            };
+            if (ep.grad_e5m2)
+              requant(std::integral_constant<int, 1>{});
+            else
+              requant(std::integral_constant<int, 0>{});
           } else {
             bf16* d0 = ep.o_row + row * f2 + j;
             bf16* d1 = d0 + f;
